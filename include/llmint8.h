@@ -1,0 +1,152 @@
+/*
+ * llmint8.h - C ABI of the B200 (sm_100a) LLM.int8() mixed-precision decomposed linear layer
+ *
+ *   Y[M, N] = X[M, K] . W^T,  W stored as int8 CB[N, K] + fp32 per-output-channel absmax SCB[N]
+ *
+ * The method (LLM.int8(), Dettmers et al.): split the feature columns of X into "outlier"
+ * columns (some entry with |x| >= threshold, default 6) and regular columns; multiply the
+ * outlier part in fp16 against the matching fp16 weights; quantize the regular part
+ * vector-wise (one absmax per row of X, one per output channel of W), multiply in int8 with
+ * int32 accumulation, dequantize by the outer product of the two absmax vectors / 127^2 and
+ * add the two parts in fp16.  Sources: "A gentle introduction to 8-bit matrix multiplication
+ * for transformers at scale" (Hugging Face blog, zh translation), sections 模型量化介绍,
+ * LLM.int8() 温和总结, MatMul 内部 and 用法; "LLM.int8(): 8-Bit Matrix Multiplication for
+ * Transformers at Scale" (azimuth.plus summary), sections الابتكار الأول, الابتكار الثاني and
+ * الصورة الكاملة.
+ *
+ * Conventions for every call
+ *   - fp16 tensors are IEEE binary16 bit patterns (uint16_t); all tensors are dense and
+ *     row-major (last index contiguous).
+ *   - Every tensor pointer is a DEVICE pointer (cudaMalloc / torch CUDA memory) on the
+ *     current device and 16-byte aligned.  The caller owns every buffer; the library never
+ *     allocates or frees device memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are asynchronous
+ *     on that stream: the returned status covers argument checks and launch errors only.
+ *     Conditions found on the device (outlier capacity exceeded, a bounded wait that timed
+ *     out) are written to the status word of the workspace; read them with
+ *     llmint8_device_status().  Each call that takes a workspace overwrites that word.
+ *   - Shapes: M >= 1; K and N are multiples of 16 and >= 16; K <= 131072 (so that
+ *     |C| <= K * 127^2 < 2^31).  Violations return LLMINT8_ERR_UNSUPPORTED_SHAPE.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef LLMINT8_H
+#define LLMINT8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LLMINT8_API __attribute__((visibility("default")))
+#else
+#define LLMINT8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LLMINT8_OK = 0,
+    LLMINT8_ERR_INVALID_ARG = 1,         /* null or misaligned pointer, NaN threshold, ... */
+    LLMINT8_ERR_UNSUPPORTED_SHAPE = 2,   /* shape outside the rules above */
+    LLMINT8_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the matching *_workspace_size() */
+    LLMINT8_ERR_OUTLIER_CAPACITY = 4,    /* (device) more outlier columns than the capacity */
+    LLMINT8_ERR_TIMEOUT = 5,             /* (device) a bounded wait in a kernel gave up */
+    LLMINT8_ERR_CUDA = 6                 /* a CUDA runtime call or launch failed */
+} llmint8_status;
+
+/*
+ * Weight quantization, once per layer ("weights are quantized by column" of the logical
+ * K x N weight = per output channel; blog section MatMul 内部; CB / SCB of section 用法).
+ *   W   fp16 [N, K]  input, nn.Linear layout (row n = output channel n).
+ *   CB  int8 [N, K]  output: CB[n,k] = round_half_even(fl32(W[n,k] * fl32(127 / SCB[n]))).
+ *   SCB fp32 [N]     output: SCB[n] = max_k |W[n,k]| (0 gives an all-zero row).
+ * Pure function of W: calling it twice gives identical bytes.
+ */
+LLMINT8_API llmint8_status llmint8_quantize_weight_colwise(const uint16_t *W, int64_t N, int64_t K,
+                                               int8_t *CB, float *SCB, void *stream);
+
+/*
+ * Outlier-column detection and row-wise quantization of the activations (the first
+ * steps of the method: outlier features are the columns of the hidden state holding a
+ * value of magnitude >= threshold; hidden states are quantized by row).
+ *   X           fp16 [M, K] input.
+ *   threshold   |x| >= threshold marks column j an outlier; +inf allowed (no outliers),
+ *               <= 0 marks every column; NaN -> LLMINT8_ERR_INVALID_ARG.
+ *   Xq          int8 [M, K] output; outlier columns hold 0.
+ *   SCA         fp32 [M] output: absmax of row i over the regular columns (0 if none / all 0).
+ *   outlier_idx int32 [cap] output: the outlier columns in ascending order (first `cap`).
+ *   n_outliers  int32 [1] output (device): the true number of outlier columns.
+ *   cap         capacity of outlier_idx (0 <= cap <= K).  n_outliers > cap sets the device
+ *               status LLMINT8_ERR_OUTLIER_CAPACITY (Xq and SCA stay exact).
+ *   ws          device workspace of llmint8_quantize_workspace_size(M, K) bytes.
+ */
+LLMINT8_API llmint8_status llmint8_quantize_rows_and_find_outliers(const uint16_t *X, int64_t M, int64_t K,
+                                                       float threshold, int8_t *Xq, float *SCA,
+                                                       int32_t *outlier_idx, int32_t *n_outliers,
+                                                       int64_t cap, void *ws, size_t ws_bytes,
+                                                       void *stream);
+
+LLMINT8_API size_t llmint8_quantize_workspace_size(int64_t M, int64_t K);
+
+/*
+ * The decomposed linear layer (the whole method: outlier columns -> fp16 product against
+ * the matching fp16 weight rows; the rest -> vector-wise int8 product with int32
+ * accumulation, dequantized by the outer product SCA_i * SCB_n / 127^2; the two summed
+ * into the fp16 output).
+ *   X       fp16 [M, K] input activations.
+ *   CB, SCB int8 [N, K], fp32 [N] from llmint8_quantize_weight_colwise.
+ *   bias    fp16 [N] or NULL.
+ *   W_fp16  fp16 [N, K] or NULL.  NULL (inference, weights kept only in int8): the fp16
+ *           weights of the outlier columns are fp16(fl32(fl32(CB * SCB) / 127)).
+ *           Non-NULL: the original fp16 weights are used for the outlier columns.
+ *   threshold   as in llmint8_quantize_rows_and_find_outliers.
+ *   max_outliers capacity for outlier columns, 0 <= max_outliers <= K; it sizes the
+ *           workspace.  More outlier columns than this sets LLMINT8_ERR_OUTLIER_CAPACITY in
+ *           the device status (the output is then incomplete but memory stays in bounds).
+ *   Y       fp16 [M, N] output: fp16(C*SCA_i*SCB_n/127^2 + sum_{j in O} X[i,j]*W_o[n,j] + bias_n),
+ *           evaluated in fp32 with int32 C.
+ *   ws      device workspace of llmint8_linear_workspace_size(M, N, K, max_outliers) bytes.
+ *   C_debug int32 [M, N] or NULL: when given, also receives the exact int8 accumulators C.
+ */
+LLMINT8_API llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
+                              const float *SCB, int64_t N, const uint16_t *bias,
+                              const uint16_t *W_fp16, float threshold, int64_t max_outliers,
+                              uint16_t *Y, void *ws, size_t ws_bytes, void *stream,
+                              int32_t *C_debug);
+
+LLMINT8_API size_t llmint8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t max_outliers);
+
+/*
+ * Weight dequantization W_out[n,k] = fp16(fl32(fl32(CB[n,k] * SCB[n]) / 127)) (blog
+ * section 用法: the fp16 weights are recovered as (CB * SCB) / 127).
+ */
+LLMINT8_API llmint8_status llmint8_dequant(const int8_t *CB, const float *SCB, int64_t N, int64_t K,
+                               uint16_t *W_out, void *stream);
+
+/*
+ * Synchronizes `stream` and returns the device status word of a workspace used by the
+ * last llmint8_linear / llmint8_quantize_rows_and_find_outliers call on it
+ * (LLMINT8_OK, LLMINT8_ERR_OUTLIER_CAPACITY or LLMINT8_ERR_TIMEOUT), or LLMINT8_ERR_CUDA.
+ */
+LLMINT8_API llmint8_status llmint8_device_status(const void *ws, void *stream);
+
+/* Also returns the device outlier count of a llmint8_linear workspace (synchronizes). */
+LLMINT8_API llmint8_status llmint8_workspace_outlier_count(const void *ws, void *stream, int32_t *count);
+
+/* Static English text for a status code. */
+LLMINT8_API const char *llmint8_status_string(llmint8_status status);
+
+/*
+ * Upper bound, in nanoseconds, of every wait inside the GEMM kernels of later calls
+ * (process-wide; default 1e9).  A wait that runs out records LLMINT8_ERR_TIMEOUT in the
+ * device status and the kernel winds down and returns.  Tests set a tiny bound to
+ * exercise that path.  ns == 0 restores the default.
+ */
+LLMINT8_API llmint8_status llmint8_set_wait_timeout_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLMINT8_H */

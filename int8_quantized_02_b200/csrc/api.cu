@@ -1,0 +1,233 @@
+// C ABI of the LLM.int8() layer: argument checks, workspace layout and kernel launches.
+// Declarations and the contract of every entry point are in include/llmint8.h.
+#include <math.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace llmint8;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+bool shape_ok_mk(int64_t M, int64_t K) {
+    return M >= 1 && M <= (int64_t)INT32_MAX && K >= 16 && K % 16 == 0 && K <= 131072;
+}
+bool shape_ok_n(int64_t N) { return N >= 16 && N % 16 == 0 && N <= (int64_t)INT32_MAX; }
+
+// Workspace of llmint8_linear, every region 256-byte aligned.
+struct LinearLayout {
+    ScanPlan plan;
+    int64_t cap = 0, pitch = 0;
+    size_t partial = 0, bitmap = 0, idx = 0, sca = 0, xq = 0, xo = 0, wo = 0, total = 0;
+};
+
+LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t cap) {
+    LinearLayout L;
+    L.plan = scan_plan(M, K);
+    L.cap = cap;
+    L.pitch = align_up(cap, 64);
+    size_t off = sizeof(WsHeader);
+    auto take = [&](size_t bytes) {
+        size_t at = off;
+        off = (size_t)align_up((int64_t)(off + bytes), 256);
+        return at;
+    };
+    L.partial = take((size_t)(L.plan.splits * L.plan.nwords) * 4);
+    L.bitmap = take((size_t)L.plan.nwords * 4);
+    L.idx = take((size_t)std::max<int64_t>(cap, 1) * 4);
+    L.sca = take((size_t)M * 4);
+    L.xq = take((size_t)(M * K));
+    L.xo = take((size_t)(M * L.pitch) * 2);
+    L.wo = take((size_t)(N * L.pitch) * 2);
+    L.total = off;
+    return L;
+}
+
+struct QuantLayout {
+    ScanPlan plan;
+    size_t partial = 0, bitmap = 0, total = 0;
+};
+
+QuantLayout quant_layout(int64_t M, int64_t K) {
+    QuantLayout L;
+    L.plan = scan_plan(M, K);
+    size_t off = sizeof(WsHeader);
+    L.partial = off;
+    off = (size_t)align_up((int64_t)(off + (size_t)(L.plan.splits * L.plan.nwords) * 4), 256);
+    L.bitmap = off;
+    off = (size_t)align_up((int64_t)(off + (size_t)L.plan.nwords * 4), 256);
+    L.total = off;
+    return L;
+}
+
+template <class T>
+T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+llmint8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *llmint8_status_string(llmint8_status s) {
+    switch (s) {
+        case LLMINT8_OK: return "ok";
+        case LLMINT8_ERR_INVALID_ARG: return "invalid argument";
+        case LLMINT8_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case LLMINT8_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case LLMINT8_ERR_OUTLIER_CAPACITY: return "more outlier columns than the capacity";
+        case LLMINT8_ERR_TIMEOUT: return "a bounded wait in a kernel timed out";
+        case LLMINT8_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+llmint8_status llmint8_set_wait_timeout_ns(uint64_t ns) {
+    g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
+    return LLMINT8_OK;
+}
+
+size_t llmint8_quantize_workspace_size(int64_t M, int64_t K) {
+    if (!shape_ok_mk(M, K)) return 0;
+    return quant_layout(M, K).total;
+}
+
+size_t llmint8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t max_outliers) {
+    if (!shape_ok_mk(M, K) || !shape_ok_n(N) || max_outliers < 0 || max_outliers > K) return 0;
+    return linear_layout(M, N, K, max_outliers).total;
+}
+
+llmint8_status llmint8_quantize_weight_colwise(const uint16_t *W, int64_t N, int64_t K,
+                                               int8_t *CB, float *SCB, void *stream) {
+    if (!W || !CB || !SCB) return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(CB) || !aligned4(SCB)) return LLMINT8_ERR_INVALID_ARG;
+    if (!shape_ok_mk(N, K)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    return from_cuda(launch_quantize_weight(reinterpret_cast<const __half *>(W), N, K, CB, SCB,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+llmint8_status llmint8_dequant(const int8_t *CB, const float *SCB, int64_t N, int64_t K,
+                               uint16_t *W_out, void *stream) {
+    if (!CB || !SCB || !W_out) return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(CB) || !aligned16(W_out) || !aligned4(SCB)) return LLMINT8_ERR_INVALID_ARG;
+    if (!shape_ok_mk(N, K)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    return from_cuda(launch_dequant(CB, SCB, N, K, reinterpret_cast<__half *>(W_out),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+llmint8_status llmint8_quantize_rows_and_find_outliers(const uint16_t *X, int64_t M, int64_t K,
+                                                       float threshold, int8_t *Xq, float *SCA,
+                                                       int32_t *outlier_idx, int32_t *n_outliers,
+                                                       int64_t cap, void *ws, size_t ws_bytes,
+                                                       void *stream) {
+    if (!X || !Xq || !SCA || !n_outliers || !ws || (cap > 0 && !outlier_idx))
+        return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(Xq) || !aligned4(SCA) || !aligned4(n_outliers) ||
+        !aligned16(ws) || (outlier_idx && !aligned4(outlier_idx)))
+        return LLMINT8_ERR_INVALID_ARG;
+    if (isnan(threshold)) return LLMINT8_ERR_INVALID_ARG;
+    if (!shape_ok_mk(M, K)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    if (cap < 0 || cap > K) return LLMINT8_ERR_INVALID_ARG;
+    const QuantLayout L = quant_layout(M, K);
+    if (ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    WsHeader *h = at<WsHeader>(ws, 0);
+    const __half *Xh = reinterpret_cast<const __half *>(X);
+    uint32_t *bitmap = at<uint32_t>(ws, L.bitmap);
+    cudaError_t e = launch_outlier_detect(Xh, M, K, threshold, L.plan, at<uint32_t>(ws, L.partial),
+                                          bitmap, outlier_idx, cap, n_outliers, &h->status, s);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    return from_cuda(launch_quantize_rows(Xh, M, K, bitmap, outlier_idx, n_outliers, cap, 0, Xq,
+                                          SCA, nullptr, s));
+}
+
+llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
+                              const float *SCB, int64_t N, const uint16_t *bias,
+                              const uint16_t *W_fp16, float threshold, int64_t max_outliers,
+                              uint16_t *Y, void *ws, size_t ws_bytes, void *stream,
+                              int32_t *C_debug) {
+    if (!X || !CB || !SCB || !Y || !ws) return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(CB) || !aligned16(SCB) || !aligned16(Y) || !aligned16(ws) ||
+        (bias && !aligned16(bias)) || (W_fp16 && !aligned16(W_fp16)) ||
+        (C_debug && !aligned16(C_debug)))
+        return LLMINT8_ERR_INVALID_ARG;
+    if (isnan(threshold)) return LLMINT8_ERR_INVALID_ARG;
+    if (!shape_ok_mk(M, K) || !shape_ok_n(N)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    if (max_outliers < 0 || max_outliers > K) return LLMINT8_ERR_INVALID_ARG;
+    const LinearLayout L = linear_layout(M, N, K, max_outliers);
+    if (ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    WsHeader *h = at<WsHeader>(ws, 0);
+    const __half *Xh = reinterpret_cast<const __half *>(X);
+    uint32_t *bitmap = at<uint32_t>(ws, L.bitmap);
+    int32_t *idx = at<int32_t>(ws, L.idx);
+    float *SCA = at<float>(ws, L.sca);
+    int8_t *Xq = at<int8_t>(ws, L.xq);
+    __half *Xo = at<__half>(ws, L.xo);
+    __half *Wo = at<__half>(ws, L.wo);
+
+    cudaError_t e = launch_outlier_detect(Xh, M, K, threshold, L.plan, at<uint32_t>(ws, L.partial),
+                                          bitmap, idx, max_outliers, &h->n_outliers, &h->status,
+                                          s);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    e = launch_quantize_rows(Xh, M, K, bitmap, idx, &h->n_outliers, max_outliers, L.pitch, Xq, SCA,
+                             max_outliers > 0 ? Xo : nullptr, s);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (max_outliers > 0) {
+        e = launch_gather_outlier_w(CB, SCB, reinterpret_cast<const __half *>(W_fp16), N, K, idx,
+                                    &h->n_outliers, max_outliers, L.pitch, Wo, s);
+        if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    }
+    GemmLaunch g;
+    g.Xq = Xq;
+    g.CB = CB;
+    g.Xo = Xo;
+    g.Wo = Wo;
+    g.pitch = L.pitch;
+    g.count = &h->n_outliers;
+    g.cap = max_outliers;
+    g.SCA = SCA;
+    g.SCB = SCB;
+    g.bias = reinterpret_cast<const __half *>(bias);
+    g.Y = reinterpret_cast<__half *>(Y);
+    g.C_debug = C_debug;
+    g.status = &h->status;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.timeout_ns = g_timeout_ns.load();
+    return from_cuda(launch_gemm(g, s));
+}
+
+llmint8_status llmint8_device_status(const void *ws, void *stream) {
+    if (!ws) return LLMINT8_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    uint32_t st = 0;
+    if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    return static_cast<llmint8_status>(st);
+}
+
+llmint8_status llmint8_workspace_outlier_count(const void *ws, void *stream, int32_t *count) {
+    if (!ws || !count) return LLMINT8_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    const WsHeader *h = static_cast<const WsHeader *>(ws);
+    if (cudaMemcpy(count, &h->n_outliers, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    return LLMINT8_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,396 @@
+// The LLM.int8() product on the 5th-generation tensor cores of sm_100a.
+//
+// One persistent CTA per SM computes 128 x 256 output tiles of
+//     Y = fp16( C * SCA_i * SCB_n / 127^2 + P + bias_n ),
+//     C = Xq . CB^T    (int8 x int8 -> int32, tcgen05.mma kind::i8, exact)
+//     P = Xo . Wo^T    (fp16 x fp16 -> fp32, tcgen05.mma kind::f16, the outlier columns)
+// which is the decomposition of the LLM.int8() summary (sections الابتكار الثاني and
+// الصورة الكاملة) and of the blog's three steps (section LLM.int8() 温和总结): the regular part
+// goes through the int8 product dequantized by the outer product of the row and column
+// absmax vectors, the outlier part through a 16-bit product, and the two are summed in the
+// epilogue before the single rounding to fp16.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: k-blocks of Xq / CB (128 B of K each), then of Xo / Wo
+//               (64 fp16 of K each) - both fill the same 48 KB shared-memory stages;
+//   warp 1      TMEM allocator and MMA issuer (one thread);
+//   warps 2..5  epilogue: TMEM -> registers -> dequantize, add P and bias -> fp16 -> global.
+// TMEM (512 columns): with no outlier columns the int32 accumulator is double-buffered
+// (2 x 256 columns) so the epilogue of a tile overlaps the main loop of the next; with
+// outlier columns the second half holds the fp32 outlier accumulator P instead.
+// Every wait is bounded (BoundedWait); a timeout records LLMINT8_ERR_TIMEOUT, drains the
+// copies and MMAs in flight, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace llmint8 {
+
+namespace {
+
+constexpr int BM = 128;                 // tile rows (M)
+constexpr int BN = 256;                 // tile columns (N)
+constexpr int BKB = 128;                // bytes of K per stage row (128 int8 or 64 fp16)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BKB;       // 16 KB
+constexpr int B_BYTES = BN * BKB;       // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+
+struct Tail {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + (int)sizeof(Tail);
+
+struct Args {
+    const int32_t *count;
+    int64_t cap;
+    const float *SCA;
+    const float *SCB;
+    const __half *bias;
+    __half *Y;
+    int32_t *C_debug;
+    uint32_t *status;
+    int M, N, K;
+    int num_kb;
+    int tiles_m, tiles_n;
+    uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmXo,
+                    const __grid_constant__ CUtensorMap tmWo, const Args a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Tail *tail = reinterpret_cast<Tail *>(smem + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // Outlier configuration of this call (uniform over the grid).
+    const int n_out = (int)min((int64_t)*a.count, a.cap);
+    const int nob = (n_out + 63) / 64;                 // fp16 k-blocks of 64 columns
+    const bool all_outliers = n_out >= a.K;            // then C == 0: skip the int8 blocks
+    const int nkb = all_outliers ? 0 : a.num_kb;
+    const int acc_stages = nob > 0 ? 1 : 2;
+    const int total_tiles = a.tiles_m * a.tiles_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_addr(&tail->full[s]), 1);
+            mbar_init(smem_addr(&tail->empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_addr(&tail->acc_full[s]), 1);
+            mbar_init(smem_addr(&tail->acc_empty[s]), 4);
+        }
+        mbar_init(smem_addr(&tail->mma_done), 1);
+        tail->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        if (nob > 0) {
+            tma_prefetch_desc(&tmXo);
+            tma_prefetch_desc(&tmWo);
+        }
+    }
+    if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tail->tmem_base;
+    const BoundedWait wait{&tail->abort_flag, a.status, a.timeout_ns};
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer ----
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t used = 0, last_parity = 0;   // per stage: issued at least once / parity
+            for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+                const int m0 = (tile % a.tiles_m) * BM;
+                const int n0 = (tile / a.tiles_m) * BN;
+                for (int kb = 0; kb < nkb + nob; ++kb) {
+                    if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
+                    const uint32_t full = smem_addr(&tail->full[stage]);
+                    const uint32_t sa = smem_addr(smem + stage * STAGE_BYTES);
+                    mbar_arrive_expect_tx(full, STAGE_BYTES);
+                    if (kb < nkb) {
+                        tma_load_2d(sa, &tmA, kb * BKB, m0, full);
+                        tma_load_2d(sa + A_BYTES, &tmB, kb * BKB, n0, full);
+                    } else {
+                        const int x = (kb - nkb) * (BKB / 2);
+                        tma_load_2d(sa, &tmXo, x, m0, full);
+                        tma_load_2d(sa + A_BYTES, &tmWo, x, n0, full);
+                    }
+                    used |= 1u << stage;
+                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+        drain:
+            // wait for every copy this thread issued to land before the CTA may exit
+            for (int s = 0; s < STAGES; ++s)
+                if (used & (1u << s))
+                    drain_wait(smem_addr(&tail->full[s]), (last_parity >> s) & 1u, a.status);
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------------------- MMA issuer ----
+        if (lane == 0) {
+            const uint32_t id_i8 = idesc_i8(BM, BN);
+            const uint32_t id_f16 = idesc_f16(BM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+                if (!wait(smem_addr(&tail->acc_empty[acc]), acc_phase ^ 1)) break;
+                tc_fence_after();
+                const uint32_t d_i32 = tmem + (uint32_t)(acc * 256);
+                const uint32_t d_f32 = tmem + 256u;
+                bool ok = true;
+                for (int kb = 0; kb < nkb + nob; ++kb) {
+                    if (!wait(smem_addr(&tail->full[stage]), phase)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_addr(smem + stage * STAGE_BYTES);
+                    const uint32_t sb = sa + A_BYTES;
+                    if (kb < nkb) {
+#pragma unroll
+                        for (int k = 0; k < BKB / 32; ++k)
+                            mma_i8(d_i32, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), id_i8,
+                                   (kb | k) != 0);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < BKB / 32; ++k)
+                            mma_f16(d_f32, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k),
+                                    id_f16, ((kb - nkb) | k) != 0);
+                    }
+                    tc_commit(smem_addr(&tail->empty[stage]));   // frees the stage
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(smem_addr(&tail->acc_full[acc]));      // accumulators ready
+                if (++acc == acc_stages) {
+                    acc = 0;
+                    acc_phase ^= 1;
+                }
+            }
+            // every MMA issued by this thread has completed once mma_done arrives
+            tc_commit(smem_addr(&tail->mma_done));
+            drain_wait(smem_addr(&tail->mma_done), 0, a.status);
+        }
+    } else {
+        // ----------------------------------------------------------------- epilogue ----
+        const int q = warp & 3;                        // TMEM lane quadrant of this warp
+        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+            int ok = 0;
+            if (lane == 0) ok = wait(smem_addr(&tail->acc_full[acc]), acc_phase) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const int m0 = (tile % a.tiles_m) * BM;
+            const int n0 = (tile / a.tiles_m) * BN;
+            const int row = m0 + q * 32 + lane;
+            const bool row_ok = row < a.M;
+            const float rs = row_ok ? a.SCA[row] * (1.0f / 16129.0f) : 0.0f;
+            for (int c = 0; c < BN / 32; ++c) {
+                const int nb = n0 + c * 32;
+                if (nb >= a.N) break;
+                uint32_t ci[32], pf[32];
+                if (nkb > 0) tmem_ld_32x32(tl + (uint32_t)(acc * 256 + c * 32), ci);
+                if (nob > 0) tmem_ld_32x32(tl + (uint32_t)(256 + c * 32), pf);
+                tmem_wait_ld();
+                if (nkb == 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) ci[j] = 0u;
+                }
+                if (nob == 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) pf[j] = 0u;
+                }
+                const int groups = min(32, a.N - nb) / 16;   // 1 or 2 groups of 16 columns
+                if (row_ok) {
+                    __half *yrow = a.Y + (int64_t)row * a.N + nb;
+                    int32_t *crow = a.C_debug ? a.C_debug + (int64_t)row * a.N + nb : nullptr;
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        if (g < groups) {
+                            uint32_t packed[8];
+#pragma unroll
+                            for (int j4 = 0; j4 < 4; ++j4) {
+                                const float4 sb = __ldg(reinterpret_cast<const float4 *>(
+                                    a.SCB + nb + g * 16 + j4 * 4));
+                                float b[4] = {0.f, 0.f, 0.f, 0.f};
+                                if (a.bias) {
+                                    const uint2 bb = __ldg(reinterpret_cast<const uint2 *>(
+                                        a.bias + nb + g * 16 + j4 * 4));
+                                    const float2 b01 = __half22float2(
+                                        *reinterpret_cast<const __half2 *>(&bb.x));
+                                    const float2 b23 = __half22float2(
+                                        *reinterpret_cast<const __half2 *>(&bb.y));
+                                    b[0] = b01.x; b[1] = b01.y; b[2] = b23.x; b[3] = b23.y;
+                                }
+                                const float sbv[4] = {sb.x, sb.y, sb.z, sb.w};
+                                float y[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int j = g * 16 + j4 * 4 + e;
+                                    y[e] = fmaf((float)(int32_t)ci[j], rs * sbv[e],
+                                                __uint_as_float(pf[j]) + b[e]);
+                                }
+                                packed[j4 * 2] = pack_half2(y[0], y[1]);
+                                packed[j4 * 2 + 1] = pack_half2(y[2], y[3]);
+                            }
+                            uint4 *dst = reinterpret_cast<uint4 *>(yrow + g * 16);
+                            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                            if (crow) {
+                                uint4 *cd = reinterpret_cast<uint4 *>(crow + g * 16);
+#pragma unroll
+                                for (int v = 0; v < 4; ++v)
+                                    cd[v] = make_uint4(ci[g * 16 + v * 4], ci[g * 16 + v * 4 + 1],
+                                                       ci[g * 16 + v * 4 + 2],
+                                                       ci[g * 16 + v * 4 + 3]);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&tail->acc_empty[acc]));
+            if (++acc == acc_stages) {
+                acc = 0;
+                acc_phase ^= 1;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// 2-D row-major map over [rows, cols] elements with a (box_cols x box_rows) box, 128 B swizzle.
+bool make_map(CUtensorMap *tm, const void *base, CUtensorMapDataType dt, int elem_bytes,
+              int64_t cols, int64_t rows, int64_t pitch_elems, uint32_t box_cols,
+              uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(pitch_elems * elem_bytes)};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(tm, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    bool attr_set = false;
+};
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s) {
+    static std::mutex mu;
+    static DeviceInfo info[64];
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int sms;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        DeviceInfo &d = info[dev];
+        if (!d.attr_set) {
+            err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+            if (err != cudaSuccess) return err;
+            err = cudaFuncSetAttribute(llmint8_gemm_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+            if (err != cudaSuccess) return err;
+            d.attr_set = true;
+        }
+        sms = d.sms;
+    }
+    CUtensorMap tmA, tmB, tmXo, tmWo;
+    memset(&tmXo, 0, sizeof(tmXo));
+    memset(&tmWo, 0, sizeof(tmWo));
+    bool ok = make_map(&tmA, g.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.K, g.M, g.K, BKB, BM) &&
+              make_map(&tmB, g.CB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.K, g.N, g.K, BKB, BN);
+    if (ok && g.cap > 0)
+        ok = make_map(&tmXo, g.Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, g.pitch, g.M, g.pitch,
+                      BKB / 2, BM) &&
+             make_map(&tmWo, g.Wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, g.pitch, g.N, g.pitch,
+                      BKB / 2, BN);
+    if (!ok) return cudaErrorInvalidValue;
+    Args a;
+    a.count = g.count;
+    a.cap = g.cap;
+    a.SCA = g.SCA;
+    a.SCB = g.SCB;
+    a.bias = g.bias;
+    a.Y = g.Y;
+    a.C_debug = g.C_debug;
+    a.status = g.status;
+    a.M = (int)g.M;
+    a.N = (int)g.N;
+    a.K = (int)g.K;
+    a.num_kb = (int)ceil_div(g.K, BKB);
+    a.tiles_m = (int)ceil_div(g.M, BM);
+    a.tiles_n = (int)ceil_div(g.N, BN);
+    a.timeout_ns = g.timeout_ns;
+    const int tiles = a.tiles_m * a.tiles_n;
+    const int grid = std::min(tiles, sms);
+    llmint8_gemm_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmXo, tmWo, a);
+    return cudaGetLastError();
+}
+
+}  // namespace llmint8

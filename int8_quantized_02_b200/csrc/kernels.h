@@ -1,0 +1,57 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace llmint8 {
+
+// Row-split plan of the outlier scan: the columns are covered by `col_blocks` CTAs of
+// 256 threads x 8 columns, the rows by `splits` ranges of `rows_per_split` rows.
+struct ScanPlan {
+    int64_t col_blocks = 0, splits = 0, rows_per_split = 0, nwords = 0;
+};
+ScanPlan scan_plan(int64_t M, int64_t K);
+
+cudaError_t launch_outlier_detect(const __half *X, int64_t M, int64_t K, float threshold,
+                                  const ScanPlan &plan, uint32_t *partial, uint32_t *bitmap,
+                                  int32_t *idx, int64_t cap, int32_t *count, uint32_t *status,
+                                  cudaStream_t s);
+cudaError_t launch_quantize_rows(const __half *X, int64_t M, int64_t K, const uint32_t *bitmap,
+                                 const int32_t *idx, const int32_t *count, int64_t cap,
+                                 int64_t xo_pitch, int8_t *Xq, float *SCA, __half *Xo,
+                                 cudaStream_t s);
+cudaError_t launch_gather_outlier_w(const int8_t *CB, const float *SCB, const __half *W16,
+                                    int64_t N, int64_t K, const int32_t *idx,
+                                    const int32_t *count, int64_t cap, int64_t pitch, __half *Wo,
+                                    cudaStream_t s);
+cudaError_t launch_quantize_weight(const __half *W, int64_t N, int64_t K, int8_t *CB, float *SCB,
+                                   cudaStream_t s);
+cudaError_t launch_dequant(const int8_t *CB, const float *SCB, int64_t N, int64_t K,
+                           __half *W_out, cudaStream_t s);
+
+// The tcgen05 GEMM with the fused fp16 outlier product and dequantizing epilogue.
+struct GemmLaunch {
+    const int8_t *Xq;        // [M, K]
+    const int8_t *CB;        // [N, K]
+    const __half *Xo;        // [M, pitch]   (may be null when cap == 0)
+    const __half *Wo;        // [N, pitch]
+    int64_t pitch;           // columns of Xo / Wo (multiple of 64)
+    const int32_t *count;    // device outlier count
+    int64_t cap;             // capacity (columns usable in Xo / Wo)
+    const float *SCA;        // [M]
+    const float *SCB;        // [N]
+    const __half *bias;      // [N] or null
+    __half *Y;               // [M, N]
+    int32_t *C_debug;        // [M, N] or null
+    uint32_t *status;
+    int64_t M, N, K;
+    uint64_t timeout_ns;
+};
+cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s);
+
+}  // namespace llmint8

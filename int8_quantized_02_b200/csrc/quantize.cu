@@ -1,0 +1,390 @@
+// Memory-bound kernels of the LLM.int8() layer on sm_100a:
+//   outlier_scan      - per-column "some |x| >= threshold" flags, one bitmap word per 32
+//                       columns and per row split, written without atomics;
+//   outlier_compact   - OR of the row-split bitmaps, ascending index list, count, status;
+//   quantize_rows     - row absmax over the regular columns, absmax quantization to int8
+//                       (outlier columns zeroed) and the compact gather of the fp16 outlier
+//                       columns Xo;
+//   gather_outlier_w  - the fp16 weights of the outlier columns, Wo[n, j];
+//   quantize_weight   - per-output-channel absmax quantization of W (one-time setup);
+//   dequant           - (CB * SCB) / 127 back to fp16.
+// Rounding follows the definition exactly: multiplier = fl32(127 / absmax) (IEEE division),
+// product rounded once to fp32, then round-half-to-even to an integer.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace llmint8 {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]) {
+    const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float2 t = __half22float2(h[e]);
+        f[2 * e] = t.x;
+        f[2 * e + 1] = t.y;
+    }
+}
+
+__device__ __forceinline__ int quant1(float x, float s) {
+    int q = __float2int_rn(__fmul_rn(x, s));
+    return max(-127, min(127, q));
+}
+
+__device__ __forceinline__ uint2 quant8(const float (&f)[8], float s, uint32_t skip_mask) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        int q = ((skip_mask >> e) & 1u) ? 0 : quant1(f[e], s);
+        uint32_t b = (uint32_t)(q & 0xff);
+        if (e < 4) lo |= b << (8 * e);
+        else hi |= b << (8 * (e - 4));
+    }
+    return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ float block_max(float v, float *red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) red[0] = v;
+    }
+    __syncthreads();
+    return red[0];
+}
+
+// grid (ceil(K/8/256), splits); thread = 8 consecutive columns, loops over its row split.
+__global__ void __launch_bounds__(kThreads)
+outlier_scan_kernel(const __half *__restrict__ X, int64_t M, int64_t K, float threshold,
+                    int64_t rows_per_split, uint32_t *__restrict__ partial, int64_t nwords) {
+    const int64_t chunk = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    const int64_t nchunks = K / 8;
+    const int64_t r0 = (int64_t)blockIdx.y * rows_per_split;
+    const int64_t r1 = min(M, r0 + rows_per_split);
+    uint32_t bits = 0;
+    if (chunk < nchunks) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(X) + r0 * nchunks + chunk;
+        int64_t r = r0;
+        for (; r + 4 <= r1; r += 4) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = __ldcs(p + u * nchunks);
+            p += 4 * nchunks;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float f[8];
+                unpack8(v[u], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) bits |= (fabsf(f[e]) >= threshold ? 1u : 0u) << e;
+            }
+        }
+        for (; r < r1; ++r) {
+            float f[8];
+            unpack8(__ldcs(p), f);
+            p += nchunks;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) bits |= (fabsf(f[e]) >= threshold ? 1u : 0u) << e;
+        }
+    }
+    // four neighbouring threads hold the four bytes of one 32-column word
+    uint32_t word = bits << (8 * (threadIdx.x & 3));
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+    if ((threadIdx.x & 3) == 0 && chunk < nchunks)
+        partial[(int64_t)blockIdx.y * nwords + chunk / 4] = word;
+}
+
+// One CTA of 1024 threads: OR over the row splits, popcount, exclusive scan, ascending
+// index list.  Also writes the workspace status word (resetting it for this call).
+constexpr int kCompactThreads = 1024;
+constexpr int kMaxWordsPerThread = 4;   // nwords <= 4096 (K <= 131072)
+
+__global__ void __launch_bounds__(kCompactThreads)
+outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t nwords,
+                       int32_t *__restrict__ idx, int64_t cap, int32_t *__restrict__ count_out,
+                       uint32_t *__restrict__ bitmap_out, uint32_t *__restrict__ status) {
+    __shared__ int warp_tot[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int wpt = (int)ceil_div(nwords, kCompactThreads);
+    const int64_t w0 = (int64_t)tid * wpt;
+    uint32_t w[kMaxWordsPerThread];
+    int cnt = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxWordsPerThread; ++i) {
+        w[i] = 0;
+        const int64_t wi = w0 + i;
+        if (i < wpt && wi < nwords) {
+            uint32_t v = 0;
+            for (int s = 0; s < splits; ++s) v |= partial[(int64_t)s * nwords + wi];
+            w[i] = v;
+            bitmap_out[wi] = v;
+            cnt += __popc(v);
+        }
+    }
+    // block-wide exclusive scan of cnt
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int v = warp_tot[lane];
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int t = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += t;
+        }
+        warp_tot[lane] = x - v;   // exclusive prefix of warp totals
+    }
+    __syncthreads();
+    int pos = warp_tot[warp] + incl - cnt;
+#pragma unroll
+    for (int i = 0; i < kMaxWordsPerThread; ++i) {
+        uint32_t v = w[i];
+        while (v) {
+            const int b = __ffs(v) - 1;
+            v &= v - 1;
+            if (pos < cap) idx[pos] = (int32_t)((w0 + i) * 32 + b);
+            ++pos;
+        }
+    }
+    if (tid == kCompactThreads - 1) {
+        *count_out = pos;
+        *status = (pos > cap) ? (uint32_t)LLMINT8_ERR_OUTLIER_CAPACITY : (uint32_t)LLMINT8_OK;
+    }
+}
+
+// One CTA per row.  Row values stay in registers for K <= 8 * 256 * kCache.
+constexpr int kCache = 8;
+
+__global__ void __launch_bounds__(kThreads)
+quantize_rows_kernel(const __half *__restrict__ X, int64_t K, const uint32_t *__restrict__ bitmap,
+                     const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
+                     int64_t cap, int64_t xo_pitch, int8_t *__restrict__ Xq,
+                     float *__restrict__ SCA, __half *__restrict__ Xo) {
+    __shared__ float red[32];
+    const int64_t row = blockIdx.x;
+    const int64_t nchunks = K / 8;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(X + row * K);
+    uint4 cache[kCache];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kCache; ++i) {
+        const int64_t c = threadIdx.x + (int64_t)i * kThreads;
+        if (c < nchunks) {
+            cache[i] = xr[c];
+            const uint32_t skip = (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu;
+            float f[8];
+            unpack8(cache[i], f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (!((skip >> e) & 1u)) amax = fmaxf(amax, fabsf(f[e]));
+        }
+    }
+    for (int64_t c = threadIdx.x + (int64_t)kCache * kThreads; c < nchunks; c += kThreads) {
+        const uint32_t skip = (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu;
+        float f[8];
+        unpack8(xr[c], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if (!((skip >> e) & 1u)) amax = fmaxf(amax, fabsf(f[e]));
+    }
+    amax = block_max(amax, red);
+    if (threadIdx.x == 0) SCA[row] = amax;
+    const float s = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    uint2 *qr = reinterpret_cast<uint2 *>(Xq + row * K);
+#pragma unroll
+    for (int i = 0; i < kCache; ++i) {
+        const int64_t c = threadIdx.x + (int64_t)i * kThreads;
+        if (c < nchunks) {
+            const uint32_t skip = (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu;
+            float f[8];
+            unpack8(cache[i], f);
+            qr[c] = quant8(f, s, amax > 0.0f ? skip : 0xffu);
+        }
+    }
+    for (int64_t c = threadIdx.x + (int64_t)kCache * kThreads; c < nchunks; c += kThreads) {
+        const uint32_t skip = (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu;
+        float f[8];
+        unpack8(xr[c], f);
+        qr[c] = quant8(f, s, amax > 0.0f ? skip : 0xffu);
+    }
+    if (Xo != nullptr) {
+        const int64_t n_o = min((int64_t)*count, cap);
+        const int64_t n_o64 = align_up(n_o, 64);
+        const __half *x = X + row * K;
+        for (int64_t j = threadIdx.x; j < n_o64; j += kThreads)
+            Xo[row * xo_pitch + j] = j < n_o ? x[idx[j]] : __float2half_rn(0.0f);
+    }
+}
+
+// One warp per output channel n.
+__global__ void __launch_bounds__(kThreads)
+gather_outlier_w_kernel(const int8_t *__restrict__ CB, const float *__restrict__ SCB,
+                        const __half *__restrict__ W16, int64_t N, int64_t K,
+                        const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
+                        int64_t cap, int64_t pitch, __half *__restrict__ Wo) {
+    const int64_t n = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (n >= N) return;
+    const int64_t n_o = min((int64_t)*count, cap);
+    const int64_t n_o64 = align_up(n_o, 64);
+    const float scb = SCB[n];
+    for (int64_t j = lane; j < n_o64; j += 32) {
+        __half v = __float2half_rn(0.0f);
+        if (j < n_o) {
+            const int64_t col = idx[j];
+            if (W16 != nullptr)
+                v = W16[n * K + col];
+            else
+                v = __float2half_rn(__fdiv_rn(__fmul_rn((float)CB[n * K + col], scb), 127.0f));
+        }
+        Wo[n * pitch + j] = v;
+    }
+}
+
+// One CTA per output channel n.
+__global__ void __launch_bounds__(kThreads)
+quantize_weight_kernel(const __half *__restrict__ W, int64_t K, int8_t *__restrict__ CB,
+                       float *__restrict__ SCB) {
+    __shared__ float red[32];
+    const int64_t n = blockIdx.x;
+    const int64_t nchunks = K / 8;
+    const uint4 *wr = reinterpret_cast<const uint4 *>(W + n * K);
+    uint4 cache[kCache];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kCache; ++i) {
+        const int64_t c = threadIdx.x + (int64_t)i * kThreads;
+        if (c < nchunks) {
+            cache[i] = wr[c];
+            float f[8];
+            unpack8(cache[i], f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+        }
+    }
+    for (int64_t c = threadIdx.x + (int64_t)kCache * kThreads; c < nchunks; c += kThreads) {
+        float f[8];
+        unpack8(wr[c], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+    }
+    amax = block_max(amax, red);
+    if (threadIdx.x == 0) SCB[n] = amax;
+    const float s = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    const uint32_t skip = amax > 0.0f ? 0u : 0xffu;
+    uint2 *qr = reinterpret_cast<uint2 *>(CB + n * K);
+#pragma unroll
+    for (int i = 0; i < kCache; ++i) {
+        const int64_t c = threadIdx.x + (int64_t)i * kThreads;
+        if (c < nchunks) {
+            float f[8];
+            unpack8(cache[i], f);
+            qr[c] = quant8(f, s, skip);
+        }
+    }
+    for (int64_t c = threadIdx.x + (int64_t)kCache * kThreads; c < nchunks; c += kThreads) {
+        float f[8];
+        unpack8(wr[c], f);
+        qr[c] = quant8(f, s, skip);
+    }
+}
+
+// Grid-stride over 8-element chunks.
+__global__ void __launch_bounds__(kThreads)
+dequant_kernel(const int8_t *__restrict__ CB, const float *__restrict__ SCB, int64_t N, int64_t K,
+               __half *__restrict__ W_out) {
+    const int64_t per_row = K / 8;
+    const int64_t total = N * per_row;
+    for (int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x; c < total;
+         c += (int64_t)gridDim.x * kThreads) {
+        const int64_t n = c / per_row;
+        const float scb = SCB[n];
+        const uint2 q = reinterpret_cast<const uint2 *>(CB)[c];
+        __align__(16) __half out[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t word = e < 4 ? q.x : q.y;
+            const int v = (int)(int8_t)((word >> (8 * (e & 3))) & 0xffu);
+            out[e] = __float2half_rn(__fdiv_rn(__fmul_rn((float)v, scb), 127.0f));
+        }
+        reinterpret_cast<uint4 *>(W_out)[c] = *reinterpret_cast<const uint4 *>(out);
+    }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers ----------
+
+ScanPlan scan_plan(int64_t M, int64_t K) {
+    ScanPlan p;
+    p.col_blocks = ceil_div(K / 8, kThreads);
+    const int64_t target_ctas = 296;   // two waves' worth of CTAs on a 148-SM part
+    int64_t splits = std::max<int64_t>(1, target_ctas / p.col_blocks);
+    splits = std::min<int64_t>(splits, M);
+    p.rows_per_split = ceil_div(M, splits);
+    p.splits = ceil_div(M, p.rows_per_split);
+    p.nwords = ceil_div(K, 32);
+    return p;
+}
+
+cudaError_t launch_outlier_detect(const __half *X, int64_t M, int64_t K, float threshold,
+                                  const ScanPlan &plan, uint32_t *partial, uint32_t *bitmap,
+                                  int32_t *idx, int64_t cap, int32_t *count, uint32_t *status,
+                                  cudaStream_t s) {
+    dim3 grid((unsigned)plan.col_blocks, (unsigned)plan.splits);
+    outlier_scan_kernel<<<grid, kThreads, 0, s>>>(X, M, K, threshold, plan.rows_per_split,
+                                                  partial, plan.nwords);
+    outlier_compact_kernel<<<1, kCompactThreads, 0, s>>>(partial, (int)plan.splits, plan.nwords,
+                                                         idx, cap, count, bitmap, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rows(const __half *X, int64_t M, int64_t K, const uint32_t *bitmap,
+                                 const int32_t *idx, const int32_t *count, int64_t cap,
+                                 int64_t xo_pitch, int8_t *Xq, float *SCA, __half *Xo,
+                                 cudaStream_t s) {
+    quantize_rows_kernel<<<(unsigned)M, kThreads, 0, s>>>(X, K, bitmap, idx, count, cap, xo_pitch,
+                                                          Xq, SCA, Xo);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_outlier_w(const int8_t *CB, const float *SCB, const __half *W16,
+                                    int64_t N, int64_t K, const int32_t *idx,
+                                    const int32_t *count, int64_t cap, int64_t pitch, __half *Wo,
+                                    cudaStream_t s) {
+    const unsigned blocks = (unsigned)ceil_div(N, kThreads / 32);
+    gather_outlier_w_kernel<<<blocks, kThreads, 0, s>>>(CB, SCB, W16, N, K, idx, count, cap,
+                                                        pitch, Wo);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_weight(const __half *W, int64_t N, int64_t K, int8_t *CB, float *SCB,
+                                   cudaStream_t s) {
+    quantize_weight_kernel<<<(unsigned)N, kThreads, 0, s>>>(W, K, CB, SCB);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(const int8_t *CB, const float *SCB, int64_t N, int64_t K,
+                           __half *W_out, cudaStream_t s) {
+    const int64_t total = N * (K / 8);
+    const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(total, kThreads), 148 * 16);
+    dequant_kernel<<<blocks, kThreads, 0, s>>>(CB, SCB, N, K, W_out);
+    return cudaGetLastError();
+}
+
+}  // namespace llmint8

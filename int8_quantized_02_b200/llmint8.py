@@ -1,0 +1,218 @@
+"""Python binding of the C ABI in ``include/llmint8.h`` (argument marshalling only).
+
+Every function here takes torch CUDA tensors, allocates any missing output or workspace
+with torch, and calls the entry point of the same name in ``libllmint8.so`` on the
+current torch stream.  All arithmetic runs in the library's sm_100a kernels; there is no
+fallback: a missing library raises ``LLMInt8LibraryError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libllmint8.so")
+_lock = threading.Lock()
+_lib = None
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED_SHAPE = 2
+ERR_WORKSPACE_TOO_SMALL = 3
+ERR_OUTLIER_CAPACITY = 4
+ERR_TIMEOUT = 5
+ERR_CUDA = 6
+
+# Names and prototypes exactly as declared in include/llmint8.h.
+_P, _I64, _F32, _SZ, _U64 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t,
+                             ctypes.c_uint64)
+PROTOTYPES = {
+    "llmint8_quantize_weight_colwise": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "llmint8_quantize_rows_and_find_outliers": (
+        ctypes.c_int, [_P, _I64, _I64, _F32, _P, _P, _P, _P, _I64, _P, _SZ, _P]),
+    "llmint8_quantize_workspace_size": (_SZ, [_I64, _I64]),
+    "llmint8_linear": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _F32, _I64, _P, _P,
+                                      _SZ, _P, _P]),
+    "llmint8_linear_workspace_size": (_SZ, [_I64, _I64, _I64, _I64]),
+    "llmint8_dequant": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _P]),
+    "llmint8_device_status": (ctypes.c_int, [_P, _P]),
+    "llmint8_workspace_outlier_count": (ctypes.c_int, [_P, _P, _P]),
+    "llmint8_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "llmint8_set_wait_timeout_ns": (ctypes.c_int, [_U64]),
+}
+
+
+class LLMInt8LibraryError(RuntimeError):
+    """The compiled library is missing or does not load."""
+
+
+class LLMInt8Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} (status {code})")
+        self.code = code
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """The ctypes handle of libllmint8.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise LLMInt8LibraryError(
+                    f"{_LIB_PATH} is missing; build it with `python -m int8_quantized_02_b200.build`")
+            try:
+                lib = ctypes.CDLL(_LIB_PATH)
+            except OSError as e:  # pragma: no cover - depends on the machine
+                raise LLMInt8LibraryError(str(e)) from e
+            for name, (res, args) in PROTOTYPES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+        return _lib
+
+
+def status_string(code: int) -> str:
+    return load().llmint8_status_string(int(code)).decode()
+
+
+llmint8_status_string = status_string
+
+
+def _check(code: int, what: str):
+    if code != OK:
+        raise LLMInt8Error(code, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("llmint8 tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("llmint8 tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _want(t: torch.Tensor, dtype: torch.dtype, shape, name: str):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def default_max_outliers(K: int, threshold: float) -> int:
+    """Capacity used when the caller gives none: every column when the threshold marks
+    all of them (threshold <= 0), else min(K, 512)."""
+    return K if threshold <= 0 else min(K, 512)
+
+
+def llmint8_quantize_workspace_size(M: int, K: int) -> int:
+    return int(load().llmint8_quantize_workspace_size(M, K))
+
+
+def llmint8_linear_workspace_size(M: int, N: int, K: int, max_outliers: int) -> int:
+    return int(load().llmint8_linear_workspace_size(M, N, K, max_outliers))
+
+
+def llmint8_quantize_weight_colwise(W: torch.Tensor, CB=None, SCB=None, stream=None):
+    """W fp16 [N, K] -> (CB int8 [N, K], SCB fp32 [N])."""
+    N, K = W.shape
+    _want(W, torch.float16, (N, K), "W")
+    CB = torch.empty((N, K), dtype=torch.int8, device=W.device) if CB is None else CB
+    SCB = torch.empty((N,), dtype=torch.float32, device=W.device) if SCB is None else SCB
+    _want(CB, torch.int8, (N, K), "CB")
+    _want(SCB, torch.float32, (N,), "SCB")
+    _check(load().llmint8_quantize_weight_colwise(_ptr(W), N, K, _ptr(CB), _ptr(SCB),
+                                                  _stream(stream)),
+           "llmint8_quantize_weight_colwise")
+    return CB, SCB
+
+
+def llmint8_quantize_rows_and_find_outliers(X: torch.Tensor, threshold: float = 6.0,
+                                            cap: int | None = None, workspace=None,
+                                            stream=None):
+    """X fp16 [M, K] -> (Xq int8 [M, K], SCA fp32 [M], outlier_idx int32 [cap],
+    n_outliers int32 [1], workspace).  The first n_outliers entries of outlier_idx are valid."""
+    M, K = X.shape
+    _want(X, torch.float16, (M, K), "X")
+    cap = K if cap is None else int(cap)
+    dev = X.device
+    Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    SCA = torch.empty((M,), dtype=torch.float32, device=dev)
+    idx = torch.empty((max(cap, 1),), dtype=torch.int32, device=dev)
+    cnt = torch.empty((1,), dtype=torch.int32, device=dev)
+    need = llmint8_quantize_workspace_size(M, K)
+    ws = torch.empty((need,), dtype=torch.uint8, device=dev) if workspace is None else workspace
+    _check(load().llmint8_quantize_rows_and_find_outliers(
+        _ptr(X), M, K, ctypes.c_float(threshold), _ptr(Xq), _ptr(SCA), _ptr(idx), _ptr(cnt), cap,
+        _ptr(ws), ws.numel(), _stream(stream)), "llmint8_quantize_rows_and_find_outliers")
+    return Xq, SCA, idx, cnt, ws
+
+
+def llmint8_linear(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor, bias=None, W_fp16=None,
+                   threshold: float = 6.0, max_outliers: int | None = None, Y=None,
+                   workspace=None, C_debug=None, stream=None):
+    """The LLM.int8() layer: Y fp16 [M, N] from X fp16 [M, K] and the int8 weight (CB, SCB)."""
+    M, K = X.shape
+    N = CB.shape[0]
+    _want(X, torch.float16, (M, K), "X")
+    _want(CB, torch.int8, (N, K), "CB")
+    _want(SCB, torch.float32, (N,), "SCB")
+    if bias is not None:
+        _want(bias, torch.float16, (N,), "bias")
+    if W_fp16 is not None:
+        _want(W_fp16, torch.float16, (N, K), "W_fp16")
+    if C_debug is not None:
+        _want(C_debug, torch.int32, (M, N), "C_debug")
+    cap = default_max_outliers(K, threshold) if max_outliers is None else int(max_outliers)
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    _want(Y, torch.float16, (M, N), "Y")
+    if workspace is None:
+        workspace = torch.empty((llmint8_linear_workspace_size(M, N, K, cap),), dtype=torch.uint8,
+                                device=X.device)
+    _check(load().llmint8_linear(_ptr(X), M, K, _ptr(CB), _ptr(SCB), N, _ptr(bias), _ptr(W_fp16),
+                                 ctypes.c_float(threshold), cap, _ptr(Y), _ptr(workspace),
+                                 workspace.numel(), _stream(stream), _ptr(C_debug)),
+           "llmint8_linear")
+    return Y
+
+
+def llmint8_dequant(CB: torch.Tensor, SCB: torch.Tensor, out=None, stream=None):
+    """(CB int8 [N, K], SCB fp32 [N]) -> fp16 [N, K] = (CB * SCB) / 127."""
+    N, K = CB.shape
+    _want(CB, torch.int8, (N, K), "CB")
+    _want(SCB, torch.float32, (N,), "SCB")
+    out = torch.empty((N, K), dtype=torch.float16, device=CB.device) if out is None else out
+    _want(out, torch.float16, (N, K), "out")
+    _check(load().llmint8_dequant(_ptr(CB), _ptr(SCB), N, K, _ptr(out), _stream(stream)),
+           "llmint8_dequant")
+    return out
+
+
+def llmint8_device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronizes the stream; the device status code of the last call on `workspace`."""
+    return int(load().llmint8_device_status(_ptr(workspace), _stream(stream)))
+
+
+def llmint8_workspace_outlier_count(workspace: torch.Tensor, stream=None) -> int:
+    n = ctypes.c_int32(0)
+    _check(load().llmint8_workspace_outlier_count(_ptr(workspace), _stream(stream),
+                                                  ctypes.byref(n)),
+           "llmint8_workspace_outlier_count")
+    return int(n.value)
+
+
+def llmint8_set_wait_timeout_ns(ns: int) -> None:
+    _check(load().llmint8_set_wait_timeout_ns(int(ns)), "llmint8_set_wait_timeout_ns")

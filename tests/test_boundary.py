@@ -1,0 +1,98 @@
+"""The C-ABI library: it loads without a GPU, exports every symbol of include/llmint8.h, and
+its host-only entry points behave (workspace sizes, status strings).  No compute calls."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from int8_quantized_02_b200 import build as build_mod
+from int8_quantized_02_b200 import llmint8
+
+HEADER = os.path.join(build_mod.ROOT, "include", "llmint8.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return llmint8.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(llmint8_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("llmint8_quantize_weight_colwise", "llmint8_quantize_rows_and_find_outliers",
+              "llmint8_linear", "llmint8_dequant"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    out = subprocess.run(["nm", "-D", "--defined-only", llmint8.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(lib, n)
+    # the binding declares a prototype for each of them, and nothing else
+    assert sorted(llmint8.PROTOTYPES) == names
+
+
+def test_only_the_c_abi_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", llmint8.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    ours = set(re.findall(r"\bT (\w+)", out))
+    assert ours == set(declared_functions())
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = llmint8.status_string(code)
+        assert s and s != "unknown status"
+    assert llmint8.status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    f = llmint8.llmint8_linear_workspace_size
+    base = f(16, 1024, 1024, 0)
+    assert base > 16 * 1024          # holds at least Xq
+    assert f(16, 1024, 1024, 64) > base
+    assert f(32, 1024, 1024, 64) > f(16, 1024, 1024, 64)
+    # shapes outside the rules give 0
+    assert f(0, 1024, 1024, 0) == 0
+    assert f(16, 1000, 1024, 0) == 0          # N not a multiple of 16
+    assert f(16, 1024, 1000, 0) == 0          # K not a multiple of 16
+    assert f(16, 1024, 262144, 0) == 0        # K too large for int32 accumulation
+    assert f(16, 1024, 1024, 2048) == 0       # capacity above K
+    assert f(16, 1024, 1024, -1) == 0
+    q = llmint8.llmint8_quantize_workspace_size
+    assert q(16, 1024) >= 256 and q(0, 1024) == 0
+    assert q(4096, 16384) % 256 == 0
+
+
+def test_default_capacity():
+    assert llmint8.default_max_outliers(4096, 6.0) == 512
+    assert llmint8.default_max_outliers(4096, 0.0) == 4096
+    assert llmint8.default_max_outliers(64, 6.0) == 64
+
+
+def test_wait_timeout_setter(lib):
+    assert lib.llmint8_set_wait_timeout_ns(ctypes.c_uint64(5)) == 0
+    assert lib.llmint8_set_wait_timeout_ns(ctypes.c_uint64(0)) == 0   # restores the default
+
+
+def test_argument_errors_before_any_launch(lib):
+    # null pointers and bad shapes are rejected on the host, before any CUDA call
+    assert lib.llmint8_linear(None, 16, 1024, None, None, 1024, None, None,
+                              ctypes.c_float(6.0), 0, None, None, 0, None, None) == \
+        llmint8.ERR_INVALID_ARG
+    assert lib.llmint8_dequant(None, None, 16, 16, None, None) == llmint8.ERR_INVALID_ARG
