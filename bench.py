@@ -1,0 +1,477 @@
+"""Benchmark of the LLM.int8() decomposed linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  Workloads (seeded synthetic inputs, int8_quantized_02_b200.synth):
+  decode     (default) X [b, 4096] for b in (1, 8, 16), six outlier columns |x| in [6, 60] on
+             every row; CB [16384, 4096] quantized once beforehand.  One step = the three
+             llmint8_linear calls.  Metric: weight-streaming GB/s =
+             sum_b (N*K + 4N + 2bK + 2bN) / time.
+  ffn6.7b    X [2048, 4096] . W1^T (16384 outputs), then X2 [2048, 16384] . W2^T (4096 outputs);
+             six outlier columns of U(6, 20) on 75 % of rows.  Metric: TOPS = 2MNK / time.
+  proj175b   X [4096, 12288] . W^T (49152 outputs), W ~ N(0, 0.01).  TOPS.
+  sweep      X [4096, 8192] . W^T (8192 outputs); one step = K' in {0, 6, 64, 512} at
+             threshold 6, plus threshold=inf and threshold=0.  TOPS.
+Multi-GPU (torchrun): replicas only - every rank runs the same workload on its own GPU with no
+data-path collective; value = units of all ranks / max-over-ranks time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from int8_quantized_02_b200 import synth  # noqa: E402
+
+DECODE_BATCHES = (1, 8, 16)
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------- helpers ----
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.samples = []
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(
+                    ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                    timeout=5).stdout.strip()
+                parts = [p.strip() for p in out.split(",")]
+                if len(parts) == 6:
+                    self.samples.append(parts)
+            except Exception:  # noqa: BLE001 - sampling is best effort
+                pass
+            self._stop.wait(0.1)
+
+    def __enter__(self):
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._thread.join(timeout=10)
+
+    def summary(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if s[2 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "int8_quantized_02_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the product kernel from the committed ncu summary of this
+    workload, when it was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"kernel_source_hash:\s*(\w+)", text)
+    m_val = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_val or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_val.group(1))
+
+
+# -------------------------------------------------------------------------- workloads ----
+
+class Call:
+    """One llmint8_linear call with its resident inputs (and rotating weight copies)."""
+
+    def __init__(self, L, torch, X, CBs, SCBs, threshold, name, units, kernel_bytes,
+                 h2d_bytes, d2h_bytes, cap, rotation):
+        self.L, self.torch = L, torch
+        self.X, self.CBs, self.SCBs = X, CBs, SCBs
+        self.t, self.name = threshold, name
+        self.units, self.kernel_bytes = units, kernel_bytes
+        self.h2d_bytes, self.d2h_bytes = h2d_bytes, d2h_bytes
+        M, K = X.shape
+        N = CBs[0].shape[0]
+        self.M, self.K, self.N = M, K, N
+        self.cap = cap
+        self.ws = torch.empty((L.llmint8_linear_workspace_size(M, N, K, cap),),
+                              dtype=torch.uint8, device="cuda")
+        self.Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        self.rotation = rotation          # shared by all calls on the same weight copies
+
+    def run(self, X=None, Y=None):
+        i = self.rotation[0] % len(self.CBs)
+        self.rotation[0] += 1
+        self.L.llmint8_linear(self.X if X is None else X, self.CBs[i], self.SCBs[i],
+                              threshold=self.t, max_outliers=self.cap,
+                              Y=self.Y if Y is None else Y, workspace=self.ws)
+
+
+def _weights(L, torch, N, K, std, copies):
+    W = torch.from_numpy(synth.weight(N, K, std, seed=0)).cuda()
+    CB, SCB = L.llmint8_quantize_weight_colwise(W)
+    del W
+    CBs, SCBs = [CB], [SCB]
+    for _ in range(copies - 1):
+        CBs.append(CB.clone())
+        SCBs.append(SCB.clone())
+    return CBs, SCBs
+
+
+def build_workload(name, L, torch):
+    calls = []
+    if name == "decode":
+        N, K = 16384, 4096
+        copies = max(2, -(-3 * L2_BYTES // (N * K)) + 1)   # > 3 x L2 of weights in rotation
+        CBs, SCBs = _weights(L, torch, N, K, 0.02, copies)
+        rotation = [0]
+        for b in DECODE_BATCHES:
+            wl = synth.decode(b)
+            X = torch.from_numpy(wl.make_x()[0]).cuda()
+            nbytes = N * K + 4 * N + 2 * b * K + 2 * b * N
+            calls.append(Call(L, torch, X, CBs, SCBs, 6.0, wl.name, nbytes,
+                              N * K + 4 * N + b * K + 4 * b + 2 * b * N, 2 * b * K, 2 * b * N, 64,
+                              rotation))
+        unit, metric_bound = "GB/s", "hbm"
+    elif name in ("ffn6.7b", "proj175b", "sweep"):
+        if name == "ffn6.7b":
+            specs = [(synth.FFN_W1, 6.0), (synth.FFN_W2, 6.0)]
+        elif name == "proj175b":
+            specs = [(synth.PROJ_175B, 6.0)]
+        else:
+            specs = [(synth.sweep(k), 6.0) for k in (0, 6, 64, 512)] + \
+                [(synth.sweep(6, float("inf")), float("inf")), (synth.sweep(0, 0.0), 0.0)]
+        cache = {}
+        for wl, t in specs:
+            key = (wl.N, wl.K, wl.w_std)
+            if key not in cache:
+                cache[key] = _weights(L, torch, wl.N, wl.K, wl.w_std, 1)
+            CBs, SCBs = cache[key]
+            X = torch.from_numpy(wl.make_x()[0]).cuda()
+            cap = wl.K if t <= 0 else 512
+            calls.append(Call(L, torch, X, CBs, SCBs, t, wl.name, wl.int8_ops,
+                              wl.M * wl.K * 2 + wl.N * wl.K + 2 * wl.M * wl.N,
+                              2 * wl.M * wl.K, 2 * wl.M * wl.N, cap, [0]))
+        unit, metric_bound = "TOPS", "tensor"
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    return calls, unit, metric_bound
+
+
+def unit_value(units, seconds, unit):
+    return units / seconds / 1e9 if unit == "GB/s" else units / seconds / 1e12
+
+
+# ------------------------------------------------------------------------ our arm ----
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from int8_quantized_02_b200 import llmint8 as L
+
+    torch.cuda.set_device(local_rank)
+    L.load()
+    calls, unit, bound = build_workload(args.workload, L, torch)
+    step_units = sum(c.units for c in calls)
+
+    def step():
+        for c in calls:
+            c.run()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for c in calls:
+        st = L.llmint8_device_status(c.ws)
+        if st != L.OK:
+            raise SystemExit(f"{c.name}: device status {L.status_string(st)}")
+
+    # ---- timed region: whole steps, inputs resident, CUDA events on the launching stream
+    stream = torch.cuda.current_stream()
+    # per-call profile events around the product kernel
+    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in calls] for _ in range(args.steps)]
+    launches0 = L.llmint8_kernel_launch_count()
+    barrier()
+    with ClockSampler(local_rank) as clk:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(args.steps):
+            for j, c in enumerate(calls):
+                L.llmint8_set_profile_events(*kev[s][j])
+                c.run()
+        e1.record(stream)
+        L.llmint8_set_profile_events(None, None)
+        torch.cuda.synchronize()
+    barrier()
+    launches = L.llmint8_kernel_launch_count() - launches0
+    elapsed = e0.elapsed_time(e1) / 1e3
+    t = torch.tensor([elapsed], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed = float(t.item())
+    kern_s = sum(kev[s][j][0].elapsed_time(kev[s][j][1]) for s in range(args.steps)
+                 for j in range(len(calls))) / 1e3
+    kern_bytes = sum(c.kernel_bytes for c in calls) * args.steps
+    for c in calls:
+        st = L.llmint8_device_status(c.ws)
+        if st != L.OK:
+            raise SystemExit(f"{c.name}: device status {L.status_string(st)}")
+
+    # ---- end to end through the public API: pinned host X in, host Y out, every call
+    hosts = [(c.X.cpu().pin_memory(),
+              torch.empty((c.M, c.N), dtype=torch.float16).pin_memory()) for c in calls]
+    xd = [torch.empty_like(c.X) for c in calls]
+    e2e_steps = max(1, min(args.steps, 50))
+    for _ in range(2):
+        for j, c in enumerate(calls):
+            xd[j].copy_(hosts[j][0], non_blocking=True)
+            c.run(X=xd[j])
+            hosts[j][1].copy_(c.Y, non_blocking=True)
+    barrier()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        for j, c in enumerate(calls):
+            xd[j].copy_(hosts[j][0], non_blocking=True)
+            c.run(X=xd[j])
+            hosts[j][1].copy_(c.Y, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_t = torch.tensor([a0.elapsed_time(a1) / 1e3], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_s = float(e2e_t.item())
+
+    peaks = measured_peaks()
+    if bound == "hbm":
+        achieved = kern_bytes / kern_s / 1e9
+        peak = peaks["hbm_gbs"]
+        roof_unit = "GB/s"
+        traffic = profiled_traffic(args.workload)
+    else:
+        kern_ops = sum(c.units for c in calls) * args.steps
+        achieved = kern_ops / kern_s / 1e12
+        peak = 2.0 * peaks["bf16_tflops"]           # int8 dense = 2 x bf16 dense (nominal ratio)
+        roof_unit = "TOPS"
+        traffic = profiled_traffic(args.workload)
+    result = {
+        "metric": "LLM.int8 linear TOPS (prefill) / weight GB/s (decode); fraction of roofline",
+        "value": unit_value(step_units * args.steps * world, elapsed, unit),
+        "unit": unit,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": elapsed / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "i8/i32 (fp16 in/out, fp16 outlier product)",
+        "data": "synthetic (seeded, int8_quantized_02_b200.synth)",
+        "config": workload_config(args.workload, calls),
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": roof_unit,
+                     "frac": achieved / peak,
+                     "peak_source": f"{peaks['source']} "
+                                    + ("hbm_gbs" if bound == "hbm" else "2 x bf16_tflops (burst)"),
+                     "kernel": "llmint8_gemm_kernel",
+                     "traffic": traffic},
+        "e2e": {"value": unit_value(step_units * e2e_steps * world, e2e_s, unit), "unit": unit,
+                "h2d_bytes_per_step": sum(c.h2d_bytes for c in calls),
+                "d2h_bytes_per_step": sum(c.d2h_bytes for c in calls)},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "per_call": {c.name: None for c in calls},
+    }
+    # per-call achieved figure of the product kernel
+    for j, c in enumerate(calls):
+        ks = sum(kev[s][j][0].elapsed_time(kev[s][j][1]) for s in range(args.steps)) / 1e3
+        v = (c.kernel_bytes / (ks / args.steps) / 1e9) if bound == "hbm" else \
+            (c.units / (ks / args.steps) / 1e12)
+        result["per_call"][c.name] = {"kernel_us": ks / args.steps * 1e6,
+                                      ("GB/s" if bound == "hbm" else "TOPS"): v}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args.workload)
+    return result
+
+
+def workload_config(name, calls):
+    cfg = {"workload": name,
+           "calls": [{"name": c.name, "M": c.M, "K": c.K, "N": c.N, "threshold": c.t,
+                      "max_outliers": c.cap} for c in calls],
+           "parallelism": "replicas"}
+    if name == "decode":
+        cfg["l2"] = (f"{len(calls[0].CBs)} rotating int8 weight copies "
+                     f"({len(calls[0].CBs) * calls[0].N * calls[0].K / 2**20:.0f} MiB > 126 MiB L2)")
+    else:
+        cfg["l2"] = "inputs larger than L2 (weights and activations)"
+    return cfg
+
+
+# ------------------------------------------------------------------- oracle (CPU) ----
+
+def _oracle_sample(name):
+    """A bounded sample of the workload for the CPU oracle and its metric units."""
+    if name == "decode":
+        N, K, b = 16384, 4096, 16
+        rows = 2048                                   # 1/8 of the output channels
+        W = synth.weight(rows, K, 0.02, seed=0)
+        X = synth.decode(b).make_x()[0]
+        units = rows * K + 4 * rows + 2 * b * K + 2 * b * rows
+        desc = f"decode b={b}: X [16, 4096] against {rows} of the {N} output channels"
+        return X, W, 6.0, units, desc
+    wl = {"ffn6.7b": synth.FFN_W1, "proj175b": synth.PROJ_175B, "sweep": synth.sweep(6)}[name]
+    rows_x, rows_w = 256, 512
+    X = wl.make_x()[0][:rows_x].copy()
+    W = synth.weight(rows_w, wl.K, wl.w_std, seed=0)
+    units = 2 * rows_x * rows_w * wl.K
+    desc = f"{wl.name}: first {rows_x} rows of X against {rows_w} output channels"
+    return X, W, wl.threshold, units, desc
+
+
+def cpu_baseline(name, reps=None):
+    from oracle import oracle
+    X, W, t, units, desc = _oracle_sample(name)
+    CB, SCB = oracle.quantize_weight_colwise(W)
+    oracle.linear(X[:1], CB[:16], SCB[:16], threshold=t)   # load + warm
+    times = []
+    deadline = time.perf_counter() + 15.0
+    while True:
+        t0 = time.perf_counter()
+        oracle.linear(X, CB, SCB, threshold=t)
+        times.append(time.perf_counter() - t0)
+        if (reps is not None and len(times) >= reps) or (reps is None and
+                                                           time.perf_counter() > deadline):
+            break
+    unit = "GB/s" if name == "decode" else "TOPS"
+    sec = statistics.median(times)
+    return {"value": unit_value(units, sec, unit), "unit": unit,
+            "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count())), "kind": "oracle",
+            "sample": f"{desc}; median of {len(times)} runs of {sec:.3f} s"}
+
+
+def run_reference(args, rank, world):
+    """The oracle timed on the host cores on a bounded sample of the same workload."""
+    if rank != 0:
+        return None
+    from oracle import oracle
+    X, W, t, units, desc = _oracle_sample(args.workload)
+    CB, SCB = oracle.quantize_weight_colwise(W)
+    for _ in range(min(args.warmup, 1)):
+        oracle.linear(X, CB, SCB, threshold=t)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.linear(X, CB, SCB, threshold=t)
+    sec = time.perf_counter() - t0
+    unit = "GB/s" if args.workload == "decode" else "TOPS"
+    value = unit_value(units * args.steps, sec, unit)
+    return {
+        "impl": "reference",
+        "metric": "LLM.int8 linear TOPS (prefill) / weight GB/s (decode); fraction of roofline",
+        "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8/i32 (fp16 in/out)",
+        "data": "synthetic (seeded, int8_quantized_02_b200.synth)",
+        "config": {"workload": args.workload, "sample": desc, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": unit,
+                         "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count())),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="decode",
+                    choices=("decode", "ffn6.7b", "proj175b", "sweep"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -145,6 +145,19 @@ LLMINT8_API const char *llmint8_status_string(llmint8_status status);
  */
 LLMINT8_API llmint8_status llmint8_set_wait_timeout_ns(uint64_t ns);
 
+/*
+ * Measurement hooks (no counterpart on the pages; they let a benchmark time the product
+ * kernel of a call with CUDA events and count launches):
+ *   llmint8_set_profile_events(start, stop): two cudaEvent_t.  While both are non-NULL,
+ *     every llmint8_linear call records `start` on its stream immediately before its
+ *     product kernel (the GEMM) and `stop` immediately after it.  NULL, NULL disables.
+ *     Process-wide; the caller owns the events and must keep them alive while set.
+ *   llmint8_kernel_launch_count(): number of kernels this library has launched in the
+ *     process so far.
+ */
+LLMINT8_API llmint8_status llmint8_set_profile_events(void *start, void *stop);
+LLMINT8_API uint64_t llmint8_kernel_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

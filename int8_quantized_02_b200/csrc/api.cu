@@ -14,6 +14,8 @@ namespace {
 
 constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<uint64_t> g_launches{0};
+std::atomic<cudaEvent_t> g_prof_start{nullptr}, g_prof_stop{nullptr};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -78,7 +80,19 @@ llmint8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK :
 
 }  // namespace
 
+void llmint8::note_launches(int n) { g_launches.fetch_add((uint64_t)n); }
+
 extern "C" {
+
+llmint8_status llmint8_set_profile_events(void *start, void *stop) {
+    if ((start == nullptr) != (stop == nullptr)) return LLMINT8_ERR_INVALID_ARG;
+    g_prof_start.store(static_cast<cudaEvent_t>(start));
+    g_prof_stop.store(static_cast<cudaEvent_t>(stop));
+    return LLMINT8_OK;
+}
+
+uint64_t llmint8_kernel_launch_count(void) { return g_launches.load(); }
+
 
 const char *llmint8_status_string(llmint8_status s) {
     switch (s) {
@@ -207,7 +221,12 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     g.N = N;
     g.K = K;
     g.timeout_ns = g_timeout_ns.load();
-    return from_cuda(launch_gemm(g, s));
+    cudaEvent_t ev0 = g_prof_start.load(), ev1 = g_prof_stop.load();
+    if (ev0 && cudaEventRecord(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    e = launch_gemm(g, s);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (ev1 && cudaEventRecord(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    return LLMINT8_OK;
 }
 
 llmint8_status llmint8_device_status(const void *ws, void *stream) {

@@ -390,6 +390,7 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s) {
     const int tiles = a.tiles_m * a.tiles_n;
     const int grid = std::min(tiles, sms);
     llmint8_gemm_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmXo, tmWo, a);
+    note_launches(1);
     return cudaGetLastError();
 }
 

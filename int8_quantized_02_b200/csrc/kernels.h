@@ -10,6 +10,9 @@
 
 namespace llmint8 {
 
+// Adds n to the process-wide count of kernels launched by the library.
+void note_launches(int n);
+
 // Row-split plan of the outlier scan: the columns are covered by `col_blocks` CTAs of
 // 256 threads x 8 columns, the rows by `splits` ranges of `rows_per_split` rows.
 struct ScanPlan {

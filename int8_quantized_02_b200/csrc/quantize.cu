@@ -351,6 +351,7 @@ cudaError_t launch_outlier_detect(const __half *X, int64_t M, int64_t K, float t
                                                   partial, plan.nwords);
     outlier_compact_kernel<<<1, kCompactThreads, 0, s>>>(partial, (int)plan.splits, plan.nwords,
                                                          idx, cap, count, bitmap, status);
+    note_launches(2);
     return cudaGetLastError();
 }
 
@@ -360,6 +361,7 @@ cudaError_t launch_quantize_rows(const __half *X, int64_t M, int64_t K, const ui
                                  cudaStream_t s) {
     quantize_rows_kernel<<<(unsigned)M, kThreads, 0, s>>>(X, K, bitmap, idx, count, cap, xo_pitch,
                                                           Xq, SCA, Xo);
+    note_launches(1);
     return cudaGetLastError();
 }
 
@@ -370,12 +372,14 @@ cudaError_t launch_gather_outlier_w(const int8_t *CB, const float *SCB, const __
     const unsigned blocks = (unsigned)ceil_div(N, kThreads / 32);
     gather_outlier_w_kernel<<<blocks, kThreads, 0, s>>>(CB, SCB, W16, N, K, idx, count, cap,
                                                         pitch, Wo);
+    note_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_weight(const __half *W, int64_t N, int64_t K, int8_t *CB, float *SCB,
                                    cudaStream_t s) {
     quantize_weight_kernel<<<(unsigned)N, kThreads, 0, s>>>(W, K, CB, SCB);
+    note_launches(1);
     return cudaGetLastError();
 }
 
@@ -384,6 +388,7 @@ cudaError_t launch_dequant(const int8_t *CB, const float *SCB, int64_t N, int64_
     const int64_t total = N * (K / 8);
     const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(total, kThreads), 148 * 16);
     dequant_kernel<<<blocks, kThreads, 0, s>>>(CB, SCB, N, K, W_out);
+    note_launches(1);
     return cudaGetLastError();
 }
 

@@ -41,6 +41,8 @@ PROTOTYPES = {
     "llmint8_workspace_outlier_count": (ctypes.c_int, [_P, _P, _P]),
     "llmint8_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "llmint8_set_wait_timeout_ns": (ctypes.c_int, [_U64]),
+    "llmint8_set_profile_events": (ctypes.c_int, [_P, _P]),
+    "llmint8_kernel_launch_count": (_U64, []),
 }
 
 
@@ -216,3 +218,15 @@ def llmint8_workspace_outlier_count(workspace: torch.Tensor, stream=None) -> int
 
 def llmint8_set_wait_timeout_ns(ns: int) -> None:
     _check(load().llmint8_set_wait_timeout_ns(int(ns)), "llmint8_set_wait_timeout_ns")
+
+
+def llmint8_set_profile_events(start=None, stop=None) -> None:
+    """Record torch.cuda.Event pair (start, stop) around the product kernel of every later
+    llmint8_linear call; (None, None) disables."""
+    s = None if start is None else ctypes.c_void_p(start.cuda_event)
+    e = None if stop is None else ctypes.c_void_p(stop.cuda_event)
+    _check(load().llmint8_set_profile_events(s, e), "llmint8_set_profile_events")
+
+
+def llmint8_kernel_launch_count() -> int:
+    return int(load().llmint8_kernel_launch_count())
