@@ -244,6 +244,13 @@ def run_ours(args, rank, world, local_rank):
     # per-call profile events around the product kernel
     kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in calls] for _ in range(args.steps)]
+    # torch creates an event's CUDA handle on its first record(): record each once here so
+    # the library can re-record the same handles around the product kernel
+    for row in kev:
+        for ev_a, ev_b in row:
+            ev_a.record(stream)
+            ev_b.record(stream)
+    torch.cuda.synchronize()
     launches0 = L.llmint8_kernel_launch_count()
     barrier()
     with ClockSampler(local_rank) as clk:

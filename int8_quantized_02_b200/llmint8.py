@@ -225,6 +225,8 @@ def llmint8_set_profile_events(start=None, stop=None) -> None:
     llmint8_linear call; (None, None) disables."""
     s = None if start is None else ctypes.c_void_p(start.cuda_event)
     e = None if stop is None else ctypes.c_void_p(stop.cuda_event)
+    if (start is not None and not start.cuda_event) or (stop is not None and not stop.cuda_event):
+        raise ValueError("record the events once before handing them to the library")
     _check(load().llmint8_set_profile_events(s, e), "llmint8_set_profile_events")
 
 
