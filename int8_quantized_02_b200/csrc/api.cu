@@ -15,6 +15,11 @@ namespace {
 constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<uint64_t> g_launches{0};
+std::atomic<unsigned long long> g_epoch{1};   // one per call that writes a status word
+
+StatusRef next_status(WsHeader *h) {
+    return StatusRef{&h->status, g_epoch.fetch_add(1) << 4};
+}
 std::atomic<cudaEvent_t> g_prof_start{nullptr}, g_prof_stop{nullptr};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -77,6 +82,13 @@ T *at(void *ws, size_t off) {
 }
 
 llmint8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA; }
+
+// The single-launch decode kernel covers few activation rows and an X that fits in shared
+// memory once quantized; threshold <= 0 (every column fp16) goes through the GEMM path.
+bool use_decode_path(int64_t M, int64_t K, float threshold, int64_t cap) {
+    return M <= kDecodeMaxM && K <= kDecodeMaxK && threshold > 0.0f &&
+           cap <= kDecodeMaxOutliers;
+}
 
 }  // namespace
 
@@ -160,7 +172,7 @@ llmint8_status llmint8_quantize_rows_and_find_outliers(const uint16_t *X, int64_
     const __half *Xh = reinterpret_cast<const __half *>(X);
     uint32_t *bitmap = at<uint32_t>(ws, L.bitmap);
     cudaError_t e = launch_outlier_detect(Xh, M, K, threshold, L.plan, at<uint32_t>(ws, L.partial),
-                                          bitmap, outlier_idx, cap, n_outliers, &h->status, s);
+                                          bitmap, outlier_idx, cap, n_outliers, next_status(h), s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     return from_cuda(launch_quantize_rows(Xh, M, K, bitmap, outlier_idx, n_outliers, cap, 0, Xq,
                                           SCA, nullptr, s));
@@ -183,7 +195,36 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     if (ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsHeader *h = at<WsHeader>(ws, 0);
+    const StatusRef status = next_status(h);
     const __half *Xh = reinterpret_cast<const __half *>(X);
+    cudaEvent_t ev0 = g_prof_start.load(), ev1 = g_prof_stop.load();
+    cudaError_t e;
+
+    if (use_decode_path(M, K, threshold, max_outliers)) {
+        // one launch: quantization of X per CTA + weight-streaming tcgen05 product
+        DecodeLaunch d;
+        d.X = Xh;
+        d.CB = CB;
+        d.SCB = SCB;
+        d.W16 = reinterpret_cast<const __half *>(W_fp16);
+        d.bias = reinterpret_cast<const __half *>(bias);
+        d.Y = reinterpret_cast<__half *>(Y);
+        d.C_debug = C_debug;
+        d.count = &h->n_outliers;
+        d.status = status;
+        d.M = M;
+        d.N = N;
+        d.K = K;
+        d.cap = max_outliers;
+        d.threshold = threshold;
+        d.timeout_ns = g_timeout_ns.load();
+        if (ev0 && cudaEventRecord(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+        e = launch_decode(d, s);
+        if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+        if (ev1 && cudaEventRecord(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+        return LLMINT8_OK;
+    }
+
     uint32_t *bitmap = at<uint32_t>(ws, L.bitmap);
     int32_t *idx = at<int32_t>(ws, L.idx);
     float *SCA = at<float>(ws, L.sca);
@@ -191,9 +232,8 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     __half *Xo = at<__half>(ws, L.xo);
     __half *Wo = at<__half>(ws, L.wo);
 
-    cudaError_t e = launch_outlier_detect(Xh, M, K, threshold, L.plan, at<uint32_t>(ws, L.partial),
-                                          bitmap, idx, max_outliers, &h->n_outliers, &h->status,
-                                          s);
+    e = launch_outlier_detect(Xh, M, K, threshold, L.plan, at<uint32_t>(ws, L.partial), bitmap,
+                              idx, max_outliers, &h->n_outliers, status, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     e = launch_quantize_rows(Xh, M, K, bitmap, idx, &h->n_outliers, max_outliers, L.pitch, Xq, SCA,
                              max_outliers > 0 ? Xo : nullptr, s);
@@ -216,12 +256,11 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     g.bias = reinterpret_cast<const __half *>(bias);
     g.Y = reinterpret_cast<__half *>(Y);
     g.C_debug = C_debug;
-    g.status = &h->status;
+    g.status = status;
     g.M = M;
     g.N = N;
     g.K = K;
     g.timeout_ns = g_timeout_ns.load();
-    cudaEvent_t ev0 = g_prof_start.load(), ev1 = g_prof_stop.load();
     if (ev0 && cudaEventRecord(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
     e = launch_gemm(g, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
@@ -233,10 +272,10 @@ llmint8_status llmint8_device_status(const void *ws, void *stream) {
     if (!ws) return LLMINT8_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    uint32_t st = 0;
+    unsigned long long st = 0;
     if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    return static_cast<llmint8_status>(st);
+    return static_cast<llmint8_status>(st & 0xFull);
 }
 
 llmint8_status llmint8_workspace_outlier_count(const void *ws, void *stream, int32_t *count) {

@@ -14,9 +14,9 @@ namespace llmint8 {
 
 // Layout of the first 256 bytes of every workspace.
 struct WsHeader {
-    uint32_t status;      // llmint8_status of the last call (device conditions)
-    int32_t n_outliers;   // true number of outlier columns found by the last call
-    uint32_t pad[62];
+    unsigned long long status;  // (call epoch << 4) | llmint8_status, see StatusRef
+    int32_t n_outliers;         // true number of outlier columns found by the last call
+    uint32_t pad[61];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
@@ -59,12 +59,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The device status word of a workspace holds (epoch << 4) | code, where every library
+// call gets a new, larger epoch.  Writers use atomicMax: within one call the most severe
+// code wins (OK < OUTLIER_CAPACITY < TIMEOUT) and a value left by an older call is always
+// replaced, whatever order the kernels and CTAs of the call write in.
+struct StatusRef {
+    unsigned long long *word;
+    unsigned long long tag;     // epoch << 4
+    __device__ __forceinline__ void raise(llmint8_status code) const {
+        atomicMax(word, tag | (unsigned long long)code);
+    }
+};
+
 // Every wait of a pipeline goes through this: it gives up after `timeout_ns`, or as soon
 // as another thread of the CTA gave up, records LLMINT8_ERR_TIMEOUT in the workspace
 // status word and returns false so that the caller can wind the kernel down.
 struct BoundedWait {
     volatile int *abort_flag;   // shared memory, one per CTA
-    uint32_t *status;           // global status word
+    StatusRef status;
     uint64_t timeout_ns;
 
     __device__ __forceinline__ bool operator()(uint32_t bar, uint32_t parity) const {
@@ -76,7 +88,7 @@ struct BoundedWait {
                 if (*abort_flag) return false;
                 if (global_timer_ns() - t0 > timeout_ns) {
                     *abort_flag = 1;
-                    atomicCAS(status, 0u, (uint32_t)LLMINT8_ERR_TIMEOUT);
+                    status.raise(LLMINT8_ERR_TIMEOUT);
                     return false;
                 }
             }
@@ -86,13 +98,13 @@ struct BoundedWait {
 
 // Wait used while winding down (draining copies / MMAs still in flight): ignores the abort
 // flag, bounded by a fixed limit.
-__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32_t *status) {
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, StatusRef status) {
     constexpr uint64_t kDrainNs = 1000000000ull;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 0u && global_timer_ns() - t0 > kDrainNs) {
-            atomicCAS(status, 0u, (uint32_t)LLMINT8_ERR_TIMEOUT);
+            status.raise(LLMINT8_ERR_TIMEOUT);
             return false;
         }
     }
@@ -170,6 +182,25 @@ __device__ __forceinline__ void tmem_ld_32x32(uint32_t taddr, uint32_t (&r)[32])
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
           "=r"(r[31])
         : "r"(taddr));
+}
+// Warp-wide: 32 lanes x 16 consecutive 32-bit columns from TMEM into registers.
+__device__ __forceinline__ void tmem_ld_32x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+// Makes this thread's generic-proxy shared-memory writes visible to the async proxy
+// (TMA, tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Named barrier over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");

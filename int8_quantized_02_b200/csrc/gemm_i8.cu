@@ -60,7 +60,7 @@ struct Args {
     const __half *bias;
     __half *Y;
     int32_t *C_debug;
-    uint32_t *status;
+    StatusRef status;
     int M, N, K;
     int num_kb;
     int tiles_m, tiles_n;

@@ -8,6 +8,8 @@
 
 #include <algorithm>
 
+#include "common.cuh"
+
 namespace llmint8 {
 
 // Adds n to the process-wide count of kernels launched by the library.
@@ -22,7 +24,7 @@ ScanPlan scan_plan(int64_t M, int64_t K);
 
 cudaError_t launch_outlier_detect(const __half *X, int64_t M, int64_t K, float threshold,
                                   const ScanPlan &plan, uint32_t *partial, uint32_t *bitmap,
-                                  int32_t *idx, int64_t cap, int32_t *count, uint32_t *status,
+                                  int32_t *idx, int64_t cap, int32_t *count, StatusRef status,
                                   cudaStream_t s);
 cudaError_t launch_quantize_rows(const __half *X, int64_t M, int64_t K, const uint32_t *bitmap,
                                  const int32_t *idx, const int32_t *count, int64_t cap,
@@ -51,10 +53,37 @@ struct GemmLaunch {
     const __half *bias;      // [N] or null
     __half *Y;               // [M, N]
     int32_t *C_debug;        // [M, N] or null
-    uint32_t *status;
+    StatusRef status;
     int64_t M, N, K;
     uint64_t timeout_ns;
 };
 cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s);
+
+}  // namespace llmint8
+
+namespace llmint8 {
+
+// Single-launch decode path (M <= kDecodeMaxM): per CTA, outlier detection and row
+// quantization of X into shared memory, then a TMA-fed tcgen05 product with the weight
+// rows as the 128-row operand, fused outlier and dequantization epilogue.
+constexpr int kDecodeMaxM = 16;
+constexpr int kDecodeMaxK = 8192;
+constexpr int kDecodeMaxOutliers = 256;
+
+struct DecodeLaunch {
+    const __half *X;         // [M, K]
+    const int8_t *CB;        // [N, K]
+    const float *SCB;        // [N]
+    const __half *W16;       // [N, K] or null
+    const __half *bias;      // [N] or null
+    __half *Y;               // [M, N]
+    int32_t *C_debug;        // [M, N] or null
+    int32_t *count;          // device outlier count (workspace header)
+    StatusRef status;
+    int64_t M, N, K, cap;
+    float threshold;
+    uint64_t timeout_ns;
+};
+cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s);
 
 }  // namespace llmint8

@@ -111,7 +111,7 @@ constexpr int kMaxWordsPerThread = 4;   // nwords <= 4096 (K <= 131072)
 __global__ void __launch_bounds__(kCompactThreads)
 outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t nwords,
                        int32_t *__restrict__ idx, int64_t cap, int32_t *__restrict__ count_out,
-                       uint32_t *__restrict__ bitmap_out, uint32_t *__restrict__ status) {
+                       uint32_t *__restrict__ bitmap_out, StatusRef status) {
     __shared__ int warp_tot[32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wpt = (int)ceil_div(nwords, kCompactThreads);
@@ -163,7 +163,7 @@ outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t
     }
     if (tid == kCompactThreads - 1) {
         *count_out = pos;
-        *status = (pos > cap) ? (uint32_t)LLMINT8_ERR_OUTLIER_CAPACITY : (uint32_t)LLMINT8_OK;
+        status.raise(pos > cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
     }
 }
 
@@ -344,7 +344,7 @@ ScanPlan scan_plan(int64_t M, int64_t K) {
 
 cudaError_t launch_outlier_detect(const __half *X, int64_t M, int64_t K, float threshold,
                                   const ScanPlan &plan, uint32_t *partial, uint32_t *bitmap,
-                                  int32_t *idx, int64_t cap, int32_t *count, uint32_t *status,
+                                  int32_t *idx, int64_t cap, int32_t *count, StatusRef status,
                                   cudaStream_t s) {
     dim3 grid((unsigned)plan.col_blocks, (unsigned)plan.splits);
     outlier_scan_kernel<<<grid, kThreads, 0, s>>>(X, M, K, threshold, plan.rows_per_split,

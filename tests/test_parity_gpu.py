@@ -222,3 +222,73 @@ def test_linear_rejects_bad_arguments():
         L.llmint8_quantize_weight_colwise(torch.zeros((16, 72), dtype=torch.float16,
                                                       device="cuda"))
     assert e.value.code == L.ERR_UNSUPPORTED_SHAPE
+
+
+# ------------------------------------------------ single-launch decode path (M <= 16) ----
+
+DECODE_CASES = [(1, 64, 64), (2, 1040, 144), (7, 4096, 400), (8, 4096, 16384),
+                (16, 4096, 16384), (16, 8192, 1024), (16, 16, 48), (13, 2048, 2064)]
+
+
+@pytest.mark.parametrize("variant", ["plain", "bias_fp16w", "no_outliers"])
+@pytest.mark.parametrize("M,K,N", DECODE_CASES, ids=lambda v: str(v))
+def test_decode_path_matches_oracle(M, K, N, variant):
+    n_out = 0 if variant == "no_outliers" else min(6, K // 8)
+    X = _x(M, K, n_out, lo=6.0, hi=60.0, row_frac=1.0, seed=M * 7 + K)
+    W = synth.weight(N, K, 0.02, seed=N + 1)
+    if variant == "bias_fp16w":
+        _check_linear(X, W, 6.0, bias=synth.bias(N, seed=3), keep_fp16=True, cap=64)
+    else:
+        _check_linear(X, W, 6.0, cap=64)
+
+
+def test_decode_path_planted_rows():
+    X = _x(16, 1024, 3, lo=6.0, hi=20.0, row_frac=0.5, seed=21)
+    X[2] = 0                          # zero row
+    X[5, 10] = 6.0                    # exactly the threshold
+    X[9] = 0
+    X[9, 100] = -9.0                  # outlier-only row
+    X[11, :] = 0.125                  # constant row: absmax ties everywhere
+    W = synth.weight(272, 1024, 0.02, seed=21)
+    _check_linear(X, W, 6.0, cap=64)
+
+
+def test_gemm_path_small_M():
+    # a capacity above the decode kernel's limit routes M <= 16 through the GEMM path
+    X = _x(16, 1024, 5, seed=22)
+    W = synth.weight(512, 1024, 0.02, seed=22)
+    _check_linear(X, W, 6.0, cap=512)
+
+
+def test_decode_capacity_overflow_reports_status():
+    X = _x(8, 512, 10, lo=7.0, hi=9.0, row_frac=1.0, seed=23)
+    W = synth.weight(256, 512, 0.02, seed=23)
+    CB, SCB = L.llmint8_quantize_weight_colwise(dev(W))
+    ws = torch.empty((L.llmint8_linear_workspace_size(8, 256, 512, 4),), dtype=torch.uint8,
+                     device="cuda")
+    L.llmint8_linear(dev(X), CB, SCB, threshold=6.0, max_outliers=4, workspace=ws)
+    assert L.llmint8_device_status(ws) == L.ERR_OUTLIER_CAPACITY
+    assert L.llmint8_workspace_outlier_count(ws) == 10
+    # a later call on the same workspace reports its own status again
+    _check_linear(X, W, 6.0, cap=64)
+
+
+def test_decode_bounded_wait_timeout_is_reported():
+    X = _x(16, 4096, 6, seed=24)
+    W = synth.weight(4096, 4096, 0.02, seed=24)
+    CB, SCB = L.llmint8_quantize_weight_colwise(dev(W))
+    ws = torch.empty((L.llmint8_linear_workspace_size(16, 4096, 4096, 64),), dtype=torch.uint8,
+                     device="cuda")
+    seen = set()
+    try:
+        L.llmint8_set_wait_timeout_ns(1)
+        for _ in range(3):
+            L.llmint8_linear(dev(X), CB, SCB, threshold=6.0, max_outliers=64, workspace=ws)
+            seen.add(L.llmint8_device_status(ws))
+            if L.ERR_TIMEOUT in seen:
+                break
+    finally:
+        L.llmint8_set_wait_timeout_ns(0)
+    assert L.ERR_TIMEOUT in seen
+    assert seen <= {L.OK, L.ERR_TIMEOUT}
+    _check_linear(X, W, 6.0, cap=64)
