@@ -18,7 +18,7 @@ std::atomic<uint64_t> g_launches{0};
 std::atomic<unsigned long long> g_epoch{1};   // one per call that writes a status word
 
 StatusRef next_status(WsHeader *h) {
-    return StatusRef{&h->status, g_epoch.fetch_add(1) << 4};
+    return StatusRef{&h->status, &h->timeout, g_epoch.fetch_add(1) << 4};
 }
 std::atomic<cudaEvent_t> g_prof_start{nullptr}, g_prof_stop{nullptr};
 
@@ -272,10 +272,11 @@ llmint8_status llmint8_device_status(const void *ws, void *stream) {
     if (!ws) return LLMINT8_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    unsigned long long st = 0;
-    if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
+    unsigned long long words[2] = {0, 0};   // status, timeout
+    if (cudaMemcpy(words, ws, sizeof(words), cudaMemcpyDeviceToHost) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    return static_cast<llmint8_status>(st & 0xFull);
+    if ((words[1] >> 4) == (words[0] >> 4)) return LLMINT8_ERR_TIMEOUT;
+    return static_cast<llmint8_status>(words[0] & 0xFull);
 }
 
 llmint8_status llmint8_workspace_outlier_count(const void *ws, void *stream, int32_t *count) {

@@ -14,9 +14,10 @@ namespace llmint8 {
 
 // Layout of the first 256 bytes of every workspace.
 struct WsHeader {
-    unsigned long long status;  // (call epoch << 4) | llmint8_status, see StatusRef
-    int32_t n_outliers;         // true number of outlier columns found by the last call
-    uint32_t pad[61];
+    unsigned long long status;   // (call epoch << 4) | llmint8_status, one writer per call
+    unsigned long long timeout;  // (call epoch << 4) | LLMINT8_ERR_TIMEOUT after a timeout
+    int32_t n_outliers;          // true number of outlier columns found by the last call
+    uint32_t pad[59];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
@@ -59,15 +60,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// The device status word of a workspace holds (epoch << 4) | code, where every library
-// call gets a new, larger epoch.  Writers use atomicMax: within one call the most severe
-// code wins (OK < OUTLIER_CAPACITY < TIMEOUT) and a value left by an older call is always
-// replaced, whatever order the kernels and CTAs of the call write in.
+// Device-side conditions of a call.  Every call gets a new epoch.  Exactly one thread of
+// the call stores (epoch << 4) | code into the status word (the outlier-count result,
+// written before anything can time out in that kernel); any thread whose bounded wait
+// gives up stores (epoch << 4) | TIMEOUT into the timeout word.  The host reports TIMEOUT
+// when both words carry the same epoch, else the status word's code.  Plain stores of one
+// value per word: no ordering between CTAs or kernels matters and the workspace needs no
+// initialization.
 struct StatusRef {
     unsigned long long *word;
+    unsigned long long *timeout_word;
     unsigned long long tag;     // epoch << 4
-    __device__ __forceinline__ void raise(llmint8_status code) const {
-        atomicMax(word, tag | (unsigned long long)code);
+    __device__ __forceinline__ void set(llmint8_status code) const {
+        *reinterpret_cast<volatile unsigned long long *>(word) = tag | (unsigned long long)code;
+    }
+    __device__ __forceinline__ void timed_out() const {
+        *reinterpret_cast<volatile unsigned long long *>(timeout_word) =
+            tag | (unsigned long long)LLMINT8_ERR_TIMEOUT;
     }
 };
 
@@ -88,7 +97,7 @@ struct BoundedWait {
                 if (*abort_flag) return false;
                 if (global_timer_ns() - t0 > timeout_ns) {
                     *abort_flag = 1;
-                    status.raise(LLMINT8_ERR_TIMEOUT);
+                    status.timed_out();
                     return false;
                 }
             }
@@ -104,7 +113,7 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, Status
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 0u && global_timer_ns() - t0 > kDrainNs) {
-            status.raise(LLMINT8_ERR_TIMEOUT);
+            status.timed_out();
             return false;
         }
     }

@@ -237,7 +237,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 tail->n_out = min(total, a.cap);
                 if (blockIdx.x == 0) {
                     *a.count = total;
-                    a.status.raise(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
+                    a.status.set(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
                 }
             }
         }

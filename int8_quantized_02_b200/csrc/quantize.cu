@@ -163,7 +163,7 @@ outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t
     }
     if (tid == kCompactThreads - 1) {
         *count_out = pos;
-        status.raise(pos > cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
+        status.set(pos > cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
     }
 }
 
