@@ -115,7 +115,7 @@ def _check_linear(X, W, t, bias=None, keep_fp16=False, cap=None):
     M, K = X.shape
     N = W.shape[0]
     C = torch.empty((M, N), dtype=torch.int32, device="cuda")
-    cap = L.default_max_outliers(K, t) if cap is None else cap
+    cap = L.default_max_outliers(K, t) if cap is None else min(cap, K)
     ws = torch.empty((L.llmint8_linear_workspace_size(M, N, K, cap),), dtype=torch.uint8,
                      device="cuda")
     Y = L.llmint8_linear(dev(X), CB, SCB, bias=None if bias is None else dev(bias),
