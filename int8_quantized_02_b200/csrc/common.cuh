@@ -227,6 +227,16 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return d;
 }
 
+// Order in which a tile walks its k-blocks: rotated by a tile-dependent offset, so that the
+// CTAs streaming different tiles at the same moment read different column ranges of the
+// 2^n-strided weight rows (spreading the requests over the DRAM channels) instead of all
+// hitting the same offset.  Integer accumulation makes the order irrelevant to the result.
+__host__ __device__ __forceinline__ int rotated_kblock(int it, int tile, int kblocks) {
+    const int r = (int)(((unsigned)tile * 7u) % (unsigned)kblocks);
+    const int kb = it + r;
+    return kb >= kblocks ? kb - kblocks : kb;
+}
+
 // Instruction descriptors (kind::i8 and kind::f16), K-major A and B, dense.
 //   bits 4-5 accumulator type (1 = f32, 2 = s32); 7-9 A type; 10-12 B type
 //   (i8: 1 = signed; f16: 0 = fp16); 17-22 N/8; 24-28 M/16.

@@ -139,7 +139,8 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             uint32_t phase = 0, used = 0, last_parity = 0;
             for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
                 const int n0 = tile * DBM;
-                for (int kb = 0; kb < a.kblocks; ++kb) {
+                for (int it = 0; it < a.kblocks; ++it) {
+                    const int kb = rotated_kblock(it, tile, a.kblocks);
                     if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
                     const uint32_t full = smem_addr(&tail->full[stage]);
                     mbar_arrive_expect_tx(full, DSTAGE);
@@ -245,28 +246,34 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         named_barrier(1, PHASE_A_THREADS);
 
         // int8 rows into the swizzled operand; X at the outlier columns into xo
+        float mult[DM];
+#pragma unroll
+        for (int m = 0; m < DM; ++m) {
+            const float amax = tail->sca[m];
+            mult[m] = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+        }
         for (int c = t; c < nchunks; c += PHASE_A_THREADS) {
             const uint32_t fl = tail->flags[c];
+            uint4 v[DM];
+#pragma unroll
+            for (int m = 0; m < DM; ++m)
+                if (m < a.M) v[m] = __ldg(X4 + (int64_t)m * nchunks + c);
 #pragma unroll
             for (int m = 0; m < DM; ++m) {
-                if (m < a.M) {
-                    const float amax = tail->sca[m];
-                    if (amax > 0.0f) {
-                        const float s = __fdiv_rn(127.0f, amax);
-                        float f[8];
-                        unpack8(__ldg(X4 + (int64_t)m * nchunks + c), f);
-                        uint32_t lo = 0, hi = 0;
+                if (m < a.M && mult[m] > 0.0f) {
+                    float f[8];
+                    unpack8(v[m], f);
+                    uint32_t lo = 0, hi = 0;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            int q = 0;
-                            if (!((fl >> e) & 1u))
-                                q = max(-127, min(127, __float2int_rn(__fmul_rn(f[e], s))));
-                            const uint32_t b = (uint32_t)(q & 0xff);
-                            if (e < 4) lo |= b << (8 * e);
-                            else hi |= b << (8 * (e - 4));
-                        }
-                        *reinterpret_cast<uint2 *>(xq + xq_offset(m, c * 8)) = make_uint2(lo, hi);
+                    for (int e = 0; e < 8; ++e) {
+                        int q = 0;
+                        if (!((fl >> e) & 1u))
+                            q = max(-127, min(127, __float2int_rn(__fmul_rn(f[e], mult[m]))));
+                        const uint32_t b = (uint32_t)(q & 0xff);
+                        if (e < 4) lo |= b << (8 * e);
+                        else hi |= b << (8 * (e - 4));
                     }
+                    *reinterpret_cast<uint2 *>(xq + xq_offset(m, c * 8)) = make_uint2(lo, hi);
                 }
             }
         }
@@ -290,7 +297,8 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                     tc_fence_after();
                     const uint32_t d = tmem + (uint32_t)(acc * DM);
                     bool ok = true;
-                    for (int kb = 0; kb < a.kblocks; ++kb) {
+                    for (int it = 0; it < a.kblocks; ++it) {
+                        const int kb = rotated_kblock(it, tile, a.kblocks);
                         if (!wait(smem_addr(&tail->full[stage]), phase)) {
                             ok = false;
                             break;
@@ -301,7 +309,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
 #pragma unroll
                         for (int k = 0; k < DBK / 32; ++k)
                             mma_i8(d, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
-                                   (kb | k) != 0);
+                                   (it | k) != 0);
                         tc_commit(smem_addr(&tail->empty[stage]));
                         if (++stage == S) {
                             stage = 0;

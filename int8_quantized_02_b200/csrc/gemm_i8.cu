@@ -133,8 +133,9 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const uint32_t sa = smem_addr(smem + stage * STAGE_BYTES);
                     mbar_arrive_expect_tx(full, STAGE_BYTES);
                     if (kb < nkb) {
-                        tma_load_2d(sa, &tmA, kb * BKB, m0, full);
-                        tma_load_2d(sa + A_BYTES, &tmB, kb * BKB, n0, full);
+                        const int kr = rotated_kblock(kb, tile / a.tiles_m, nkb);
+                        tma_load_2d(sa, &tmA, kr * BKB, m0, full);
+                        tma_load_2d(sa + A_BYTES, &tmB, kr * BKB, n0, full);
                     } else {
                         const int x = (kb - nkb) * (BKB / 2);
                         tma_load_2d(sa, &tmXo, x, m0, full);

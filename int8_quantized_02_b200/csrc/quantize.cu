@@ -182,10 +182,14 @@ quantize_rows_kernel(const __half *__restrict__ X, int64_t K, const uint32_t *__
     uint4 cache[kCache];
     float amax = 0.0f;
 #pragma unroll
+    for (int i = 0; i < kCache; ++i) {       // issue every load before using any
+        const int64_t c = threadIdx.x + (int64_t)i * kThreads;
+        cache[i] = c < nchunks ? xr[c] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
     for (int i = 0; i < kCache; ++i) {
         const int64_t c = threadIdx.x + (int64_t)i * kThreads;
         if (c < nchunks) {
-            cache[i] = xr[c];
             const uint32_t skip = (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu;
             float f[8];
             unpack8(cache[i], f);
@@ -267,10 +271,14 @@ quantize_weight_kernel(const __half *__restrict__ W, int64_t K, int8_t *__restri
     uint4 cache[kCache];
     float amax = 0.0f;
 #pragma unroll
+    for (int i = 0; i < kCache; ++i) {       // issue every load before using any
+        const int64_t c = threadIdx.x + (int64_t)i * kThreads;
+        cache[i] = c < nchunks ? wr[c] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
     for (int i = 0; i < kCache; ++i) {
         const int64_t c = threadIdx.x + (int64_t)i * kThreads;
         if (c < nchunks) {
-            cache[i] = wr[c];
             float f[8];
             unpack8(cache[i], f);
 #pragma unroll
