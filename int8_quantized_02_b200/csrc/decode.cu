@@ -2,15 +2,17 @@
 //
 // At decode sizes the layer is bound by streaming the int8 weight CB from HBM once, so the
 // whole method runs in one kernel that never stops the weight stream:
-//   warp 0        TMA producer: from the first cycle streams 128-row x 128-byte tiles of CB
-//                 (16 KB) through a ring of shared-memory stages;
-//   warps 1..7    meanwhile quantize X for this CTA (every CTA redundantly; X is a few
-//                 hundred KB at most and stays in L2): per 8-column chunk one thread sees all
-//                 rows, so it knows which of its columns are outliers (|x| >= threshold in
-//                 any row) and the row maxima over its regular columns; block-wide maxima
-//                 give SCA; the int8 rows are written straight into shared memory in the
-//                 128-byte-swizzled K-major layout the tensor core reads, outlier columns 0;
-//   warp 1        then issues tcgen05.mma kind::i8 with the weight tile as the 128-row
+//   all warps     first quantize X for this CTA (every CTA redundantly; X is a few hundred
+//                 KB at most and stays in L2): per 8-column chunk one thread sees all rows,
+//                 so it knows which of its columns are outliers (|x| >= threshold in any row)
+//                 and the row maxima over its regular columns; block-wide maxima give SCA;
+//                 the int8 rows are written straight into shared memory in the
+//                 128-byte-swizzled K-major layout the tensor core reads, outlier columns 0.
+//                 This runs before the weight stream starts: started together, the X loads
+//                 queue behind every SM's weight requests and take several times longer;
+//   warp 0        TMA producer: streams 128-row x 128-byte tiles of CB (16 KB) through a
+//                 ring of shared-memory stages;
+//   warp 1        issues tcgen05.mma kind::i8 with the weight tile as the 128-row
 //                 operand and the quantized X (padded to 16 rows) as the 16-column operand:
 //                 D[n, m] = sum_k CB[n, k] * Xq[m, k] into a 128 x 16 int32 TMEM
 //                 accumulator (double-buffered over tiles);
@@ -40,7 +42,6 @@ constexpr int DTHREADS = 256;
 constexpr int DMAX_STAGES = 12;
 constexpr int DCAP = kDecodeMaxOutliers;
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
-constexpr int PHASE_A_THREADS = DTHREADS - 32;
 
 struct DTail {
     uint64_t full[DMAX_STAGES];
@@ -109,9 +110,17 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     DTail *tail = reinterpret_cast<DTail *>(smem + a.tail_off);
     uint8_t *xq = smem + a.xq_off;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = threadIdx.x;
     const int S = a.stages;
+    const int nchunks = a.K / 8;
+    const int kpad = a.kblocks * DBK;
+    const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
+    // While the quantization below runs, the stage buffers are idle: X is kept there when it
+    // fits ([row][chunk] of 16-byte chunks), so the second pass reads shared memory.
+    uint4 *stash = reinterpret_cast<uint4 *>(smem);
+    const bool stashed = (int64_t)a.M * a.K * 2 <= (int64_t)S * DSTAGE;
 
-    if (threadIdx.x == 0) {
+    if (t == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(smem_addr(&tail->full[s]), 1);
             mbar_init(smem_addr(&tail->empty[s]), 1);
@@ -123,57 +132,28 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         mbar_init(smem_addr(&tail->mma_done), 1);
         tail->abort_flag = 0;
         fence_mbar_init();
+        tma_prefetch_desc(&tmCB);
     }
+    if (t < DM) tail->rowmax[t] = 0u;
     if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), 32);
+    // zero the operand (rows >= M and columns >= K must read as 0)
+    for (int i = t; i < kpad * DM / 16; i += DTHREADS)
+        reinterpret_cast<uint4 *>(xq)[i] = make_uint4(0, 0, 0, 0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tail->tmem_base;
     const BoundedWait wait{&tail->abort_flag, a.status, a.timeout_ns};
 
-    if (warp == 0) {
-        // --------------------------------------------------- weight stream (TMA) ----
-        if (lane == 0) {
-            tma_prefetch_desc(&tmCB);
-            int stage = 0;
-            uint32_t phase = 0, used = 0, last_parity = 0;
-            for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
-                const int n0 = tile * DBM;
-                for (int it = 0; it < a.kblocks; ++it) {
-                    const int kb = rotated_kblock(it, tile, a.kblocks);
-                    if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
-                    const uint32_t full = smem_addr(&tail->full[stage]);
-                    mbar_arrive_expect_tx(full, DSTAGE);
-                    tma_load_2d(smem_addr(smem + stage * DSTAGE), &tmCB, kb * DBK, n0, full);
-                    used |= 1u << stage;
-                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-                    if (++stage == S) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
-                }
-            }
-        drain:
-            for (int s = 0; s < S; ++s)
-                if (used & (1u << s))
-                    drain_wait(smem_addr(&tail->full[s]), (last_parity >> s) & 1u, a.status);
-        }
-    } else {
-        // ----------------------------------------- phase A: quantize X in this CTA ----
-        const int t = threadIdx.x - 32;               // 0 .. PHASE_A_THREADS-1
-        const int kpad = a.kblocks * DBK;
-        // zero the operand (rows >= M and columns >= K must read as 0)
-        for (int i = t; i < kpad * DM / 16; i += PHASE_A_THREADS)
-            reinterpret_cast<uint4 *>(xq)[i] = make_uint4(0, 0, 0, 0);
-        if (t < DM) tail->rowmax[t] = 0u;
-        named_barrier(1, PHASE_A_THREADS);
-
-        const int nchunks = a.K / 8;
-        const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
+    // ---------------- phase A: quantize X in this CTA, before the weight stream starts ----
+    // (its loads would otherwise queue behind the weight requests of every SM)
+    {
+        // pass 1: per 8-column chunk one thread sees every row -> outlier bits of its
+        // columns and the row maxima over its regular columns
         float rmax[DM];
 #pragma unroll
         for (int m = 0; m < DM; ++m) rmax[m] = 0.0f;
-        for (int c = t; c < nchunks; c += PHASE_A_THREADS) {
+        for (int c = t; c < nchunks; c += DTHREADS) {
             uint4 v[DM];
 #pragma unroll
             for (int m = 0; m < DM; ++m)
@@ -187,6 +167,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         fl |= (fabsf(f[e]) >= a.threshold ? 1u : 0u) << e;
+                    if (stashed) stash[m * nchunks + c] = v[m];
                 }
             }
 #pragma unroll
@@ -208,7 +189,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             for (int o = 16; o > 0; o >>= 1) r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, o));
             if (lane == 0 && m < a.M) atomicMax(&tail->rowmax[m], __float_as_uint(r));
         }
-        named_barrier(1, PHASE_A_THREADS);
+        __syncthreads();
 
         // ascending outlier list (one warp), its count, and the device status of the call
         if (warp == 1) {
@@ -243,21 +224,22 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             }
         }
         if (t < DM) tail->sca[t] = __uint_as_float(tail->rowmax[t]);
-        named_barrier(1, PHASE_A_THREADS);
+        __syncthreads();
 
-        // int8 rows into the swizzled operand; X at the outlier columns into xo
+        // pass 2: int8 rows into the swizzled operand; X at the outlier columns into xo
         float mult[DM];
 #pragma unroll
         for (int m = 0; m < DM; ++m) {
             const float amax = tail->sca[m];
             mult[m] = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
         }
-        for (int c = t; c < nchunks; c += PHASE_A_THREADS) {
+        for (int c = t; c < nchunks; c += DTHREADS) {
             const uint32_t fl = tail->flags[c];
             uint4 v[DM];
 #pragma unroll
             for (int m = 0; m < DM; ++m)
-                if (m < a.M) v[m] = __ldg(X4 + (int64_t)m * nchunks + c);
+                if (m < a.M)
+                    v[m] = stashed ? stash[m * nchunks + c] : __ldg(X4 + (int64_t)m * nchunks + c);
 #pragma unroll
             for (int m = 0; m < DM; ++m) {
                 if (m < a.M && mult[m] > 0.0f) {
@@ -278,106 +260,135 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             }
         }
         const int n_out = tail->n_out;
-        for (int i = t; i < n_out * DM; i += PHASE_A_THREADS) {
+        for (int i = t; i < n_out * DM; i += DTHREADS) {
             const int j = i / DM, m = i % DM;
             tail->xo[i] = m < a.M ? a.X[(int64_t)m * a.K + tail->idx[j]] : __float2half_rn(0.f);
         }
+        // generic-proxy writes (xq, and the stash about to be overwritten by TMA) must be
+        // ordered before the async proxy touches that shared memory
         fence_proxy_async_smem();
-        named_barrier(1, PHASE_A_THREADS);
+        __syncthreads();
+    }
+    const int n_out = tail->n_out;
 
-        if (warp == 1) {
-            // ------------------------------------------------------------- MMA issue ----
-            if (lane == 0) {
-                const uint32_t idesc = idesc_i8(DBM, DM);
-                const uint32_t xq_base = smem_addr(xq);
-                int stage = 0, acc = 0;
-                uint32_t phase = 0, acc_phase = 0;
-                for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
-                    if (!wait(smem_addr(&tail->acc_empty[acc]), acc_phase ^ 1)) break;
-                    tc_fence_after();
-                    const uint32_t d = tmem + (uint32_t)(acc * DM);
-                    bool ok = true;
-                    for (int it = 0; it < a.kblocks; ++it) {
-                        const int kb = rotated_kblock(it, tile, a.kblocks);
-                        if (!wait(smem_addr(&tail->full[stage]), phase)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t sa = smem_addr(smem + stage * DSTAGE);
-                        const uint32_t sb = xq_base + (uint32_t)(kb * DM * 128);
-#pragma unroll
-                        for (int k = 0; k < DBK / 32; ++k)
-                            mma_i8(d, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
-                                   (it | k) != 0);
-                        tc_commit(smem_addr(&tail->empty[stage]));
-                        if (++stage == S) {
-                            stage = 0;
-                            phase ^= 1;
-                        }
-                    }
-                    if (!ok) break;
-                    tc_commit(smem_addr(&tail->acc_full[acc]));
-                    acc ^= 1;
-                    if (acc == 0) acc_phase ^= 1;
-                }
-                tc_commit(smem_addr(&tail->mma_done));
-                drain_wait(smem_addr(&tail->mma_done), 0, a.status);
-            }
-        } else if (warp >= 4) {
-            // -------------------------------------------------------------- epilogue ----
-            const int q = warp & 3;
-            const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-            const float inv = 1.0f / 16129.0f;
-            int acc = 0;
-            uint32_t acc_phase = 0;
+    if (warp == 0) {
+        // --------------------------------------------------- weight stream (TMA) ----
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, used = 0, last_parity = 0;
             for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
-                int ok = 0;
-                if (lane == 0) ok = wait(smem_addr(&tail->acc_full[acc]), acc_phase) ? 1 : 0;
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
+                const int n0 = tile * DBM;
+                for (int it = 0; it < a.kblocks; ++it) {
+                    const int kb = rotated_kblock(it, tile, a.kblocks);
+                    if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
+                    const uint32_t full = smem_addr(&tail->full[stage]);
+                    mbar_arrive_expect_tx(full, DSTAGE);
+                    tma_load_2d(smem_addr(smem + stage * DSTAGE), &tmCB, kb * DBK, n0, full);
+                    used |= 1u << stage;
+                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+        drain:
+            for (int s = 0; s < S; ++s)
+                if (used & (1u << s))
+                    drain_wait(smem_addr(&tail->full[s]), (last_parity >> s) & 1u, a.status);
+        }
+    } else if (warp == 1) {
+        // ----------------------------------------------------------------- MMA issue ----
+        if (lane == 0) {
+            const uint32_t idesc = idesc_i8(DBM, DM);
+            const uint32_t xq_base = smem_addr(xq);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
+                if (!wait(smem_addr(&tail->acc_empty[acc]), acc_phase ^ 1)) break;
                 tc_fence_after();
-                uint32_t d[DM];
-                tmem_ld_32x16(tl + (uint32_t)(acc * DM), d);
-                tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&tail->acc_empty[acc]));
+                const uint32_t d = tmem + (uint32_t)(acc * DM);
+                bool ok = true;
+                for (int it = 0; it < a.kblocks; ++it) {
+                    const int kb = rotated_kblock(it, tile, a.kblocks);
+                    if (!wait(smem_addr(&tail->full[stage]), phase)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_addr(smem + stage * DSTAGE);
+                    const uint32_t sb = xq_base + (uint32_t)(kb * DM * 128);
+#pragma unroll
+                    for (int k = 0; k < DBK / 32; ++k)
+                        mma_i8(d, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
+                               (it | k) != 0);
+                    tc_commit(smem_addr(&tail->empty[stage]));
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(smem_addr(&tail->acc_full[acc]));
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
+            }
+            tc_commit(smem_addr(&tail->mma_done));
+            drain_wait(smem_addr(&tail->mma_done), 0, a.status);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------------ epilogue ----
+        const int q = warp & 3;
+        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+        const float inv = 1.0f / 16129.0f;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
+            int ok = 0;
+            if (lane == 0) ok = wait(smem_addr(&tail->acc_full[acc]), acc_phase) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t d[DM];
+            tmem_ld_32x16(tl + (uint32_t)(acc * DM), d);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&tail->acc_empty[acc]));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
 
-                const int n = tile * DBM + q * 32 + lane;
-                if (n < a.N) {
-                    const float sb = a.SCB[n];
-                    const float b = a.bias ? __half2float(a.bias[n]) : 0.0f;
-                    float o[DM];
+            const int n = tile * DBM + q * 32 + lane;
+            if (n < a.N) {
+                const float sb = a.SCB[n];
+                const float b = a.bias ? __half2float(a.bias[n]) : 0.0f;
+                float o[DM];
 #pragma unroll
-                    for (int m = 0; m < DM; ++m) o[m] = 0.0f;
-                    const int8_t *cbrow = a.CB + (int64_t)n * a.K;
-                    for (int j = 0; j < n_out; ++j) {
-                        const int col = tail->idx[j];
-                        const float w = a.W16 ? __half2float(a.W16[(int64_t)n * a.K + col])
-                                              : __half2float(__float2half_rn(__fdiv_rn(
-                                                    __fmul_rn((float)cbrow[col], sb), 127.0f)));
-                        const uint4 *xv = reinterpret_cast<const uint4 *>(tail->xo + j * DM);
-                        const uint4 x0 = xv[0], x1 = xv[1];
-                        float f0[8], f1[8];
-                        unpack8(x0, f0);
-                        unpack8(x1, f1);
+                for (int m = 0; m < DM; ++m) o[m] = 0.0f;
+                const int8_t *cbrow = a.CB + (int64_t)n * a.K;
+                for (int j = 0; j < n_out; ++j) {
+                    const int col = tail->idx[j];
+                    const float w = a.W16 ? __half2float(a.W16[(int64_t)n * a.K + col])
+                                          : __half2float(__float2half_rn(__fdiv_rn(
+                                                __fmul_rn((float)cbrow[col], sb), 127.0f)));
+                    const uint4 *xv = reinterpret_cast<const uint4 *>(tail->xo + j * DM);
+                    const uint4 x0 = xv[0], x1 = xv[1];
+                    float f0[8], f1[8];
+                    unpack8(x0, f0);
+                    unpack8(x1, f1);
 #pragma unroll
-                        for (int m = 0; m < 8; ++m) {
-                            o[m] = fmaf(f0[m], w, o[m]);
-                            o[m + 8] = fmaf(f1[m], w, o[m + 8]);
-                        }
+                    for (int m = 0; m < 8; ++m) {
+                        o[m] = fmaf(f0[m], w, o[m]);
+                        o[m + 8] = fmaf(f1[m], w, o[m + 8]);
                     }
+                }
 #pragma unroll
-                    for (int m = 0; m < DM; ++m) {
-                        if (m < a.M) {
-                            const float y = fmaf((float)(int32_t)d[m], tail->sca[m] * inv * sb,
-                                                 o[m] + b);
-                            a.Y[(int64_t)m * a.N + n] = __float2half_rn(y);
-                            if (a.C_debug) a.C_debug[(int64_t)m * a.N + n] = (int32_t)d[m];
-                        }
+                for (int m = 0; m < DM; ++m) {
+                    if (m < a.M) {
+                        const float y = fmaf((float)(int32_t)d[m], tail->sca[m] * inv * sb,
+                                             o[m] + b);
+                        a.Y[(int64_t)m * a.N + n] = __float2half_rn(y);
+                        if (a.C_debug) a.C_debug[(int64_t)m * a.N + n] = (int32_t)d[m];
                     }
                 }
             }
