@@ -81,6 +81,12 @@ T *at(void *ws, size_t off) {
     return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
 }
 
+// Profile events become real event-record nodes when the call is captured into a CUDA
+// graph (a plain record inside stream capture only expresses a dependency).
+cudaError_t record_profile_event(cudaEvent_t ev, cudaStream_t s) {
+    return cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+}
+
 llmint8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA; }
 
 // The single-launch decode kernel covers few activation rows and an X that fits in shared
@@ -218,10 +224,10 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
         d.cap = max_outliers;
         d.threshold = threshold;
         d.timeout_ns = g_timeout_ns.load();
-        if (ev0 && cudaEventRecord(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+        if (ev0 && record_profile_event(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
         e = launch_decode(d, s);
         if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-        if (ev1 && cudaEventRecord(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+        if (ev1 && record_profile_event(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
         return LLMINT8_OK;
     }
 
@@ -261,10 +267,10 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     g.N = N;
     g.K = K;
     g.timeout_ns = g_timeout_ns.load();
-    if (ev0 && cudaEventRecord(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (ev0 && record_profile_event(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
     e = launch_gemm(g, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-    if (ev1 && cudaEventRecord(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (ev1 && record_profile_event(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
     return LLMINT8_OK;
 }
 

@@ -55,6 +55,8 @@ struct DTail {
     int n_total;                         // outlier columns found
     uint32_t rowmax[DM];                 // float bits (non-negative: int order == float order)
     float sca[DM];
+    float mult[DM];                      // fl32(127 / sca), 0 for an all-zero row
+    uint64_t xbar;                       // completion of the bulk copies of X
     uint8_t flags[kDecodeMaxK / 8];      // per 8-column chunk: outlier bit per column
     int32_t idx[DCAP];                   // outlier columns (ascending)
     alignas(16) __half xo[DCAP * DM];    // X at the outlier columns, [j][m] (read as uint4)
@@ -62,6 +64,7 @@ struct DTail {
 
 static_assert(offsetof(DTail, xo) % 16 == 0, "xo is read with 16-byte loads");
 static_assert(offsetof(DTail, full) % 8 == 0, "mbarriers are 8-byte aligned");
+static_assert(offsetof(DTail, xbar) % 8 == 0, "mbarriers are 8-byte aligned");
 
 struct DArgs {
     const __half *X;
@@ -76,6 +79,7 @@ struct DArgs {
     int M, N, K, cap;
     float threshold;
     int stages;
+    int kslice;                          // columns of X per bulk-copied slice
     int kblocks;
     int tiles;
     uint32_t xq_off;                     // byte offset of the quantized X in shared memory
@@ -112,13 +116,12 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = threadIdx.x;
     const int S = a.stages;
-    const int nchunks = a.K / 8;
     const int kpad = a.kblocks * DBK;
-    const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
-    // While the quantization below runs, the stage buffers are idle: X is kept there when it
-    // fits ([row][chunk] of 16-byte chunks), so the second pass reads shared memory.
-    uint4 *stash = reinterpret_cast<uint4 *>(smem);
-    const bool stashed = (int64_t)a.M * a.K * 2 <= (int64_t)S * DSTAGE;
+    // While the quantization below runs the stage buffers are idle: X is brought there by
+    // bulk copies, a column slice of all rows at a time ([row][column] fp16).
+    __half *stash = reinterpret_cast<__half *>(smem);
+    const int ks = a.kslice;                           // columns per slice (multiple of 128)
+    const int nslices = (a.K + ks - 1) / ks;
 
     if (t == 0) {
         for (int s = 0; s < S; ++s) {
@@ -130,6 +133,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             mbar_init(smem_addr(&tail->acc_empty[s]), 4);
         }
         mbar_init(smem_addr(&tail->mma_done), 1);
+        mbar_init(smem_addr(&tail->xbar), 1);
         tail->abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmCB);
@@ -144,130 +148,157 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     tc_fence_after();
     const uint32_t tmem = tail->tmem_base;
     const BoundedWait wait{&tail->abort_flag, a.status, a.timeout_ns};
+    uint32_t xphase = 0;
+    bool x_ok = true;
+
+    // Copies columns [k0, k0 + width) of every row of X into the stash (one thread issues,
+    // everyone waits).  Returns false if the copy did not land in time.
+    auto load_slice = [&](int k0, int width) -> bool {
+        if (t == 0) {
+            const uint32_t bar = smem_addr(&tail->xbar);
+            mbar_arrive_expect_tx(bar, (uint32_t)(a.M * width * 2));
+            for (int m = 0; m < a.M; ++m)
+                bulk_load_1d(smem_addr(stash + m * ks), a.X + (int64_t)m * a.K + k0,
+                             (uint32_t)(width * 2), bar);
+        }
+        int ok = 0;
+        if (t == 0) ok = wait(smem_addr(&tail->xbar), xphase) ? 1 : 0;
+        xphase ^= 1;
+        return __syncthreads_or(ok) != 0;
+    };
 
     // ---------------- phase A: quantize X in this CTA, before the weight stream starts ----
-    // (its loads would otherwise queue behind the weight requests of every SM)
-    {
-        // pass 1: per 8-column chunk one thread sees every row -> outlier bits of its
-        // columns and the row maxima over its regular columns
-        float rmax[DM];
-#pragma unroll
-        for (int m = 0; m < DM; ++m) rmax[m] = 0.0f;
-        for (int c = t; c < nchunks; c += DTHREADS) {
-            uint4 v[DM];
-#pragma unroll
-            for (int m = 0; m < DM; ++m)
-                if (m < a.M) v[m] = __ldg(X4 + (int64_t)m * nchunks + c);
+    // (its loads would otherwise queue behind the weight requests of every SM).  Compact,
+    // rolled loops: this code runs once per CTA, so its size is paid in instruction fetch.
+    for (int sl = 0; sl < nslices && x_ok; ++sl) {
+        const int k0 = sl * ks, width = min(ks, a.K - k0), wchunks = width / 8;
+        x_ok = load_slice(k0, width);
+        if (!x_ok) break;
+        // pass 1a: outlier bits of each 8-column chunk (a column is an outlier when any
+        // row has |x| >= threshold)
+        for (int c = t; c < wchunks; c += DTHREADS) {
             uint32_t fl = 0;
+            for (int m = 0; m < a.M; ++m) {
+                float f[8];
+                unpack8(*reinterpret_cast<const uint4 *>(stash + m * ks + c * 8), f);
 #pragma unroll
-            for (int m = 0; m < DM; ++m) {
-                if (m < a.M) {
-                    float f[8];
-                    unpack8(v[m], f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        fl |= (fabsf(f[e]) >= a.threshold ? 1u : 0u) << e;
-                    if (stashed) stash[m * nchunks + c] = v[m];
-                }
+                for (int e = 0; e < 8; ++e) fl |= (fabsf(f[e]) >= a.threshold ? 1u : 0u) << e;
             }
-#pragma unroll
-            for (int m = 0; m < DM; ++m) {
-                if (m < a.M) {
-                    float f[8];
-                    unpack8(v[m], f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        if (!((fl >> e) & 1u)) rmax[m] = fmaxf(rmax[m], fabsf(f[e]));
-                }
-            }
-            tail->flags[c] = (uint8_t)fl;
+            tail->flags[k0 / 8 + c] = (uint8_t)fl;
         }
+        __syncthreads();
+        // pass 1b: row maxima over the regular columns
+        for (int m = 0; m < a.M; ++m) {
+            float r = 0.0f;
+            for (int c = t; c < wchunks; c += DTHREADS) {
+                const uint32_t fl = tail->flags[k0 / 8 + c];
+                float f[8];
+                unpack8(*reinterpret_cast<const uint4 *>(stash + m * ks + c * 8), f);
 #pragma unroll
-        for (int m = 0; m < DM; ++m) {
-            float r = rmax[m];
+                for (int e = 0; e < 8; ++e)
+                    if (!((fl >> e) & 1u)) r = fmaxf(r, fabsf(f[e]));
+            }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, o));
-            if (lane == 0 && m < a.M) atomicMax(&tail->rowmax[m], __float_as_uint(r));
+            if (lane == 0) atomicMax(&tail->rowmax[m], __float_as_uint(r));
         }
+        fence_proxy_async_smem();   // the next slice's copy overwrites what was just read
         __syncthreads();
+    }
 
-        // ascending outlier list (one warp), its count, and the device status of the call
-        if (warp == 1) {
-            const int per = (nchunks + 31) / 32;
-            const int c0 = lane * per;
-            int cnt = 0;
-            for (int c = c0; c < min(nchunks, c0 + per); ++c) cnt += __popc(tail->flags[c]);
-            int incl = cnt;
+    // ascending outlier list (one warp), its count, and the device status of the call
+    const int nchunks_all = a.K / 8;
+    if (warp == 1) {
+        const int per = (nchunks_all + 31) / 32;
+        const int c0 = lane * per, c1 = min(nchunks_all, c0 + per);
+        int cnt = 0;
+        for (int c = c0; c < c1; ++c) cnt += __popc(tail->flags[c]);
+        int incl = cnt;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            int pos = incl - cnt;
-            for (int c = c0; c < min(nchunks, c0 + per); ++c) {
-                uint32_t fl = tail->flags[c];
-                while (fl) {
-                    const int e = __ffs(fl) - 1;
-                    fl &= fl - 1;
-                    if (pos < a.cap) tail->idx[pos] = c * 8 + e;
-                    ++pos;
-                }
-            }
-            const int total = __shfl_sync(0xffffffffu, incl, 31);
-            if (lane == 0) {
-                tail->n_total = total;
-                tail->n_out = min(total, a.cap);
-                if (blockIdx.x == 0) {
-                    *a.count = total;
-                    a.status.set(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
-                }
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int pos = incl - cnt;
+        for (int c = c0; c < c1; ++c) {
+            uint32_t fl = tail->flags[c];
+            while (fl) {
+                const int e = __ffs(fl) - 1;
+                fl &= fl - 1;
+                if (pos < a.cap) tail->idx[pos] = c * 8 + e;
+                ++pos;
             }
         }
-        if (t < DM) tail->sca[t] = __uint_as_float(tail->rowmax[t]);
-        __syncthreads();
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        if (lane == 0) {
+            tail->n_total = total;
+            tail->n_out = min(total, a.cap);
+            if (blockIdx.x == 0) {
+                *a.count = total;
+                a.status.set(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
+            }
+        }
+    }
+    if (t < DM) {
+        const float amax = __uint_as_float(tail->rowmax[t]);
+        tail->sca[t] = amax;
+        tail->mult[t] = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    }
+    __syncthreads();
 
-        // pass 2: int8 rows into the swizzled operand; X at the outlier columns into xo
-        float mult[DM];
-#pragma unroll
-        for (int m = 0; m < DM; ++m) {
-            const float amax = tail->sca[m];
-            mult[m] = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    // pass 2: int8 rows into the swizzled operand (the last slice is still in the stash)
+    for (int sl = nslices - 1; sl >= 0 && x_ok; --sl) {
+        const int k0 = sl * ks, width = min(ks, a.K - k0), wchunks = width / 8;
+        if (sl != nslices - 1) {
+            fence_proxy_async_smem();
+            __syncthreads();
+            x_ok = load_slice(k0, width);
+            if (!x_ok) break;
         }
-        for (int c = t; c < nchunks; c += DTHREADS) {
-            const uint32_t fl = tail->flags[c];
-            uint4 v[DM];
+        for (int i = t; i < a.M * wchunks; i += DTHREADS) {
+            const int m = i / wchunks, c = i - m * wchunks;
+            const float mul = tail->mult[m];
+            if (mul > 0.0f) {
+                const uint32_t fl = tail->flags[k0 / 8 + c];
+                float f[8];
+                unpack8(*reinterpret_cast<const uint4 *>(stash + m * ks + c * 8), f);
+                uint32_t lo = 0, hi = 0;
 #pragma unroll
-            for (int m = 0; m < DM; ++m)
-                if (m < a.M)
-                    v[m] = stashed ? stash[m * nchunks + c] : __ldg(X4 + (int64_t)m * nchunks + c);
-#pragma unroll
-            for (int m = 0; m < DM; ++m) {
-                if (m < a.M && mult[m] > 0.0f) {
-                    float f[8];
-                    unpack8(v[m], f);
-                    uint32_t lo = 0, hi = 0;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        int q = 0;
-                        if (!((fl >> e) & 1u))
-                            q = max(-127, min(127, __float2int_rn(__fmul_rn(f[e], mult[m]))));
-                        const uint32_t b = (uint32_t)(q & 0xff);
-                        if (e < 4) lo |= b << (8 * e);
-                        else hi |= b << (8 * (e - 4));
-                    }
-                    *reinterpret_cast<uint2 *>(xq + xq_offset(m, c * 8)) = make_uint2(lo, hi);
+                for (int e = 0; e < 8; ++e) {
+                    int q = 0;
+                    if (!((fl >> e) & 1u))
+                        q = max(-127, min(127, __float2int_rn(__fmul_rn(f[e], mul))));
+                    const uint32_t b = (uint32_t)(q & 0xff);
+                    if (e < 4) lo |= b << (8 * e);
+                    else hi |= b << (8 * (e - 4));
                 }
+                *reinterpret_cast<uint2 *>(xq + xq_offset(m, k0 + c * 8)) = make_uint2(lo, hi);
             }
         }
+    }
+    {
+        // X at the outlier columns, [j][m]
         const int n_out = tail->n_out;
         for (int i = t; i < n_out * DM; i += DTHREADS) {
             const int j = i / DM, m = i % DM;
             tail->xo[i] = m < a.M ? a.X[(int64_t)m * a.K + tail->idx[j]] : __float2half_rn(0.f);
         }
-        // generic-proxy writes (xq, and the stash about to be overwritten by TMA) must be
-        // ordered before the async proxy touches that shared memory
-        fence_proxy_async_smem();
+    }
+    // generic-proxy writes (xq) and reads (the stash, about to be overwritten by TMA) must
+    // be ordered before the async proxy touches that shared memory
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (!x_ok) {
+        // the copy of X timed out (already recorded): nothing valid to compute; let the
+        // copy in flight land before the CTA exits
+        if (t == 0) drain_wait(smem_addr(&tail->xbar), xphase ^ 1, a.status);
+        tc_fence_before();
         __syncthreads();
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc(tmem, 32);
+        }
+        return;
     }
     const int n_out = tail->n_out;
 
@@ -464,6 +495,13 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     const int stages = (int)std::min<int64_t>(DMAX_STAGES, room / DSTAGE);
     if (stages < 2) return cudaErrorInvalidValue;
     a.stages = stages;
+    {
+        // X is brought into the idle stage buffers a column slice of all rows at a time
+        const int64_t per_col = 2 * d.M;
+        int64_t ks = (int64_t)stages * DSTAGE / per_col;
+        a.kslice = (int)(ks >= d.K ? d.K : ks / 128 * 128);
+        if (a.kslice < 128 && a.kslice < d.K) return cudaErrorInvalidValue;
+    }
     a.xq_off = (uint32_t)(stages * DSTAGE);
     a.tail_off = a.xq_off + xq_bytes;
     const int smem = (int)(a.tail_off + sizeof(DTail) + 1024);
