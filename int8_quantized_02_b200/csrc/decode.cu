@@ -540,10 +540,10 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     a.tiles = (int)ceil_div(d.N, DBM);
     a.own_cols = (int)align_up(ceil_div(d.K, CL), 32);
     a.timeout_ns = d.timeout_ns;
-    // the largest shared-memory plan sizes the attribute and the occupancy query once
+    // every plan fits in SMEM_LIMIT, which sizes the attribute and the occupancy query once
     const Shape worst = plan_smem(kDecodeMaxK / DBK, kMaxOwnCols);
     const Shape sh = plan_smem(a.kblocks, a.own_cols);
-    if (worst.stages < 2 || sh.stages < 2 || a.own_cols > kMaxOwnCols)
+    if (worst.stages < 2 || sh.stages < 2 || a.own_cols > kMaxOwnCols || sh.smem > SMEM_LIMIT)
         return cudaErrorInvalidValue;
     a.stages = sh.stages;
     a.xq_off = sh.xq_off;
@@ -566,11 +566,11 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
         std::lock_guard<std::mutex> lk(mu);
         if (max_clusters[dev] == 0) {
             err = cudaFuncSetAttribute(llmint8_decode_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, worst.smem);
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT);
             if (err != cudaSuccess) return err;
             cudaLaunchConfig_t qc = cfg;
             qc.gridDim = dim3(CL);
-            qc.dynamicSmemBytes = (size_t)worst.smem;
+            qc.dynamicSmemBytes = (size_t)SMEM_LIMIT;
             int n = 0;
             err = cudaOccupancyMaxActiveClusters(&n, llmint8_decode_kernel, &qc);
             if (err != cudaSuccess) return err;
