@@ -164,6 +164,9 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, const uint4 &v) {
 __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+__device__ __forceinline__ void st_cluster_u8(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 __device__ __forceinline__ void st_cluster_u16(uint32_t addr, uint16_t v) {
     asm volatile("st.shared::cluster.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
@@ -192,6 +195,12 @@ __device__ __forceinline__ void cluster_barrier_all() {
     asm volatile(
         "barrier.cluster.arrive.release.aligned;\n\t"
         "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Asks L2 to fetch a contiguous global range (16-byte aligned, size a multiple of 16); no
+// completion to wait for.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // ------------------------------------------------------------------- tcgen05 ----------

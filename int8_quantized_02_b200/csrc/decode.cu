@@ -3,13 +3,17 @@
 // At decode sizes the layer is bound by streaming the int8 weight CB from HBM once, and
 // everything else must hide under that stream.  Two kernels:
 //
-// llmint8_decode_quantize_kernel (one CTA, 1024 threads) quantizes X once: one thread per
-//   (row, 8-column chunk), so that each warp holds all 16 rows of two chunks.  The outlier
-//   bits of a chunk (|x| >= threshold in any row) are an OR across 16 lanes; the row maxima
-//   over the regular columns reduce in registers and then across warps; the int8 codes go
-//   into the workspace as a byte-exact image of the tensor-core operand (16 rows, 128-byte
-//   swizzled K-major blocks, outlier columns and padding 0), next to a table of SCA, the
-//   ascending outlier columns and X at those columns.  It lets its dependent launch at once.
+// llmint8_decode_quantize_kernel (one cluster of 8 CTAs x 1024 threads) quantizes X once:
+//   one thread per (row, 8-column chunk), each warp holding all 16 rows of two chunks, CTA r
+//   of the cluster 1/8 of the columns.  The outlier bits of a chunk (|x| >= threshold in any
+//   row) are an OR across 16 lanes; the row maxima over the regular columns reduce in
+//   registers, across warps, and across the cluster through distributed shared memory
+//   (one hardware cluster barrier); the int8 codes go into the workspace as a byte-exact
+//   image of the tensor-core operand (16 rows, 128-byte swizzled K-major blocks, outlier
+//   columns and padding 0), next to a table of SCA, the ascending outlier columns and X at
+//   those columns.  It lets its dependent launch at once, and first asks L2 to pull in the
+//   weight bytes, so that HBM streams CB from the first microsecond: every byte is still
+//   read from HBM once per call, the dependent's TMA then finds it in L2.
 //
 // llmint8_decode_kernel (one CTA per 128-row weight tile, programmatic dependent launch):
 //   warp 0        TMA producer: streams 128-row x 128-byte tiles of CB (16 KB) through a ring
@@ -43,9 +47,12 @@ constexpr int DSTAGE = DBM * DBK;       // 16 KB
 constexpr int DTHREADS = 256;
 constexpr int DMAX_STAGES = 12;
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
-constexpr int QTHREADS = 1024;          // quantize kernel
+constexpr int QTHREADS = 1024;          // quantize kernel: one cluster of QCL CTAs
 constexpr int QWARPS = QTHREADS / 32;
-constexpr int QKEEP = 8;                // chunk pairs per warp kept in registers
+constexpr int QCL = 8;
+// chunk pairs (16 columns) per warp: K <= kDecodeMaxK keeps every item in registers
+constexpr int QKEEP = (kDecodeMaxK / 16 / QCL + QWARPS - 1) / QWARPS;
+constexpr uint32_t kPrefetchLimit = 64u << 20;   // weight bytes pulled into L2 up front
 
 __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&v);
@@ -102,78 +109,116 @@ struct QArgs {
     DecodeTables *tables;
     int32_t *count;
     StatusRef status;
+    const int8_t *CB;                   // weights to start pulling into L2
+    uint32_t prefetch_bytes;
 };
 
+// One cluster of QCL CTAs.  CTA r owns the chunk pairs [r*PP, (r+1)*PP); one thread per
+// (row, chunk) item, its values kept in registers between the two passes.
 __global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(const QArgs a) {
-    // the weight stream of the dependent kernel does not need anything from here
+    // the dependent kernel's weight stream needs nothing from here
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    __shared__ uint32_t rowmax[DM];          // float bits (non-negative: int order = float)
+    __shared__ float part[QCL][DM];          // row maxima of every CTA of the cluster
+    __shared__ uint32_t pmax[DM];            // this CTA's (float bits, >= 0: int order)
     __shared__ float mult[DM];
-    __shared__ uint8_t flags[kDecodeMaxK / 8];
+    __shared__ uint8_t flags_all[kDecodeMaxK / 8];   // CTA 0: outlier bits of every chunk
     __shared__ int n_out_s;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int m = lane & 15;                 // the row this thread handles
     const int half = lane >> 4;              // which chunk of the warp's pair
+    const uint32_t r = cluster_ctarank();
     const int nchunks = a.K / 8;
     const int npairs = nchunks / 2;          // K is a multiple of 16
-    const int img_bytes = (int)decode_image_bytes(a.K);
+    const int pp = (npairs + QCL - 1) / QCL;
+    const int p0 = (int)r * pp, p1 = min(npairs, p0 + pp);
     const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
 
-    for (int i = t; i < img_bytes / 16; i += QTHREADS)
-        reinterpret_cast<uint4 *>(a.image)[i] = make_uint4(0, 0, 0, 0);
-    if (t < DM) rowmax[t] = 0u;
+    uint4 v[QKEEP];
+#pragma unroll
+    for (int i = 0; i < QKEEP; ++i) {
+        const int p = p0 + warp + i * QWARPS;
+        v[i] = (p < p1 && m < a.M) ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
+                                   : make_uint4(0, 0, 0, 0);
+    }
+    if (t == 0 && a.prefetch_bytes) {
+        // this CTA's share of the weight bytes, so that HBM streams from the start
+        constexpr uint32_t kPiece = 65536;
+        const uint32_t share = (a.prefetch_bytes / QCL + 15u) & ~15u;
+        const uint32_t b0 = r * share, b1 = min(a.prefetch_bytes, b0 + share);
+        for (uint32_t off = b0; off < b1; off += kPiece)
+            prefetch_l2_bulk(a.CB + off, min(kPiece, b1 - off));
+    }
+    if (t < DM) pmax[t] = 0u;
     __syncthreads();
 
-    // pass 1: outlier bits (OR over the 16 lanes of a chunk) and row maxima over the regular
-    // columns; the first QKEEP pairs of each warp stay in registers for pass 2
-    uint4 keep[QKEEP];
+    // pass 1: outlier bits of each chunk (OR over its 16 lanes = rows), published to CTA 0;
+    // row maxima over the regular columns
+    uint32_t fl[QKEEP];
     float rm = 0.0f;
+    const uint32_t flags0 = map_to_rank(smem_addr(flags_all), 0);
 #pragma unroll
     for (int i = 0; i < QKEEP; ++i) {
-        const int p = warp + i * QWARPS;
-        const int c = 2 * p + half;
-        keep[i] = (p < npairs && m < a.M) ? __ldg(X4 + (int64_t)m * nchunks + c)
-                                          : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        const int p = warp + i * QWARPS;
-        if (p < npairs) {                    // uniform over the warp
+        fl[i] = 0;
+        const int p = p0 + warp + i * QWARPS;
+        if (p < p1) {                        // uniform over the warp
             float f[8];
-            unpack8(keep[i], f);
-            uint32_t fl = outlier_bits(f, a.threshold);
+            unpack8(v[i], f);
+            uint32_t b = outlier_bits(f, a.threshold);
 #pragma unroll
-            for (int o = 1; o < 16; o <<= 1) fl |= __shfl_xor_sync(0xffffffffu, fl, o);
-            if (m == 0) flags[2 * p + half] = (uint8_t)fl;
-            rm = masked_max(f, fl, rm);
+            for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
+            fl[i] = b;
+            if (m == 0) st_cluster_u8(flags0 + (uint32_t)(2 * p + half), b);
+            rm = masked_max(f, b, rm);
         }
     }
-    for (int p = warp + QKEEP * QWARPS; p < npairs; p += QWARPS) {
-        const int c = 2 * p + half;
-        const uint4 v = m < a.M ? __ldg(X4 + (int64_t)m * nchunks + c) : make_uint4(0, 0, 0, 0);
-        float f[8];
-        unpack8(v, f);
-        uint32_t fl = outlier_bits(f, a.threshold);
-#pragma unroll
-        for (int o = 1; o < 16; o <<= 1) fl |= __shfl_xor_sync(0xffffffffu, fl, o);
-        if (m == 0) flags[c] = (uint8_t)fl;
-        rm = masked_max(f, fl, rm);
-    }
     rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 16));
-    if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&rowmax[m], __float_as_uint(rm));
+    if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&pmax[m], __float_as_uint(rm));
+    __syncthreads();
+    if (t < DM) {
+        const uint32_t dst = smem_addr(&part[r][t]);
+        for (int rr = 0; rr < QCL; ++rr) st_cluster_u32(map_to_rank(dst, (uint32_t)rr), pmax[t]);
+    }
+    // every CTA's flags and partial maxima are in place after this
+    cluster_barrier_all();
+
+    if (t < DM) {
+        float amax = 0.0f;
+        for (int rr = 0; rr < QCL; ++rr) amax = fmaxf(amax, part[rr][t]);
+        mult[t] = (t < a.M && amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
+        if (r == 0) a.tables->sca[t] = amax;
+    }
     __syncthreads();
 
-    // scales; ascending outlier list (warp 0), count and status of the call
-    if (t < DM) {
-        const float amax = __uint_as_float(rowmax[t]);
-        a.tables->sca[t] = amax;
-        mult[t] = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    // pass 2: every (row, chunk) of this CTA into the operand image; rows >= M, all-zero rows
+    // and outlier columns are written as 0
+    const float mul = mult[m];
+#pragma unroll
+    for (int i = 0; i < QKEEP; ++i) {
+        const int p = p0 + warp + i * QWARPS;
+        if (p < p1) {
+            const int c = 2 * p + half;
+            uint2 q = make_uint2(0, 0);
+            if (mul > 0.0f) {
+                float f[8];
+                unpack8(v[i], f);
+                q = quant8(f, mul, fl[i]);
+            }
+            *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8)) = q;
+        }
+    }
+    if (r != 0) return;   // nothing of this CTA is read by its peers any more
+
+    // CTA 0: padding columns of the image, ascending outlier list, count, status, X there
+    const int kpad_chunks = (a.K + 127) / 128 * 16;
+    for (int i = t; i < (kpad_chunks - nchunks) * DM; i += QTHREADS) {
+        const int c = nchunks + i / DM, mm = i % DM;
+        *reinterpret_cast<uint2 *>(a.image + xq_offset(mm, c * 8)) = make_uint2(0, 0);
     }
     if (warp == 0) {
         const int per = (nchunks + 31) / 32;
         const int c0 = lane * per, c1 = min(nchunks, c0 + per);
         int cnt = 0;
-        for (int c = c0; c < c1; ++c) cnt += __popc(flags[c]);
+        for (int c = c0; c < c1; ++c) cnt += __popc(flags_all[c]);
         int incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -182,10 +227,10 @@ __global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(co
         }
         int pos = incl - cnt;
         for (int c = c0; c < c1; ++c) {
-            uint32_t fl = flags[c];
-            while (fl) {
-                const int e = __ffs(fl) - 1;
-                fl &= fl - 1;
+            uint32_t b = flags_all[c];
+            while (b) {
+                const int e = __ffs(b) - 1;
+                b &= b - 1;
                 if (pos < a.cap) a.tables->idx[pos] = c * 8 + e;
                 ++pos;
             }
@@ -199,28 +244,6 @@ __global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(co
         }
     }
     __syncthreads();
-
-    // pass 2: int8 codes into the operand image
-    const float mul = m < a.M ? mult[m] : 0.0f;
-#pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        const int p = warp + i * QWARPS;
-        const int c = 2 * p + half;
-        if (p < npairs && mul > 0.0f) {
-            float f[8];
-            unpack8(keep[i], f);
-            *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8)) = quant8(f, mul, flags[c]);
-        }
-    }
-    for (int p = warp + QKEEP * QWARPS; p < npairs; p += QWARPS) {
-        const int c = 2 * p + half;
-        if (mul > 0.0f) {
-            float f[8];
-            unpack8(__ldg(X4 + (int64_t)m * nchunks + c), f);
-            *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8)) = quant8(f, mul, flags[c]);
-        }
-    }
-    // X at the outlier columns, [j][m]
     const int n_out = n_out_s;
     for (int i = t; i < n_out * DM; i += QTHREADS) {
         const int j = i / DM, mm = i % DM;
@@ -486,10 +509,25 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     q.tables = d.tables;
     q.count = d.count;
     q.status = d.status;
-    llmint8_decode_quantize_kernel<<<1, QTHREADS, 0, s>>>(q);
-    note_launches(1);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
+    q.CB = d.CB;
+    q.prefetch_bytes = (uint32_t)std::min<int64_t>(d.N * d.K, kPrefetchLimit) & ~15u;
+    {
+        cudaLaunchConfig_t qc = {};
+        cudaLaunchAttribute qa[1];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = QCL;
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        qc.gridDim = dim3(QCL);
+        qc.blockDim = dim3(QTHREADS);
+        qc.dynamicSmemBytes = 0;
+        qc.stream = s;
+        qc.attrs = qa;
+        qc.numAttrs = 1;
+        err = cudaLaunchKernelEx(&qc, llmint8_decode_quantize_kernel, q);
+        note_launches(1);
+        if (err != cudaSuccess) return err;
+    }
 
     // 2. the weight-streaming product, allowed to start before step 1 finishes
     DArgs a;
@@ -535,8 +573,8 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    // one SM stays with the quantize kernel while this grid starts
-    cfg.gridDim = dim3((unsigned)std::min(a.tiles, std::max(1, sms - 1)));
+    // QCL SMs stay with the quantize kernel while this grid starts
+    cfg.gridDim = dim3((unsigned)std::min(a.tiles, std::max(1, sms - QCL)));
     cfg.blockDim = dim3(DTHREADS);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = s;
