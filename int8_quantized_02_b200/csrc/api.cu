@@ -90,7 +90,12 @@ T *at(void *ws, size_t off) {
 // Profile events become real event-record nodes when the call is captured into a CUDA
 // graph (a plain record inside stream capture only expresses a dependency).
 cudaError_t record_profile_event(cudaEvent_t ev, cudaStream_t s) {
-    return cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &cs);
+    if (e != cudaSuccess) return e;
+    return cs == cudaStreamCaptureStatusActive
+               ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+               : cudaEventRecord(ev, s);
 }
 
 llmint8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA; }

@@ -197,6 +197,13 @@ __device__ __forceinline__ void cluster_barrier_all() {
         "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Asks L2 to fetch one box of a tensor map (no shared memory, nothing to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *tm, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
 // Asks L2 to fetch a contiguous global range (16-byte aligned, size a multiple of 16); no
 // completion to wait for.
 __device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {

@@ -11,13 +11,14 @@
 //   (one hardware cluster barrier); the int8 codes go into the workspace as a byte-exact
 //   image of the tensor-core operand (16 rows, 128-byte swizzled K-major blocks, outlier
 //   columns and padding 0), next to a table of SCA, the ascending outlier columns and X at
-//   those columns.  It lets its dependent launch at once, and first asks L2 to pull in the
-//   weight bytes, so that HBM streams CB from the first microsecond: every byte is still
-//   read from HBM once per call, the dependent's TMA then finds it in L2.
+//   those columns.  It lets its dependent launch at once.
 //
 // llmint8_decode_kernel (one CTA per 128-row weight tile, programmatic dependent launch):
 //   warp 0        TMA producer: streams 128-row x 128-byte tiles of CB (16 KB) through a ring
-//                 of shared-memory stages from its first cycle - it needs nothing from X;
+//                 of shared-memory stages from its first cycle - it needs nothing from X - and
+//                 asks L2 for the rest of its first tile as well, so that HBM keeps streaming
+//                 while the MMA waits for the quantized X (every weight byte is still read
+//                 from HBM once per call; the later stage loads find it in L2);
 //   warp 1        waits for the quantize kernel (griddepcontrol.wait), bulk-copies the operand
 //                 image and the table into shared memory, then issues tcgen05.mma kind::i8
 //                 with the weight tile as the 128-row operand and the quantized X as the
@@ -52,7 +53,9 @@ constexpr int QWARPS = QTHREADS / 32;
 constexpr int QCL = 8;
 // chunk pairs (16 columns) per warp: K <= kDecodeMaxK keeps every item in registers
 constexpr int QKEEP = (kDecodeMaxK / 16 / QCL + QWARPS - 1) / QWARPS;
-constexpr uint32_t kPrefetchLimit = 64u << 20;   // weight bytes pulled into L2 up front
+// k-blocks of a CTA's first tile requested into L2 ahead of the stage ring, so that HBM keeps
+// streaming while the first MMA waits for the quantized X
+constexpr int kPrefetchBlocks = 64;
 
 __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&v);
@@ -109,8 +112,6 @@ struct QArgs {
     DecodeTables *tables;
     int32_t *count;
     StatusRef status;
-    const int8_t *CB;                   // weights to start pulling into L2
-    uint32_t prefetch_bytes;
 };
 
 // One cluster of QCL CTAs.  CTA r owns the chunk pairs [r*PP, (r+1)*PP); one thread per
@@ -139,14 +140,6 @@ __global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(co
         const int p = p0 + warp + i * QWARPS;
         v[i] = (p < p1 && m < a.M) ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
                                    : make_uint4(0, 0, 0, 0);
-    }
-    if (t == 0 && a.prefetch_bytes) {
-        // this CTA's share of the weight bytes, so that HBM streams from the start
-        constexpr uint32_t kPiece = 65536;
-        const uint32_t share = (a.prefetch_bytes / QCL + 15u) & ~15u;
-        const uint32_t b0 = r * share, b1 = min(a.prefetch_bytes, b0 + share);
-        for (uint32_t off = b0; off < b1; off += kPiece)
-            prefetch_l2_bulk(a.CB + off, min(kPiece, b1 - off));
     }
     if (t < DM) pmax[t] = 0u;
     __syncthreads();
@@ -326,6 +319,13 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 const int n0 = tile * DBM;
                 for (int it = 0; it < a.kblocks; ++it) {
                     const int kb = rotated_kblock(it, tile, a.kblocks);
+                    if (tile == (int)blockIdx.x && it == S) {
+                        // the ring is full: request the rest of this first tile into L2
+                        const int last = min(a.kblocks, S + kPrefetchBlocks);
+                        for (int pf = S; pf < last; ++pf)
+                            tma_prefetch_l2_2d(&tmCB, rotated_kblock(pf, tile, a.kblocks) * DBK,
+                                               n0);
+                    }
                     if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
                     const uint32_t full = smem_addr(&tail->full[stage]);
                     mbar_arrive_expect_tx(full, DSTAGE);
@@ -509,8 +509,6 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     q.tables = d.tables;
     q.count = d.count;
     q.status = d.status;
-    q.CB = d.CB;
-    q.prefetch_bytes = (uint32_t)std::min<int64_t>(d.N * d.K, kPrefetchLimit) & ~15u;
     {
         cudaLaunchConfig_t qc = {};
         cudaLaunchAttribute qa[1];
