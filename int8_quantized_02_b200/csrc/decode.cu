@@ -11,14 +11,14 @@
 //   (one hardware cluster barrier); the int8 codes go into the workspace as a byte-exact
 //   image of the tensor-core operand (16 rows, 128-byte swizzled K-major blocks, outlier
 //   columns and padding 0), next to a table of SCA, the ascending outlier columns and X at
-//   those columns.  It lets its dependent launch at once.
+//   those columns.  It lets its dependent launch at once, and its CTAs (more clusters than
+//   the quantization needs) first ask L2 for the weight bytes, so that HBM streams CB from
+//   the first microsecond while X is quantized: every weight byte is still read from HBM
+//   once per call; the dependent's stage loads find it in L2.
 //
 // llmint8_decode_kernel (one CTA per 128-row weight tile, programmatic dependent launch):
 //   warp 0        TMA producer: streams 128-row x 128-byte tiles of CB (16 KB) through a ring
-//                 of shared-memory stages from its first cycle - it needs nothing from X - and
-//                 asks L2 for the rest of its first tile as well, so that HBM keeps streaming
-//                 while the MMA waits for the quantized X (every weight byte is still read
-//                 from HBM once per call; the later stage loads find it in L2);
+//                 of shared-memory stages from its first cycle - it needs nothing from X;
 //   warp 1        waits for the quantize kernel (griddepcontrol.wait), bulk-copies the operand
 //                 image and the table into shared memory, then issues tcgen05.mma kind::i8
 //                 with the weight tile as the 128-row operand and the quantized X as the
@@ -53,9 +53,7 @@ constexpr int QWARPS = QTHREADS / 32;
 constexpr int QCL = 8;
 // chunk pairs (16 columns) per warp: K <= kDecodeMaxK keeps every item in registers
 constexpr int QKEEP = (kDecodeMaxK / 16 / QCL + QWARPS - 1) / QWARPS;
-// k-blocks of a CTA's first tile requested into L2 ahead of the stage ring, so that HBM keeps
-// streaming while the first MMA waits for the quantized X
-constexpr int kPrefetchBlocks = 64;
+constexpr uint32_t kPrefetchLimit = 64u << 20;   // weight bytes pulled into L2 up front
 
 __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&v);
@@ -112,18 +110,32 @@ struct QArgs {
     DecodeTables *tables;
     int32_t *count;
     StatusRef status;
+    const int8_t *CB;                   // weights to start pulling into L2
+    uint32_t prefetch_bytes;            // multiple of 16
 };
 
-// One cluster of QCL CTAs.  CTA r owns the chunk pairs [r*PP, (r+1)*PP); one thread per
-// (row, chunk) item, its values kept in registers between the two passes.
+// Clusters of QCL CTAs.  Every CTA first asks L2 for its slice of the weight bytes (the
+// slices are spread over many SMs: one SM's copy engine alone would take far longer than
+// HBM needs), then every cluster but the first is done.  In the first cluster CTA r owns
+// the chunk pairs [r*PP, (r+1)*PP); one thread per (row, chunk) item, its values kept in
+// registers between the two passes.
 __global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(const QArgs a) {
     // the dependent kernel's weight stream needs nothing from here
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (threadIdx.x < 32 && a.prefetch_bytes) {
+        constexpr uint32_t kPiece = 16384;
+        const uint32_t share = (a.prefetch_bytes / gridDim.x + 15u) & ~15u;
+        const uint32_t b0 = blockIdx.x * share, b1 = min(a.prefetch_bytes, b0 + share);
+        for (uint32_t off = b0 + threadIdx.x * kPiece; off < b1; off += 32 * kPiece)
+            prefetch_l2_bulk(a.CB + off, min(kPiece, b1 - off));
+    }
+    if (blockIdx.x >= QCL) return;            // a whole cluster leaves together
     __shared__ float part[QCL][DM];          // row maxima of every CTA of the cluster
     __shared__ uint32_t pmax[DM];            // this CTA's (float bits, >= 0: int order)
     __shared__ float mult[DM];
     __shared__ uint8_t flags_all[kDecodeMaxK / 8];   // CTA 0: outlier bits of every chunk
     __shared__ int n_out_s;
+    __shared__ int warp_tot[QWARPS];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int m = lane & 15;                 // the row this thread handles
     const int half = lane >> 4;              // which chunk of the warp's pair
@@ -207,41 +219,50 @@ __global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(co
         const int c = nchunks + i / DM, mm = i % DM;
         *reinterpret_cast<uint2 *>(a.image + xq_offset(mm, c * 8)) = make_uint2(0, 0);
     }
-    if (warp == 0) {
-        const int per = (nchunks + 31) / 32;
-        const int c0 = lane * per, c1 = min(nchunks, c0 + per);
-        int cnt = 0;
-        for (int c = c0; c < c1; ++c) cnt += __popc(flags_all[c]);
+    {
+        // ascending list: one chunk per thread (K/8 <= QTHREADS), block-wide exclusive scan
+        const uint32_t b0 = t < nchunks ? flags_all[t] : 0u;
+        const int cnt = __popc(b0);
         int incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += y;
         }
-        int pos = incl - cnt;
-        for (int c = c0; c < c1; ++c) {
-            uint32_t b = flags_all[c];
-            while (b) {
-                const int e = __ffs(b) - 1;
-                b &= b - 1;
-                if (pos < a.cap) a.tables->idx[pos] = c * 8 + e;
-                ++pos;
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int v0 = warp_tot[lane];
+            int x = v0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            warp_tot[lane] = x - v0;
+            if (lane == 31) {
+                n_out_s = min(x, a.cap);
+                a.tables->n_out = n_out_s;
+                *a.count = x;
+                a.status.set(x > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
             }
         }
-        const int total = __shfl_sync(0xffffffffu, incl, 31);
-        if (lane == 0) {
-            n_out_s = min(total, a.cap);
-            a.tables->n_out = n_out_s;
-            *a.count = total;
-            a.status.set(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
+        __syncthreads();
+        int pos = warp_tot[warp] + incl - cnt;
+        uint32_t b = b0;
+        while (b) {
+            const int e = __ffs(b) - 1;
+            b &= b - 1;
+            if (pos < a.cap) {
+                const int col = t * 8 + e;
+                a.tables->idx[pos] = col;
+                // X at this outlier column, [j][m]
+                for (int mm = 0; mm < DM; ++mm)
+                    a.tables->xo[pos * DM + mm] =
+                        mm < a.M ? a.X[(int64_t)mm * a.K + col] : __float2half_rn(0.0f);
+            }
+            ++pos;
         }
-    }
-    __syncthreads();
-    const int n_out = n_out_s;
-    for (int i = t; i < n_out * DM; i += QTHREADS) {
-        const int j = i / DM, mm = i % DM;
-        a.tables->xo[i] = mm < a.M ? a.X[(int64_t)mm * a.K + a.tables->idx[j]]
-                                   : __float2half_rn(0.0f);
     }
 }
 
@@ -319,13 +340,6 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 const int n0 = tile * DBM;
                 for (int it = 0; it < a.kblocks; ++it) {
                     const int kb = rotated_kblock(it, tile, a.kblocks);
-                    if (tile == (int)blockIdx.x && it == S) {
-                        // the ring is full: request the rest of this first tile into L2
-                        const int last = min(a.kblocks, S + kPrefetchBlocks);
-                        for (int pf = S; pf < last; ++pf)
-                            tma_prefetch_l2_2d(&tmCB, rotated_kblock(pf, tile, a.kblocks) * DBK,
-                                               n0);
-                    }
                     if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
                     const uint32_t full = smem_addr(&tail->full[stage]);
                     mbar_arrive_expect_tx(full, DSTAGE);
@@ -351,7 +365,8 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             const uint32_t xbar = smem_addr(&tail->xbar);
             const uint32_t img_bytes = (uint32_t)(a.kblocks * DBK * DM);
             mbar_arrive_expect_tx(xbar, img_bytes + (uint32_t)sizeof(DecodeTables));
-            bulk_load_1d(smem_addr(xq), a.image, img_bytes, xbar);
+            for (uint32_t off = 0; off < img_bytes; off += 16384)
+                bulk_load_1d(smem_addr(xq) + off, a.image + off, min(16384u, img_bytes - off), xbar);
             bulk_load_1d(smem_addr(&tail->tab), a.tables, (uint32_t)sizeof(DecodeTables), xbar);
             const bool have_x = wait(xbar, 0);
             const uint32_t idesc = idesc_i8(DBM, DM);
@@ -509,6 +524,8 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     q.tables = d.tables;
     q.count = d.count;
     q.status = d.status;
+    q.CB = d.CB;
+    q.prefetch_bytes = (uint32_t)std::min<int64_t>(d.N * d.K, kPrefetchLimit) & ~15u;
     {
         cudaLaunchConfig_t qc = {};
         cudaLaunchAttribute qa[1];
@@ -516,7 +533,11 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
         qa[0].val.clusterDim.x = QCL;
         qa[0].val.clusterDim.y = 1;
         qa[0].val.clusterDim.z = 1;
-        qc.gridDim = dim3(QCL);
+        // the prefetch is spread over ~one CTA per 512 KB of weights
+        const int64_t want = ceil_div((int64_t)q.prefetch_bytes, 512 * 1024);
+        const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(want, QCL),
+                                                                         std::max(1, sms / QCL)));
+        qc.gridDim = dim3((unsigned)(clusters * QCL));
         qc.blockDim = dim3(QTHREADS);
         qc.dynamicSmemBytes = 0;
         qc.stream = s;
