@@ -1,29 +1,24 @@
 // Decode path of the LLM.int8() layer (few activation rows, M <= 16).
 //
-// At decode sizes the layer is bound by streaming the int8 weight CB from HBM once, and
-// everything else must hide under that stream.  Two kernels:
+// At decode sizes the layer is bound by streaming the int8 weight CB from HBM once, and the
+// rest must hide under that stream.  One kernel, one CTA of 512 threads per 128-row weight
+// tile (grid-stride over tiles when there are more tiles than SMs):
 //
-// llmint8_decode_quantize_kernel (one cluster of 8 CTAs x 1024 threads) quantizes X once:
-//   one thread per (row, 8-column chunk), each warp holding all 16 rows of two chunks, CTA r
-//   of the cluster 1/8 of the columns.  The outlier bits of a chunk (|x| >= threshold in any
-//   row) are an OR across 16 lanes; the row maxima over the regular columns reduce in
-//   registers, across warps, and across the cluster through distributed shared memory
-//   (one hardware cluster barrier); the int8 codes go into the workspace as a byte-exact
-//   image of the tensor-core operand (16 rows, 128-byte swizzled K-major blocks, outlier
-//   columns and padding 0), next to a table of SCA, the ascending outlier columns and X at
-//   those columns.  It lets its dependent launch at once, and its CTAs (more clusters than
-//   the quantization needs) first ask L2 for the weight bytes, so that HBM streams CB from
-//   the first microsecond while X is quantized: every weight byte is still read from HBM
-//   once per call; the dependent's stage loads find it in L2.
-//
-// llmint8_decode_kernel (one CTA per 128-row weight tile, programmatic dependent launch):
-//   warp 0        TMA producer: streams 128-row x 128-byte tiles of CB (16 KB) through a ring
-//                 of shared-memory stages from its first cycle - it needs nothing from X;
-//   warp 1        waits for the quantize kernel (griddepcontrol.wait), bulk-copies the operand
-//                 image and the table into shared memory, then issues tcgen05.mma kind::i8
-//                 with the weight tile as the 128-row operand and the quantized X as the
-//                 16-column operand: D[n, m] = sum_k CB[n, k] Xq[m, k] into a 128 x 16 int32
-//                 TMEM accumulator (double-buffered over tiles);
+//   start         thread 0 of every CTA asks L2 for the whole of its first tile, so HBM
+//                 streams CB from the first microsecond (each weight byte is still read from
+//                 HBM once per call; the stage loads below then find it in L2);
+//   all warps     quantize X in this CTA (X is a few hundred KB at most and L2-resident):
+//                 one lane per (row, 8-column chunk), each warp holding all 16 rows of two
+//                 chunks.  The outlier bits of a chunk (|x| >= threshold in any row) are an
+//                 OR across its 16 lanes; row maxima over the regular columns reduce in
+//                 registers and across warps; the int8 codes are written straight into
+//                 shared memory in the 128-byte-swizzled K-major layout of the tensor-core
+//                 operand (rows padded to 16, outlier columns and padding 0);
+//   warp 0        TMA producer: 128-row x 128-byte tiles of CB (16 KB) through a ring of
+//                 shared-memory stages, issued as soon as the X loads are out;
+//   warp 1        tcgen05.mma kind::i8 with the weight tile as the 128-row operand and the
+//                 quantized X as the 16-column operand: D[n, m] = sum_k CB[n, k] Xq[m, k] into
+//                 a 128 x 16 int32 TMEM accumulator (double-buffered over tiles);
 //   warps 4..7    epilogue: D -> registers; y = D * SCA_m * SCB_n / 127^2
 //                 + sum_{j in O} X[m, O_j] * W_o[n, O_j] + bias_n (the fp16 outlier part of
 //                 the decomposition, weights from the bytes of the outlier columns) -> fp16.
@@ -45,15 +40,53 @@ constexpr int DM = kDecodeMaxM;         // activation rows held (MMA N)
 constexpr int DBM = 128;                // weight rows per tile (MMA M)
 constexpr int DBK = 128;                // bytes of K per stage
 constexpr int DSTAGE = DBM * DBK;       // 16 KB
-constexpr int DTHREADS = 256;
+constexpr int DTHREADS = 512;
+constexpr int DWARPS = DTHREADS / 32;
 constexpr int DMAX_STAGES = 12;
+constexpr int DCAP = kDecodeMaxOutliers;
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
-constexpr int QTHREADS = 1024;          // quantize kernel: one cluster of QCL CTAs
-constexpr int QWARPS = QTHREADS / 32;
-constexpr int QCL = 8;
-// chunk pairs (16 columns) per warp: K <= kDecodeMaxK keeps every item in registers
-constexpr int QKEEP = (kDecodeMaxK / 16 / QCL + QWARPS - 1) / QWARPS;
-constexpr uint32_t kPrefetchLimit = 64u << 20;   // weight bytes pulled into L2 up front
+// chunk pairs (16 columns) per warp kept in registers between the two quantization passes
+constexpr int QKEEP = 8;
+
+struct DTail {
+    uint64_t full[DMAX_STAGES];
+    uint64_t empty[DMAX_STAGES];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+    int n_out;                           // outlier columns used (<= cap)
+    uint32_t rowmax[DM];                 // float bits (non-negative: int order == float order)
+    float sca[DM];
+    float mult[DM];                      // fl32(127 / sca), 0 for rows >= M or all-zero rows
+    int warp_tot[DWARPS];
+    uint8_t flags[kDecodeMaxK / 8];      // outlier bits of every 8-column chunk
+    int32_t idx[DCAP];                   // outlier columns (ascending)
+    alignas(16) __half xo[DCAP * DM];    // X at the outlier columns, [j][m] (read as uint4)
+};
+static_assert(offsetof(DTail, xo) % 16 == 0, "xo is read with 16-byte loads");
+static_assert(offsetof(DTail, full) % 8 == 0, "mbarriers are 8-byte aligned");
+
+struct DArgs {
+    const __half *X;
+    const int8_t *CB;
+    const float *SCB;
+    const __half *W16;
+    const __half *bias;
+    __half *Y;
+    int32_t *C_debug;
+    int32_t *count;
+    StatusRef status;
+    int M, N, K, cap;
+    float threshold;
+    int stages;
+    int kblocks;
+    int tiles;
+    uint32_t xq_off;                     // byte offsets in shared memory
+    uint32_t tail_off;
+    uint64_t timeout_ns;
+};
 
 __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&v);
@@ -102,203 +135,6 @@ __device__ __forceinline__ uint2 quant8(const float *f, float mul, uint32_t skip
     return make_uint2(lo, hi);
 }
 
-struct QArgs {
-    const __half *X;
-    int M, K, cap;
-    float threshold;
-    uint8_t *image;
-    DecodeTables *tables;
-    int32_t *count;
-    StatusRef status;
-    const int8_t *CB;                   // weights to start pulling into L2
-    uint32_t prefetch_bytes;            // multiple of 16
-};
-
-// Clusters of QCL CTAs.  Every CTA first asks L2 for its slice of the weight bytes (the
-// slices are spread over many SMs: one SM's copy engine alone would take far longer than
-// HBM needs), then every cluster but the first is done.  In the first cluster CTA r owns
-// the chunk pairs [r*PP, (r+1)*PP); one thread per (row, chunk) item, its values kept in
-// registers between the two passes.
-__global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(const QArgs a) {
-    // the dependent kernel's weight stream needs nothing from here
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (threadIdx.x < 32 && a.prefetch_bytes) {
-        constexpr uint32_t kPiece = 16384;
-        const uint32_t share = (a.prefetch_bytes / gridDim.x + 15u) & ~15u;
-        const uint32_t b0 = blockIdx.x * share, b1 = min(a.prefetch_bytes, b0 + share);
-        for (uint32_t off = b0 + threadIdx.x * kPiece; off < b1; off += 32 * kPiece)
-            prefetch_l2_bulk(a.CB + off, min(kPiece, b1 - off));
-    }
-    if (blockIdx.x >= QCL) return;            // a whole cluster leaves together
-    __shared__ float part[QCL][DM];          // row maxima of every CTA of the cluster
-    __shared__ uint32_t pmax[DM];            // this CTA's (float bits, >= 0: int order)
-    __shared__ float mult[DM];
-    __shared__ uint8_t flags_all[kDecodeMaxK / 8];   // CTA 0: outlier bits of every chunk
-    __shared__ int n_out_s;
-    __shared__ int warp_tot[QWARPS];
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int m = lane & 15;                 // the row this thread handles
-    const int half = lane >> 4;              // which chunk of the warp's pair
-    const uint32_t r = cluster_ctarank();
-    const int nchunks = a.K / 8;
-    const int npairs = nchunks / 2;          // K is a multiple of 16
-    const int pp = (npairs + QCL - 1) / QCL;
-    const int p0 = (int)r * pp, p1 = min(npairs, p0 + pp);
-    const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
-
-    uint4 v[QKEEP];
-#pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        const int p = p0 + warp + i * QWARPS;
-        v[i] = (p < p1 && m < a.M) ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
-                                   : make_uint4(0, 0, 0, 0);
-    }
-    if (t < DM) pmax[t] = 0u;
-    __syncthreads();
-
-    // pass 1: outlier bits of each chunk (OR over its 16 lanes = rows), published to CTA 0;
-    // row maxima over the regular columns
-    uint32_t fl[QKEEP];
-    float rm = 0.0f;
-    const uint32_t flags0 = map_to_rank(smem_addr(flags_all), 0);
-#pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        fl[i] = 0;
-        const int p = p0 + warp + i * QWARPS;
-        if (p < p1) {                        // uniform over the warp
-            float f[8];
-            unpack8(v[i], f);
-            uint32_t b = outlier_bits(f, a.threshold);
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
-            fl[i] = b;
-            if (m == 0) st_cluster_u8(flags0 + (uint32_t)(2 * p + half), b);
-            rm = masked_max(f, b, rm);
-        }
-    }
-    rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 16));
-    if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&pmax[m], __float_as_uint(rm));
-    __syncthreads();
-    if (t < DM) {
-        const uint32_t dst = smem_addr(&part[r][t]);
-        for (int rr = 0; rr < QCL; ++rr) st_cluster_u32(map_to_rank(dst, (uint32_t)rr), pmax[t]);
-    }
-    // every CTA's flags and partial maxima are in place after this
-    cluster_barrier_all();
-
-    if (t < DM) {
-        float amax = 0.0f;
-        for (int rr = 0; rr < QCL; ++rr) amax = fmaxf(amax, part[rr][t]);
-        mult[t] = (t < a.M && amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
-        if (r == 0) a.tables->sca[t] = amax;
-    }
-    __syncthreads();
-
-    // pass 2: every (row, chunk) of this CTA into the operand image; rows >= M, all-zero rows
-    // and outlier columns are written as 0
-    const float mul = mult[m];
-#pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        const int p = p0 + warp + i * QWARPS;
-        if (p < p1) {
-            const int c = 2 * p + half;
-            uint2 q = make_uint2(0, 0);
-            if (mul > 0.0f) {
-                float f[8];
-                unpack8(v[i], f);
-                q = quant8(f, mul, fl[i]);
-            }
-            *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8)) = q;
-        }
-    }
-    if (r != 0) return;   // nothing of this CTA is read by its peers any more
-
-    // CTA 0: padding columns of the image, ascending outlier list, count, status, X there
-    const int kpad_chunks = (a.K + 127) / 128 * 16;
-    for (int i = t; i < (kpad_chunks - nchunks) * DM; i += QTHREADS) {
-        const int c = nchunks + i / DM, mm = i % DM;
-        *reinterpret_cast<uint2 *>(a.image + xq_offset(mm, c * 8)) = make_uint2(0, 0);
-    }
-    {
-        // ascending list: one chunk per thread (K/8 <= QTHREADS), block-wide exclusive scan
-        const uint32_t b0 = t < nchunks ? flags_all[t] : 0u;
-        const int cnt = __popc(b0);
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        if (lane == 31) warp_tot[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            const int v0 = warp_tot[lane];
-            int x = v0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            warp_tot[lane] = x - v0;
-            if (lane == 31) {
-                n_out_s = min(x, a.cap);
-                a.tables->n_out = n_out_s;
-                *a.count = x;
-                a.status.set(x > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
-            }
-        }
-        __syncthreads();
-        int pos = warp_tot[warp] + incl - cnt;
-        uint32_t b = b0;
-        while (b) {
-            const int e = __ffs(b) - 1;
-            b &= b - 1;
-            if (pos < a.cap) {
-                const int col = t * 8 + e;
-                a.tables->idx[pos] = col;
-                // X at this outlier column, [j][m]
-                for (int mm = 0; mm < DM; ++mm)
-                    a.tables->xo[pos * DM + mm] =
-                        mm < a.M ? a.X[(int64_t)mm * a.K + col] : __float2half_rn(0.0f);
-            }
-            ++pos;
-        }
-    }
-}
-
-struct DTail {
-    uint64_t full[DMAX_STAGES];
-    uint64_t empty[DMAX_STAGES];
-    uint64_t acc_full[2];
-    uint64_t acc_empty[2];
-    uint64_t mma_done;
-    uint64_t xbar;                       // operand image and table have landed
-    uint32_t tmem_base;
-    int abort_flag;
-    alignas(16) DecodeTables tab;
-};
-static_assert(offsetof(DTail, tab) % 16 == 0, "the table is a bulk-copy destination");
-static_assert(offsetof(DTail, xbar) % 8 == 0, "mbarriers are 8-byte aligned");
-
-struct DArgs {
-    const int8_t *CB;
-    const float *SCB;
-    const __half *W16;
-    const __half *bias;
-    __half *Y;
-    int32_t *C_debug;
-    const uint8_t *image;
-    const DecodeTables *tables;
-    StatusRef status;
-    int M, N, K;
-    int stages;
-    int kblocks;
-    int tiles;
-    uint32_t xq_off;                     // byte offsets in shared memory
-    uint32_t tail_off;
-    uint64_t timeout_ns;
-};
-
 __global__ void __launch_bounds__(DTHREADS, 1)
 llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -306,10 +142,23 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     DTail *tail = reinterpret_cast<DTail *>(smem + a.tail_off);
     uint8_t *xq = smem + a.xq_off;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int S = a.stages;
+    const int m = lane & 15;                 // quantization: the row this lane handles
+    const int half = lane >> 4;              //               which chunk of the warp's pair
+    const int nchunks = a.K / 8;
+    const int npairs = nchunks / 2;          // K is a multiple of 16
+    const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
 
-    if (threadIdx.x == 0) {
+    // X first, ahead of every weight request of every SM
+    uint4 keep[QKEEP];
+#pragma unroll
+    for (int i = 0; i < QKEEP; ++i) {
+        const int p = warp + i * DWARPS;
+        keep[i] = (p < npairs && m < a.M) ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
+                                          : make_uint4(0, 0, 0, 0);
+    }
+    if (t == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(smem_addr(&tail->full[s]), 1);
             mbar_init(smem_addr(&tail->empty[s]), 1);
@@ -319,40 +168,171 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             mbar_init(smem_addr(&tail->acc_empty[s]), 4);
         }
         mbar_init(smem_addr(&tail->mma_done), 1);
-        mbar_init(smem_addr(&tail->xbar), 1);
         tail->abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmCB);
+        // the whole first tile into L2: HBM keeps streaming while X is quantized
+        if ((int)blockIdx.x < a.tiles)
+            for (int kb = 0; kb < a.kblocks; ++kb)
+                tma_prefetch_l2_2d(&tmCB, kb * DBK, (int)blockIdx.x * DBM);
     }
+    if (t < DM) tail->rowmax[t] = 0u;
     if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), 32);
+    // zero the operand (rows >= M and columns >= K must read as 0)
+    for (int i = t; i < a.kblocks * DBK * DM / 16; i += DTHREADS)
+        reinterpret_cast<uint4 *>(xq)[i] = make_uint4(0, 0, 0, 0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tail->tmem_base;
     const BoundedWait wait{&tail->abort_flag, a.status, a.timeout_ns};
 
+    // weight stream: the producer lane fills the ring now; the MMA starts once X is in
+    int stage = 0;
+    uint32_t phase = 0, used = 0, last_parity = 0;
+    int ptile = blockIdx.x, pit = 0;         // next (tile, k-block) to load
+    auto produce = [&](int limit) -> bool {  // issue up to `limit` stage loads
+        for (int n = 0; n < limit && ptile < a.tiles; ++n) {
+            if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) return false;
+            const uint32_t full = smem_addr(&tail->full[stage]);
+            mbar_arrive_expect_tx(full, DSTAGE);
+            tma_load_2d(smem_addr(smem + stage * DSTAGE), &tmCB,
+                        rotated_kblock(pit, ptile, a.kblocks) * DBK, ptile * DBM, full);
+            used |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+            if (++stage == S) {
+                stage = 0;
+                phase ^= 1;
+            }
+            if (++pit == a.kblocks) {
+                pit = 0;
+                ptile += gridDim.x;
+            }
+        }
+        return true;
+    };
+    bool producing = true;
+    if (t == 0) producing = produce(S);
+
+    // ---------------------------------------------------- quantize X in this CTA ----
+    // pass 1: outlier bits (OR over the 16 lanes = rows of a chunk) and row maxima over the
+    // regular columns
+    uint32_t fl[QKEEP];
+    float rm = 0.0f;
+#pragma unroll
+    for (int i = 0; i < QKEEP; ++i) {
+        fl[i] = 0;
+        const int p = warp + i * DWARPS;
+        if (p < npairs) {                    // uniform over the warp
+            float f[8];
+            unpack8(keep[i], f);
+            uint32_t b = outlier_bits(f, a.threshold);
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
+            fl[i] = b;
+            if (m == 0) tail->flags[2 * p + half] = (uint8_t)b;
+            rm = masked_max(f, b, rm);
+        }
+    }
+    for (int p = warp + QKEEP * DWARPS; p < npairs; p += DWARPS) {
+        const uint4 v = m < a.M ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
+                                : make_uint4(0, 0, 0, 0);
+        float f[8];
+        unpack8(v, f);
+        uint32_t b = outlier_bits(f, a.threshold);
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
+        if (m == 0) tail->flags[2 * p + half] = (uint8_t)b;
+        rm = masked_max(f, b, rm);
+    }
+    rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 16));
+    if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&tail->rowmax[m], __float_as_uint(rm));
+    __syncthreads();
+
+    // scales; ascending outlier list by a block-wide scan over the chunks
+    if (t < DM) {
+        const float amax = __uint_as_float(tail->rowmax[t]);
+        tail->sca[t] = amax;
+        tail->mult[t] = (t < a.M && amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
+    }
+    {
+        const int per = (nchunks + DTHREADS - 1) / DTHREADS;   // contiguous chunks per thread
+        const int c0 = t * per, c1 = min(nchunks, c0 + per);
+        int cnt = 0;
+        for (int c = c0; c < c1; ++c) cnt += __popc(tail->flags[c]);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) tail->warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int v0 = lane < DWARPS ? tail->warp_tot[lane] : 0;
+            int x = v0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (lane < DWARPS) tail->warp_tot[lane] = x - v0;
+            if (lane == 31) {
+                tail->n_out = min(x, a.cap);
+                if (blockIdx.x == 0) {
+                    *a.count = x;
+                    a.status.set(x > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
+                }
+            }
+        }
+        __syncthreads();
+        int pos = tail->warp_tot[warp] + incl - cnt;
+        for (int c = c0; c < c1; ++c) {
+            uint32_t b = tail->flags[c];
+            while (b) {
+                const int e = __ffs(b) - 1;
+                b &= b - 1;
+                if (pos < a.cap) tail->idx[pos] = c * 8 + e;
+                ++pos;
+            }
+        }
+    }
+    __syncthreads();
+
+    // pass 2: int8 codes into the swizzled operand; X at the outlier columns into xo
+    const float mul = tail->mult[m];
+#pragma unroll
+    for (int i = 0; i < QKEEP; ++i) {
+        const int p = warp + i * DWARPS;
+        if (p < npairs && mul > 0.0f) {
+            float f[8];
+            unpack8(keep[i], f);
+            *reinterpret_cast<uint2 *>(xq + xq_offset(m, (2 * p + half) * 8)) =
+                quant8(f, mul, fl[i]);
+        }
+    }
+    for (int p = warp + QKEEP * DWARPS; p < npairs; p += DWARPS) {
+        if (mul > 0.0f) {
+            const int c = 2 * p + half;
+            float f[8];
+            unpack8(__ldg(X4 + (int64_t)m * nchunks + c), f);
+            *reinterpret_cast<uint2 *>(xq + xq_offset(m, c * 8)) = quant8(f, mul, tail->flags[c]);
+        }
+    }
+    const int n_out = tail->n_out;
+    for (int i = t; i < n_out * DM; i += DTHREADS) {
+        const int j = i / DM, mm = i % DM;
+        tail->xo[i] = mm < a.M ? a.X[(int64_t)mm * a.K + tail->idx[j]] : __float2half_rn(0.0f);
+    }
+    // the operand was written through the generic proxy; the tensor core reads it through
+    // the async proxy
+    fence_proxy_async_smem();
+    __syncthreads();
+
     if (warp == 0) {
         // --------------------------------------------------- weight stream (TMA) ----
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0, used = 0, last_parity = 0;
-            for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
-                const int n0 = tile * DBM;
-                for (int it = 0; it < a.kblocks; ++it) {
-                    const int kb = rotated_kblock(it, tile, a.kblocks);
-                    if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
-                    const uint32_t full = smem_addr(&tail->full[stage]);
-                    mbar_arrive_expect_tx(full, DSTAGE);
-                    tma_load_2d(smem_addr(smem + stage * DSTAGE), &tmCB, kb * DBK, n0, full);
-                    used |= 1u << stage;
-                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-                    if (++stage == S) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
-                }
-            }
-        drain:
+            if (producing) produce(1 << 30);
             for (int s = 0; s < S; ++s)
                 if (used & (1u << s))
                     drain_wait(smem_addr(&tail->full[s]), (last_parity >> s) & 1u, a.status);
@@ -360,41 +340,32 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issue ----
         if (lane == 0) {
-            // the quantize kernel has finished and its writes are visible after this
-            asm volatile("griddepcontrol.wait;" ::: "memory");
-            const uint32_t xbar = smem_addr(&tail->xbar);
-            const uint32_t img_bytes = (uint32_t)(a.kblocks * DBK * DM);
-            mbar_arrive_expect_tx(xbar, img_bytes + (uint32_t)sizeof(DecodeTables));
-            for (uint32_t off = 0; off < img_bytes; off += 16384)
-                bulk_load_1d(smem_addr(xq) + off, a.image + off, min(16384u, img_bytes - off), xbar);
-            bulk_load_1d(smem_addr(&tail->tab), a.tables, (uint32_t)sizeof(DecodeTables), xbar);
-            const bool have_x = wait(xbar, 0);
             const uint32_t idesc = idesc_i8(DBM, DM);
             const uint32_t xq_base = smem_addr(xq);
-            int stage = 0, acc = 0;
-            uint32_t phase = 0, acc_phase = 0;
-            for (int tile = blockIdx.x; have_x && tile < a.tiles; tile += gridDim.x) {
+            int cs = 0, acc = 0;
+            uint32_t cphase = 0, acc_phase = 0;
+            for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
                 if (!wait(smem_addr(&tail->acc_empty[acc]), acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * DM);
                 bool good = true;
                 for (int it = 0; it < a.kblocks; ++it) {
                     const int kb = rotated_kblock(it, tile, a.kblocks);
-                    if (!wait(smem_addr(&tail->full[stage]), phase)) {
+                    if (!wait(smem_addr(&tail->full[cs]), cphase)) {
                         good = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_addr(smem + stage * DSTAGE);
+                    const uint32_t sa = smem_addr(smem + cs * DSTAGE);
                     const uint32_t sb = xq_base + (uint32_t)(kb * DM * 128);
 #pragma unroll
                     for (int k = 0; k < DBK / 32; ++k)
                         mma_i8(d, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
                                (it | k) != 0);
-                    tc_commit(smem_addr(&tail->empty[stage]));
-                    if (++stage == S) {
-                        stage = 0;
-                        phase ^= 1;
+                    tc_commit(smem_addr(&tail->empty[cs]));
+                    if (++cs == S) {
+                        cs = 0;
+                        cphase ^= 1;
                     }
                 }
                 if (!good) break;
@@ -402,22 +373,17 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
             }
-            if (!have_x) drain_wait(xbar, 0, a.status);   // the copies land before exit
             tc_commit(smem_addr(&tail->mma_done));
             drain_wait(smem_addr(&tail->mma_done), 0, a.status);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------------ epilogue ----
         const int qd = warp & 3;
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
         const float inv = 1.0f / 16129.0f;
-        int okx = 0;
-        if (lane == 0) okx = wait(smem_addr(&tail->xbar), 0) ? 1 : 0;   // the table is in
-        okx = __shfl_sync(0xffffffffu, okx, 0);
-        const int n_out = okx ? tail->tab.n_out : 0;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; okx && tile < a.tiles; tile += gridDim.x) {
+        for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
             int okw = 0;
             if (lane == 0) okw = wait(smem_addr(&tail->acc_full[acc]), acc_phase) ? 1 : 0;
             okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -438,30 +404,30 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 const float b = a.bias ? __half2float(a.bias[n]) : 0.0f;
                 float o[DM];
 #pragma unroll
-                for (int m = 0; m < DM; ++m) o[m] = 0.0f;
+                for (int r = 0; r < DM; ++r) o[r] = 0.0f;
                 const int8_t *cbrow = a.CB + (int64_t)n * a.K;
                 for (int j = 0; j < n_out; ++j) {
-                    const int col = tail->tab.idx[j];
+                    const int col = tail->idx[j];
                     const float w = a.W16 ? __half2float(a.W16[(int64_t)n * a.K + col])
                                           : __half2float(__float2half_rn(__fdiv_rn(
                                                 __fmul_rn((float)cbrow[col], sb), 127.0f)));
-                    const uint4 *xv = reinterpret_cast<const uint4 *>(tail->tab.xo + j * DM);
+                    const uint4 *xv = reinterpret_cast<const uint4 *>(tail->xo + j * DM);
                     float f0[8], f1[8];
                     unpack8(xv[0], f0);
                     unpack8(xv[1], f1);
 #pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        o[m] = fmaf(f0[m], w, o[m]);
-                        o[m + 8] = fmaf(f1[m], w, o[m + 8]);
+                    for (int r = 0; r < 8; ++r) {
+                        o[r] = fmaf(f0[r], w, o[r]);
+                        o[r + 8] = fmaf(f1[r], w, o[r + 8]);
                     }
                 }
 #pragma unroll
-                for (int m = 0; m < DM; ++m) {
-                    if (m < a.M) {
-                        const float y = fmaf((float)(int32_t)d[m], tail->tab.sca[m] * inv * sb,
-                                             o[m] + b);
-                        a.Y[(int64_t)m * a.N + n] = __float2half_rn(y);
-                        if (a.C_debug) a.C_debug[(int64_t)m * a.N + n] = (int32_t)d[m];
+                for (int r = 0; r < DM; ++r) {
+                    if (r < a.M) {
+                        const float y = fmaf((float)(int32_t)d[r], tail->sca[r] * inv * sb,
+                                             o[r] + b);
+                        a.Y[(int64_t)r * a.N + n] = __float2half_rn(y);
+                        if (a.C_debug) a.C_debug[(int64_t)r * a.N + n] = (int32_t)d[r];
                     }
                 }
             }
@@ -513,55 +479,21 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
         sms = sms_cache[dev];
     }
 
-    // 1. quantize X once (one CTA)
-    QArgs q;
-    q.X = d.X;
-    q.M = (int)d.M;
-    q.K = (int)d.K;
-    q.cap = (int)d.cap;
-    q.threshold = d.threshold;
-    q.image = d.image;
-    q.tables = d.tables;
-    q.count = d.count;
-    q.status = d.status;
-    q.CB = d.CB;
-    q.prefetch_bytes = (uint32_t)std::min<int64_t>(d.N * d.K, kPrefetchLimit) & ~15u;
-    {
-        cudaLaunchConfig_t qc = {};
-        cudaLaunchAttribute qa[1];
-        qa[0].id = cudaLaunchAttributeClusterDimension;
-        qa[0].val.clusterDim.x = QCL;
-        qa[0].val.clusterDim.y = 1;
-        qa[0].val.clusterDim.z = 1;
-        // the prefetch is spread over ~one CTA per 512 KB of weights
-        const int64_t want = ceil_div((int64_t)q.prefetch_bytes, 512 * 1024);
-        const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(want, QCL),
-                                                                         std::max(1, sms / QCL)));
-        qc.gridDim = dim3((unsigned)(clusters * QCL));
-        qc.blockDim = dim3(QTHREADS);
-        qc.dynamicSmemBytes = 0;
-        qc.stream = s;
-        qc.attrs = qa;
-        qc.numAttrs = 1;
-        err = cudaLaunchKernelEx(&qc, llmint8_decode_quantize_kernel, q);
-        note_launches(1);
-        if (err != cudaSuccess) return err;
-    }
-
-    // 2. the weight-streaming product, allowed to start before step 1 finishes
     DArgs a;
+    a.X = d.X;
     a.CB = d.CB;
     a.SCB = d.SCB;
     a.W16 = d.W16;
     a.bias = d.bias;
     a.Y = d.Y;
     a.C_debug = d.C_debug;
-    a.image = d.image;
-    a.tables = d.tables;
+    a.count = d.count;
     a.status = d.status;
     a.M = (int)d.M;
     a.N = (int)d.N;
     a.K = (int)d.K;
+    a.cap = (int)d.cap;
+    a.threshold = d.threshold;
     a.kblocks = (int)ceil_div(d.K, DBK);
     a.tiles = (int)ceil_div(d.N, DBM);
     a.timeout_ns = d.timeout_ns;
@@ -587,21 +519,10 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    // QCL SMs stay with the quantize kernel while this grid starts
-    cfg.gridDim = dim3((unsigned)std::min(a.tiles, std::max(1, sms - QCL)));
-    cfg.blockDim = dim3(DTHREADS);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, llmint8_decode_kernel, tm, a);
+    const int grid = std::min(a.tiles, sms);
+    llmint8_decode_kernel<<<grid, DTHREADS, smem, s>>>(tm, a);
     note_launches(1);
-    return err != cudaSuccess ? err : cudaGetLastError();
+    return cudaGetLastError();
 }
 
 }  // namespace llmint8
