@@ -1,21 +1,22 @@
 // Decode path of the LLM.int8() layer (few activation rows, M <= 16).
 //
 // At decode sizes the layer is bound by streaming the int8 weight CB from HBM once, and the
-// rest must hide under that stream.  One kernel, one CTA of 512 threads per 128-row weight
-// tile (grid-stride over tiles when there are more tiles than SMs):
+// rest must hide under that stream.  One cooperative kernel (every CTA resident, one per SM),
+// one CTA of 512 threads per 128-row weight tile (grid-stride when there are more tiles):
 //
-//   start         thread 0 of every CTA asks L2 for the whole of its first tile, so HBM
-//                 streams CB from the first microsecond (each weight byte is still read from
-//                 HBM once per call; the stage loads below then find it in L2);
-//   all warps     quantize X in this CTA (X is a few hundred KB at most and L2-resident):
-//                 one lane per (row, 8-column chunk), each warp holding all 16 rows of two
-//                 chunks.  The outlier bits of a chunk (|x| >= threshold in any row) are an
-//                 OR across its 16 lanes; row maxima over the regular columns reduce in
-//                 registers and across warps; the int8 codes are written straight into
-//                 shared memory in the 128-byte-swizzled K-major layout of the tensor-core
-//                 operand (rows padded to 16, outlier columns and padding 0);
-//   warp 0        TMA producer: 128-row x 128-byte tiles of CB (16 KB) through a ring of
-//                 shared-memory stages, issued as soon as the X loads are out;
+//   warp 0 lane 0 TMA producer: fills a ring of shared-memory stages with 128-row x 128-byte
+//                 tiles of CB (16 KB) from the first microsecond - it needs nothing from X -
+//                 and asks L2 for the rest of its first tile, so HBM keeps streaming while
+//                 X is quantized (each weight byte is still read from HBM once per call);
+//   all warps     quantize X together.  CTA g owns 1/G of the columns: one lane per (row,
+//                 8-column chunk), each warp holding all 16 rows of two chunks, so the outlier
+//                 bits of a chunk (|x| >= threshold in any row) are an OR across 16 lanes and
+//                 the row maxima over the regular columns reduce in registers.  Outlier bits
+//                 and partial maxima go to workspace scratch; after a grid barrier every CTA
+//                 has SCA and the ascending outlier set, quantizes its columns and writes the
+//                 int8 codes into a byte image of the tensor-core operand (16 rows, 128-byte
+//                 swizzled K-major blocks, outlier columns and padding 0); after a second
+//                 grid barrier every CTA bulk-copies the whole image into shared memory;
 //   warp 1        tcgen05.mma kind::i8 with the weight tile as the 128-row operand and the
 //                 quantized X as the 16-column operand: D[n, m] = sum_k CB[n, k] Xq[m, k] into
 //                 a 128 x 16 int32 TMEM accumulator (double-buffered over tiles);
@@ -23,7 +24,8 @@
 //                 + sum_{j in O} X[m, O_j] * W_o[n, O_j] + bias_n (the fp16 outlier part of
 //                 the decomposition, weights from the bytes of the outlier columns) -> fp16.
 // Same method and rounding as the GEMM path (LLM.int8() summary, sections الابتكار الثاني
-// and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded.
+// and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded; the grid
+// barriers use a fixed bound, so every CTA always reaches both.
 #include <cudaTypedefs.h>
 
 #include <cstddef>
@@ -45,8 +47,7 @@ constexpr int DWARPS = DTHREADS / 32;
 constexpr int DMAX_STAGES = 12;
 constexpr int DCAP = kDecodeMaxOutliers;
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
-// chunk pairs (16 columns) per warp kept in registers between the two quantization passes
-constexpr int QKEEP = 8;
+constexpr int QKEEP = 4;                // chunk pairs per warp kept in registers
 
 struct DTail {
     uint64_t full[DMAX_STAGES];
@@ -54,19 +55,20 @@ struct DTail {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t mma_done;
+    uint64_t xbar;                       // the operand image has landed
     uint32_t tmem_base;
     int abort_flag;
     int n_out;                           // outlier columns used (<= cap)
+    int bar_ok;
     uint32_t rowmax[DM];                 // float bits (non-negative: int order == float order)
     float sca[DM];
     float mult[DM];                      // fl32(127 / sca), 0 for rows >= M or all-zero rows
     int warp_tot[DWARPS];
-    uint8_t flags[kDecodeMaxK / 8];      // outlier bits of every 8-column chunk
     int32_t idx[DCAP];                   // outlier columns (ascending)
     alignas(16) __half xo[DCAP * DM];    // X at the outlier columns, [j][m] (read as uint4)
 };
 static_assert(offsetof(DTail, xo) % 16 == 0, "xo is read with 16-byte loads");
-static_assert(offsetof(DTail, full) % 8 == 0, "mbarriers are 8-byte aligned");
+static_assert(offsetof(DTail, xbar) % 8 == 0, "mbarriers are 8-byte aligned");
 
 struct DArgs {
     const __half *X;
@@ -77,7 +79,10 @@ struct DArgs {
     __half *Y;
     int32_t *C_debug;
     int32_t *count;
+    DecodeScratch *scr;
+    uint8_t *image;
     StatusRef status;
+    unsigned long long epoch;
     int M, N, K, cap;
     float threshold;
     int stages;
@@ -135,6 +140,40 @@ __device__ __forceinline__ uint2 quant8(const float *f, float mul, uint32_t skip
     return make_uint2(lo, hi);
 }
 
+// Barrier over every CTA of the (cooperative, all-resident) grid.  The counter word holds
+// (epoch << 12) | arrivals; the first arrival of a call replaces whatever an earlier call
+// left, so the scratch needs no initialization.  Bounded by a fixed limit.
+__device__ __forceinline__ void grid_barrier(unsigned long long *word, unsigned long long epoch,
+                                             DTail *tail, StatusRef status) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned long long base = epoch << 12;
+        unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(word);
+        for (;;) {
+            const unsigned long long next = ((cur >> 12) == epoch) ? cur + 1ull : base + 1ull;
+            const unsigned long long prev = atomicCAS(word, cur, next);
+            if (prev == cur) break;
+            cur = prev;
+        }
+        const unsigned long long target = base + gridDim.x;
+        constexpr uint64_t kLimitNs = 1000000000ull;
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t it = 0;; ++it) {
+            unsigned long long v;
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(word) : "memory");
+            if (v == target) break;
+            if ((it & 63u) == 0u && global_timer_ns() - t0 > kLimitNs) {
+                status.timed_out();
+                tail->bar_ok = 0;
+                break;
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(DTHREADS, 1)
 llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -148,15 +187,17 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     const int half = lane >> 4;              //               which chunk of the warp's pair
     const int nchunks = a.K / 8;
     const int npairs = nchunks / 2;          // K is a multiple of 16
+    const int pp = (npairs + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int p0 = (int)blockIdx.x * pp, p1 = min(npairs, p0 + pp);   // this CTA's pairs
     const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
 
-    // X first, ahead of every weight request of every SM
+    // this CTA's columns of X first, ahead of every weight request
     uint4 keep[QKEEP];
 #pragma unroll
     for (int i = 0; i < QKEEP; ++i) {
-        const int p = warp + i * DWARPS;
-        keep[i] = (p < npairs && m < a.M) ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
-                                          : make_uint4(0, 0, 0, 0);
+        const int p = p0 + warp + i * DWARPS;
+        keep[i] = (p < p1 && m < a.M) ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
+                                      : make_uint4(0, 0, 0, 0);
     }
     if (t == 0) {
         for (int s = 0; s < S; ++s) {
@@ -168,26 +209,21 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             mbar_init(smem_addr(&tail->acc_empty[s]), 4);
         }
         mbar_init(smem_addr(&tail->mma_done), 1);
+        mbar_init(smem_addr(&tail->xbar), 1);
         tail->abort_flag = 0;
+        tail->bar_ok = 1;
         fence_mbar_init();
         tma_prefetch_desc(&tmCB);
-        // the whole first tile into L2: HBM keeps streaming while X is quantized
-        if ((int)blockIdx.x < a.tiles)
-            for (int kb = 0; kb < a.kblocks; ++kb)
-                tma_prefetch_l2_2d(&tmCB, kb * DBK, (int)blockIdx.x * DBM);
     }
     if (t < DM) tail->rowmax[t] = 0u;
     if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), 32);
-    // zero the operand (rows >= M and columns >= K must read as 0)
-    for (int i = t; i < a.kblocks * DBK * DM / 16; i += DTHREADS)
-        reinterpret_cast<uint4 *>(xq)[i] = make_uint4(0, 0, 0, 0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tail->tmem_base;
     const BoundedWait wait{&tail->abort_flag, a.status, a.timeout_ns};
 
-    // weight stream: the producer lane fills the ring now; the MMA starts once X is in
+    // weight stream: fill the ring now, ask L2 for the rest of the first tile
     int stage = 0;
     uint32_t phase = 0, used = 0, last_parity = 0;
     int ptile = blockIdx.x, pit = 0;         // next (tile, k-block) to load
@@ -212,29 +248,35 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         return true;
     };
     bool producing = true;
-    if (t == 0) producing = produce(S);
+    if (t == 0) {
+        producing = produce(S);
+        if ((int)blockIdx.x < a.tiles)
+            for (int it = S; it < a.kblocks; ++it)
+                tma_prefetch_l2_2d(&tmCB, rotated_kblock(it, blockIdx.x, a.kblocks) * DBK,
+                                   (int)blockIdx.x * DBM);
+    }
 
-    // ---------------------------------------------------- quantize X in this CTA ----
-    // pass 1: outlier bits (OR over the 16 lanes = rows of a chunk) and row maxima over the
-    // regular columns
+    // ------------------------------------------------- quantize X across the grid ----
+    // pass 1 (own columns): outlier bits (OR over the 16 lanes = rows of a chunk) to the
+    // scratch, row maxima over the regular columns
     uint32_t fl[QKEEP];
     float rm = 0.0f;
 #pragma unroll
     for (int i = 0; i < QKEEP; ++i) {
         fl[i] = 0;
-        const int p = warp + i * DWARPS;
-        if (p < npairs) {                    // uniform over the warp
+        const int p = p0 + warp + i * DWARPS;
+        if (p < p1) {                        // uniform over the warp
             float f[8];
             unpack8(keep[i], f);
             uint32_t b = outlier_bits(f, a.threshold);
 #pragma unroll
             for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
             fl[i] = b;
-            if (m == 0) tail->flags[2 * p + half] = (uint8_t)b;
+            if (m == 0) a.scr->flags[2 * p + half] = (uint8_t)b;
             rm = masked_max(f, b, rm);
         }
     }
-    for (int p = warp + QKEEP * DWARPS; p < npairs; p += DWARPS) {
+    for (int p = p0 + warp + QKEEP * DWARPS; p < p1; p += DWARPS) {
         const uint4 v = m < a.M ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
                                 : make_uint4(0, 0, 0, 0);
         float f[8];
@@ -242,24 +284,36 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         uint32_t b = outlier_bits(f, a.threshold);
 #pragma unroll
         for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
-        if (m == 0) tail->flags[2 * p + half] = (uint8_t)b;
+        if (m == 0) a.scr->flags[2 * p + half] = (uint8_t)b;
         rm = masked_max(f, b, rm);
     }
     rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 16));
     if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&tail->rowmax[m], __float_as_uint(rm));
     __syncthreads();
+    if (t < DM) a.scr->part[blockIdx.x * DM + t] = __uint_as_float(tail->rowmax[t]);
+    grid_barrier(&a.scr->bar[0], a.epoch, tail, a.status);
 
-    // scales; ascending outlier list by a block-wide scan over the chunks
-    if (t < DM) {
-        const float amax = __uint_as_float(tail->rowmax[t]);
-        tail->sca[t] = amax;
-        tail->mult[t] = (t < a.M && amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
+    // every CTA: SCA (max over the CTAs' partial maxima), multipliers, ascending outlier list
+    if (t < DM) tail->rowmax[t] = 0u;
+    __syncthreads();
+    {
+        float r = 0.0f;
+        for (int i = t; i < (int)gridDim.x * DM; i += DTHREADS)   // DTHREADS % DM == 0
+            r = fmaxf(r, __ldcg(&a.scr->part[i]));
+        // lanes l and l + 16 hold the same row
+        r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, 16));
+        if (half == 0 && r > 0.0f) atomicMax(&tail->rowmax[m], __float_as_uint(r));
     }
     {
         const int per = (nchunks + DTHREADS - 1) / DTHREADS;   // contiguous chunks per thread
         const int c0 = t * per, c1 = min(nchunks, c0 + per);
+        uint32_t bits[(kDecodeMaxK / 8 + DTHREADS - 1) / DTHREADS];
         int cnt = 0;
-        for (int c = c0; c < c1; ++c) cnt += __popc(tail->flags[c]);
+#pragma unroll
+        for (int j = 0; j < (int)(sizeof(bits) / sizeof(bits[0])); ++j) {
+            bits[j] = (c0 + j < c1) ? (uint32_t)__ldcg(&a.scr->flags[c0 + j]) : 0u;
+            cnt += __popc(bits[j]);
+        }
         int incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -287,47 +341,67 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         }
         __syncthreads();
         int pos = tail->warp_tot[warp] + incl - cnt;
-        for (int c = c0; c < c1; ++c) {
-            uint32_t b = tail->flags[c];
+#pragma unroll
+        for (int j = 0; j < (int)(sizeof(bits) / sizeof(bits[0])); ++j) {
+            uint32_t b = bits[j];
             while (b) {
                 const int e = __ffs(b) - 1;
                 b &= b - 1;
-                if (pos < a.cap) tail->idx[pos] = c * 8 + e;
+                if (pos < a.cap) tail->idx[pos] = (c0 + j) * 8 + e;
                 ++pos;
             }
         }
     }
+    if (t < DM) {
+        const float amax = __uint_as_float(tail->rowmax[t]);
+        tail->sca[t] = amax;
+        tail->mult[t] = (t < a.M && amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
+    }
     __syncthreads();
 
-    // pass 2: int8 codes into the swizzled operand; X at the outlier columns into xo
+    // pass 2 (own columns): int8 codes into the operand image, all 16 rows
     const float mul = tail->mult[m];
 #pragma unroll
     for (int i = 0; i < QKEEP; ++i) {
-        const int p = warp + i * DWARPS;
-        if (p < npairs && mul > 0.0f) {
-            float f[8];
-            unpack8(keep[i], f);
-            *reinterpret_cast<uint2 *>(xq + xq_offset(m, (2 * p + half) * 8)) =
-                quant8(f, mul, fl[i]);
+        const int p = p0 + warp + i * DWARPS;
+        if (p < p1) {
+            const int c = 2 * p + half;
+            uint2 q = make_uint2(0, 0);
+            if (mul > 0.0f) {
+                float f[8];
+                unpack8(keep[i], f);
+                q = quant8(f, mul, fl[i]);
+            }
+            *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8)) = q;
         }
     }
-    for (int p = warp + QKEEP * DWARPS; p < npairs; p += DWARPS) {
+    for (int p = p0 + warp + QKEEP * DWARPS; p < p1; p += DWARPS) {
+        const int c = 2 * p + half;
+        uint2 q = make_uint2(0, 0);
         if (mul > 0.0f) {
-            const int c = 2 * p + half;
             float f[8];
             unpack8(__ldg(X4 + (int64_t)m * nchunks + c), f);
-            *reinterpret_cast<uint2 *>(xq + xq_offset(m, c * 8)) = quant8(f, mul, tail->flags[c]);
+            q = quant8(f, mul, (uint32_t)__ldcg(&a.scr->flags[c]));
         }
+        *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8)) = q;
     }
+    if (blockIdx.x == 0) {
+        // the padding columns of the image
+        const int kpad_chunks = a.kblocks * (DBK / 8);
+        for (int i = t; i < (kpad_chunks - nchunks) * DM; i += DTHREADS)
+            *reinterpret_cast<uint2 *>(a.image + xq_offset(i % DM, (nchunks + i / DM) * 8)) =
+                make_uint2(0, 0);
+    }
+    // X at the outlier columns, [j][m]
     const int n_out = tail->n_out;
     for (int i = t; i < n_out * DM; i += DTHREADS) {
         const int j = i / DM, mm = i % DM;
         tail->xo[i] = mm < a.M ? a.X[(int64_t)mm * a.K + tail->idx[j]] : __float2half_rn(0.0f);
     }
-    // the operand was written through the generic proxy; the tensor core reads it through
-    // the async proxy
-    fence_proxy_async_smem();
-    __syncthreads();
+    // the image is read by other SMs' bulk copies (async proxy)
+    fence_proxy_async_global();
+    grid_barrier(&a.scr->bar[1], a.epoch, tail, a.status);
+    const bool run = tail->bar_ok != 0;
 
     if (warp == 0) {
         // --------------------------------------------------- weight stream (TMA) ----
@@ -340,11 +414,20 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issue ----
         if (lane == 0) {
+            // the whole quantized X, written by every CTA of the grid
+            const uint32_t xbar = smem_addr(&tail->xbar);
+            const uint32_t img_bytes = (uint32_t)(a.kblocks * DBK * DM);
+            fence_proxy_async_global();
+            mbar_arrive_expect_tx(xbar, img_bytes);
+            for (uint32_t off = 0; off < img_bytes; off += 16384)
+                bulk_load_1d(smem_addr(xq) + off, a.image + off, min(16384u, img_bytes - off),
+                             xbar);
+            const bool have_x = run && wait(xbar, 0);
             const uint32_t idesc = idesc_i8(DBM, DM);
             const uint32_t xq_base = smem_addr(xq);
             int cs = 0, acc = 0;
             uint32_t cphase = 0, acc_phase = 0;
-            for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
+            for (int tile = blockIdx.x; have_x && tile < a.tiles; tile += gridDim.x) {
                 if (!wait(smem_addr(&tail->acc_empty[acc]), acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * DM);
@@ -373,6 +456,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
             }
+            if (!have_x) drain_wait(xbar, 0, a.status);   // the copies land before exit
             tc_commit(smem_addr(&tail->mma_done));
             drain_wait(smem_addr(&tail->mma_done), 0, a.status);
         }
@@ -383,7 +467,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         const float inv = 1.0f / 16129.0f;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
+        for (int tile = blockIdx.x; run && tile < a.tiles; tile += gridDim.x) {
             int okw = 0;
             if (lane == 0) okw = wait(smem_addr(&tail->acc_full[acc]), acc_phase) ? 1 : 0;
             okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -488,7 +572,10 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     a.Y = d.Y;
     a.C_debug = d.C_debug;
     a.count = d.count;
+    a.scr = d.scratch;
+    a.image = reinterpret_cast<uint8_t *>(d.scratch) + sizeof(DecodeScratch);
     a.status = d.status;
+    a.epoch = d.status.tag >> 4;
     a.M = (int)d.M;
     a.N = (int)d.N;
     a.K = (int)d.K;
@@ -519,10 +606,22 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const int grid = std::min(a.tiles, sms);
-    llmint8_decode_kernel<<<grid, DTHREADS, smem, s>>>(tm, a);
+
+    // every CTA must be resident at once (they meet at grid barriers): cooperative launch,
+    // one CTA per SM (the shared memory allows no more)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.gridDim = dim3((unsigned)std::min({a.tiles, sms, kDecodeMaxGrid}));
+    cfg.blockDim = dim3(DTHREADS);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, llmint8_decode_kernel, tm, a);
     note_launches(1);
-    return cudaGetLastError();
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace llmint8
