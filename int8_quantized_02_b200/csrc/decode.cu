@@ -25,7 +25,7 @@
 //                 the decomposition, weights from the bytes of the outlier columns) -> fp16.
 // Same method and rounding as the GEMM path (LLM.int8() summary, sections الابتكار الثاني
 // and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded; the grid
-// barriers use a fixed bound, so every CTA always reaches both.
+// barriers use a fixed bound and no atomics, so every CTA always reaches both.
 #include <cudaTypedefs.h>
 
 #include <cstddef>
@@ -140,36 +140,35 @@ __device__ __forceinline__ uint2 quant8(const float *f, float mul, uint32_t skip
     return make_uint2(lo, hi);
 }
 
-// Barrier over every CTA of the (cooperative, all-resident) grid.  The counter word holds
-// (epoch << 12) | arrivals; the first arrival of a call replaces whatever an earlier call
-// left, so the scratch needs no initialization.  Bounded by a fixed limit.
-__device__ __forceinline__ void grid_barrier(unsigned long long *word, unsigned long long epoch,
+// Barrier over every CTA of the (cooperative, all-resident) grid, without atomics: CTA g
+// publishes the call's epoch in arrived[g] (release), then one thread per peer waits
+// (acquire) until that peer's word carries the epoch.  Words left by earlier calls hold
+// older epochs, so the scratch needs no initialization.  Bounded by a fixed limit.
+__device__ __forceinline__ void grid_barrier(unsigned long long *arrived, unsigned long long epoch,
                                              DTail *tail, StatusRef status) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        const unsigned long long base = epoch << 12;
-        unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(word);
-        for (;;) {
-            const unsigned long long next = ((cur >> 12) == epoch) ? cur + 1ull : base + 1ull;
-            const unsigned long long prev = atomicCAS(word, cur, next);
-            if (prev == cur) break;
-            cur = prev;
-        }
-        const unsigned long long target = base + gridDim.x;
+        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(arrived + blockIdx.x),
+                     "l"(epoch)
+                     : "memory");
+    }
+    if (threadIdx.x < gridDim.x) {
         constexpr uint64_t kLimitNs = 1000000000ull;
         const uint64_t t0 = global_timer_ns();
         for (uint32_t it = 0;; ++it) {
             unsigned long long v;
-            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(word) : "memory");
-            if (v == target) break;
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];"
+                         : "=l"(v)
+                         : "l"(arrived + threadIdx.x)
+                         : "memory");
+            if (v == epoch) break;
             if ((it & 63u) == 0u && global_timer_ns() - t0 > kLimitNs) {
                 status.timed_out();
                 tail->bar_ok = 0;
                 break;
             }
         }
-        __threadfence();
     }
     __syncthreads();
 }
@@ -291,7 +290,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&tail->rowmax[m], __float_as_uint(rm));
     __syncthreads();
     if (t < DM) a.scr->part[blockIdx.x * DM + t] = __uint_as_float(tail->rowmax[t]);
-    grid_barrier(&a.scr->bar[0], a.epoch, tail, a.status);
+    grid_barrier(a.scr->arrived[0], a.epoch, tail, a.status);
 
     // every CTA: SCA (max over the CTAs' partial maxima), multipliers, ascending outlier list
     if (t < DM) tail->rowmax[t] = 0u;
@@ -400,7 +399,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     }
     // the image is read by other SMs' bulk copies (async proxy)
     fence_proxy_async_global();
-    grid_barrier(&a.scr->bar[1], a.epoch, tail, a.status);
+    grid_barrier(a.scr->arrived[1], a.epoch, tail, a.status);
     const bool run = tail->bar_ok != 0;
 
     if (warp == 0) {

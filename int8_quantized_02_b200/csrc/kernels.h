@@ -73,8 +73,7 @@ constexpr int kDecodeMaxGrid = 256;
 
 // Scratch the decode kernel's CTAs exchange through (global memory).
 struct DecodeScratch {
-    unsigned long long bar[2];                    // grid barriers: (epoch << 12) | arrivals
-    unsigned long long pad[6];
+    unsigned long long arrived[2][kDecodeMaxGrid];   // grid barriers: call epoch per CTA
     float part[kDecodeMaxGrid * kDecodeMaxM];     // row maxima of each CTA's columns
     uint8_t flags[kDecodeMaxK / 8];               // outlier bits of every 8-column chunk
     // followed by the quantized-X image: 16 rows x K rounded up to 128, in 128-column blocks
