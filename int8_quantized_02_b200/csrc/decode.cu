@@ -4,11 +4,9 @@
 // rest must hide under that stream.  One cooperative kernel (every CTA resident, one per SM),
 // one CTA of 512 threads per 128-row weight tile (grid-stride when there are more tiles):
 //
-//   warp 0 lane 0 TMA producer: fills a ring of shared-memory stages with 128-row x 128-byte
-//                 tiles of CB (16 KB) from the first microsecond - it needs nothing from X -
-//                 and asks L2 for the rest of its first tile, so HBM keeps streaming while
-//                 X is quantized (each weight byte is still read from HBM once per call);
-//   all warps     quantize X together.  CTA g owns 1/G of the columns: one lane per (row,
+//   all warps     first quantize X together, with no weight traffic in flight (weight requests
+//                 issued earlier queue in front of X's loads and of the exchanges through the
+//                 scratch, and that costs more than it overlaps).  CTA g owns 1/G of the columns: one lane per (row,
 //                 8-column chunk), each warp holding all 16 rows of two chunks, so the outlier
 //                 bits of a chunk (|x| >= threshold in any row) are an OR across 16 lanes and
 //                 the row maxima over the regular columns reduce in registers.  Outlier bits
@@ -17,6 +15,8 @@
 //                 int8 codes into a byte image of the tensor-core operand (16 rows, 128-byte
 //                 swizzled K-major blocks, outlier columns and padding 0); after a second
 //                 grid barrier every CTA bulk-copies the whole image into shared memory;
+//   warp 0 lane 0 TMA producer: then streams 128-row x 128-byte tiles of CB (16 KB) through
+//                 a ring of shared-memory stages (enough in flight to keep HBM busy);
 //   warp 1        tcgen05.mma kind::i8 with the weight tile as the 128-row operand and the
 //                 quantized X as the 16-column operand: D[n, m] = sum_k CB[n, k] Xq[m, k] into
 //                 a 128 x 16 int32 TMEM accumulator (double-buffered over tiles);
@@ -222,7 +222,8 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     const uint32_t tmem = tail->tmem_base;
     const BoundedWait wait{&tail->abort_flag, a.status, a.timeout_ns};
 
-    // weight stream: fill the ring now, ask L2 for the rest of the first tile
+    // weight stream state (the producer lane starts only once X is quantized: weight requests
+    // issued earlier would queue in front of X's loads and of the exchanges below)
     int stage = 0;
     uint32_t phase = 0, used = 0, last_parity = 0;
     int ptile = blockIdx.x, pit = 0;         // next (tile, k-block) to load
@@ -246,14 +247,6 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         }
         return true;
     };
-    bool producing = true;
-    if (t == 0) {
-        producing = produce(S);
-        if ((int)blockIdx.x < a.tiles)
-            for (int it = S; it < a.kblocks; ++it)
-                tma_prefetch_l2_2d(&tmCB, rotated_kblock(it, blockIdx.x, a.kblocks) * DBK,
-                                   (int)blockIdx.x * DBM);
-    }
 
     // ------------------------------------------------- quantize X across the grid ----
     // pass 1 (own columns): outlier bits (OR over the 16 lanes = rows of a chunk) to the
@@ -405,7 +398,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     if (warp == 0) {
         // --------------------------------------------------- weight stream (TMA) ----
         if (lane == 0) {
-            if (producing) produce(1 << 30);
+            if (run) produce(1 << 30);
             for (int s = 0; s < S; ++s)
                 if (used & (1u << s))
                     drain_wait(smem_addr(&tail->full[s]), (last_parity >> s) & 1u, a.status);
