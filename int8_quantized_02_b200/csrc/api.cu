@@ -35,7 +35,6 @@ struct LinearLayout {
     ScanPlan plan;
     int64_t cap = 0, pitch = 0;
     size_t partial = 0, bitmap = 0, idx = 0, sca = 0, xq = 0, xo = 0, wo = 0, total = 0;
-    size_t dscratch = 0;   // decode path (shapes with M <= 16, K <= 8192 only)
 };
 
 LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t cap) {
@@ -56,10 +55,6 @@ LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t cap) {
     L.xq = take((size_t)(M * K));
     L.xo = take((size_t)(M * L.pitch) * 2);
     L.wo = take((size_t)(N * L.pitch) * 2);
-    if (M <= kDecodeMaxM && K <= kDecodeMaxK) {
-        off = (size_t)align_up((int64_t)off, 1024);
-        L.dscratch = take((size_t)decode_scratch_bytes(K));
-    }
     L.total = off;
     return L;
 }
@@ -217,7 +212,7 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     cudaError_t e;
 
     if (use_decode_path(M, K, threshold, max_outliers)) {
-        // one cooperative launch: X quantized across the CTAs while the weight stream starts
+        // one launch: X quantized inside each cluster while the weight stream starts
         DecodeLaunch d;
         d.X = Xh;
         d.CB = CB;
@@ -227,7 +222,6 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
         d.Y = reinterpret_cast<__half *>(Y);
         d.C_debug = C_debug;
         d.count = &h->n_outliers;
-        d.scratch = at<DecodeScratch>(ws, L.dscratch);
         d.status = status;
         d.M = M;
         d.N = N;

@@ -1,22 +1,25 @@
 // Decode path of the LLM.int8() layer (few activation rows, M <= 16).
 //
 // At decode sizes the layer is bound by streaming the int8 weight CB from HBM once, and the
-// rest must hide under that stream.  One cooperative kernel (every CTA resident, one per SM),
-// one CTA of 512 threads per 128-row weight tile (grid-stride when there are more tiles):
+// rest must hide under that stream.  One kernel in clusters of 4 CTAs (512 threads, one CTA
+// per SM, one 128-row weight tile per CTA, grid-stride when there are more tiles):
 //
-//   all warps     first quantize X together, with no weight traffic in flight (weight requests
-//                 issued earlier queue in front of X's loads and of the exchanges through the
-//                 scratch, and that costs more than it overlaps).  CTA g owns 1/G of the columns: one lane per (row,
-//                 8-column chunk), each warp holding all 16 rows of two chunks, so the outlier
-//                 bits of a chunk (|x| >= threshold in any row) are an OR across 16 lanes and
-//                 the row maxima over the regular columns reduce in registers.  Outlier bits
-//                 and partial maxima go to workspace scratch; after a grid barrier every CTA
+//   warps 1..15   quantize X, each CTA of the cluster 1/4 of the columns: one lane per (row,
+//                 8-column chunk), each warp holding all 16 rows of two chunks, values in
+//                 registers.  The outlier bits of a chunk (|x| >= threshold in any row) are an
+//                 OR across its 16 lanes; the row maxima over the regular columns reduce in
+//                 registers and across warps.  Bits and partial maxima go to every CTA of the
+//                 cluster through distributed shared memory; after a cluster barrier each CTA
 //                 has SCA and the ascending outlier set, quantizes its columns and writes the
-//                 int8 codes into a byte image of the tensor-core operand (16 rows, 128-byte
-//                 swizzled K-major blocks, outlier columns and padding 0); after a second
-//                 grid barrier every CTA bulk-copies the whole image into shared memory;
-//   warp 0 lane 0 TMA producer: then streams 128-row x 128-byte tiles of CB (16 KB) through
-//                 a ring of shared-memory stages (enough in flight to keep HBM busy);
+//                 int8 codes straight into every CTA's operand buffer (128-byte swizzled
+//                 K-major, rows padded to 16, outlier columns 0), with X at its outlier
+//                 columns into their outlier tables; a second cluster barrier and every CTA
+//                 holds the whole quantized X.  Nothing of this goes through L2 or HBM but
+//                 the first load of X;
+//   warp 0        TMA producer: once its CTA's X loads have landed (weight requests issued
+//                 earlier would queue in front of them) it fills a ring of shared-memory
+//                 stages with 128-row x 128-byte tiles of CB (16 KB) - that needs nothing
+//                 from X - and keeps streaming after the barriers;
 //   warp 1        tcgen05.mma kind::i8 with the weight tile as the 128-row operand and the
 //                 quantized X as the 16-column operand: D[n, m] = sum_k CB[n, k] Xq[m, k] into
 //                 a 128 x 16 int32 TMEM accumulator (double-buffered over tiles);
@@ -24,8 +27,9 @@
 //                 + sum_{j in O} X[m, O_j] * W_o[n, O_j] + bias_n (the fp16 outlier part of
 //                 the decomposition, weights from the bytes of the outlier columns) -> fp16.
 // Same method and rounding as the GEMM path (LLM.int8() summary, sections الابتكار الثاني
-// and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded; the grid
-// barriers use a fixed bound and no atomics, so every CTA always reaches both.
+// and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded; every
+// thread of every CTA reaches each cluster barrier exactly once, with no wait in between
+// that depends on another CTA.
 #include <cudaTypedefs.h>
 
 #include <cstddef>
@@ -44,10 +48,14 @@ constexpr int DBK = 128;                // bytes of K per stage
 constexpr int DSTAGE = DBM * DBK;       // 16 KB
 constexpr int DTHREADS = 512;
 constexpr int DWARPS = DTHREADS / 32;
+constexpr int QWARPS = DWARPS - 1;      // warps 1..15 quantize X
+constexpr int QTHREADS = QWARPS * 32;
 constexpr int DMAX_STAGES = 12;
 constexpr int DCAP = kDecodeMaxOutliers;
+constexpr int CL = 4;                   // CTAs per cluster
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
-constexpr int QKEEP = 4;                // chunk pairs per warp kept in registers
+// chunk pairs per quantization warp: every pair of this CTA's columns stays in registers
+constexpr int QKEEP = (kDecodeMaxK / 16 / CL + QWARPS - 1) / QWARPS;
 
 struct DTail {
     uint64_t full[DMAX_STAGES];
@@ -55,20 +63,22 @@ struct DTail {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t mma_done;
-    uint64_t xbar;                       // the operand image has landed
+    uint64_t xin;                        // this CTA's X loads have landed
     uint32_t tmem_base;
     int abort_flag;
     int n_out;                           // outlier columns used (<= cap)
-    int bar_ok;
-    uint32_t rowmax[DM];                 // float bits (non-negative: int order == float order)
+    int pad0;
+    uint32_t pmax[DM];                   // this CTA's row maxima (float bits, >= 0)
+    float part[CL][DM];                  // row maxima of every CTA of the cluster
     float sca[DM];
     float mult[DM];                      // fl32(127 / sca), 0 for rows >= M or all-zero rows
     int warp_tot[DWARPS];
+    alignas(16) uint8_t flags[kDecodeMaxK / 8];   // outlier bits of every 8-column chunk
     int32_t idx[DCAP];                   // outlier columns (ascending)
     alignas(16) __half xo[DCAP * DM];    // X at the outlier columns, [j][m] (read as uint4)
 };
 static_assert(offsetof(DTail, xo) % 16 == 0, "xo is read with 16-byte loads");
-static_assert(offsetof(DTail, xbar) % 8 == 0, "mbarriers are 8-byte aligned");
+static_assert(offsetof(DTail, xin) % 8 == 0, "mbarriers are 8-byte aligned");
 
 struct DArgs {
     const __half *X;
@@ -79,10 +89,7 @@ struct DArgs {
     __half *Y;
     int32_t *C_debug;
     int32_t *count;
-    DecodeScratch *scr;
-    uint8_t *image;
     StatusRef status;
-    unsigned long long epoch;
     int M, N, K, cap;
     float threshold;
     int stages;
@@ -140,37 +147,9 @@ __device__ __forceinline__ uint2 quant8(const float *f, float mul, uint32_t skip
     return make_uint2(lo, hi);
 }
 
-// Barrier over every CTA of the (cooperative, all-resident) grid, without atomics: CTA g
-// publishes the call's epoch in arrived[g] (release), then one thread per peer waits
-// (acquire) until that peer's word carries the epoch.  Words left by earlier calls hold
-// older epochs, so the scratch needs no initialization.  Bounded by a fixed limit.
-__device__ __forceinline__ void grid_barrier(unsigned long long *arrived, unsigned long long epoch,
-                                             DTail *tail, StatusRef status) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(arrived + blockIdx.x),
-                     "l"(epoch)
-                     : "memory");
-    }
-    if (threadIdx.x < gridDim.x) {
-        constexpr uint64_t kLimitNs = 1000000000ull;
-        const uint64_t t0 = global_timer_ns();
-        for (uint32_t it = 0;; ++it) {
-            unsigned long long v;
-            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];"
-                         : "=l"(v)
-                         : "l"(arrived + threadIdx.x)
-                         : "memory");
-            if (v == epoch) break;
-            if ((it & 63u) == 0u && global_timer_ns() - t0 > kLimitNs) {
-                status.timed_out();
-                tail->bar_ok = 0;
-                break;
-            }
-        }
-    }
-    __syncthreads();
+__device__ __forceinline__ void st_cluster_v2(uint32_t addr, const uint2 &v) {
+    asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y)
+                 : "memory");
 }
 
 __global__ void __launch_bounds__(DTHREADS, 1)
@@ -182,21 +161,24 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     uint8_t *xq = smem + a.xq_off;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int S = a.stages;
+    const uint32_t rank = cluster_ctarank();
     const int m = lane & 15;                 // quantization: the row this lane handles
     const int half = lane >> 4;              //               which chunk of the warp's pair
+    const int qw = warp - 1;                 // quantization warp index (warps 1..15)
     const int nchunks = a.K / 8;
     const int npairs = nchunks / 2;          // K is a multiple of 16
-    const int pp = (npairs + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int p0 = (int)blockIdx.x * pp, p1 = min(npairs, p0 + pp);   // this CTA's pairs
+    const int pp = (npairs + CL - 1) / CL;
+    const int p0 = (int)rank * pp, p1 = min(npairs, p0 + pp);   // this CTA's pairs
     const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
 
-    // this CTA's columns of X first, ahead of every weight request
+    // this CTA's columns of X, first of all memory traffic
     uint4 keep[QKEEP];
 #pragma unroll
     for (int i = 0; i < QKEEP; ++i) {
-        const int p = p0 + warp + i * DWARPS;
-        keep[i] = (p < p1 && m < a.M) ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
-                                      : make_uint4(0, 0, 0, 0);
+        const int p = p0 + qw + i * QWARPS;
+        keep[i] = (warp > 0 && p < p1 && m < a.M)
+                      ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
+                      : make_uint4(0, 0, 0, 0);
     }
     if (t == 0) {
         for (int s = 0; s < S; ++s) {
@@ -208,22 +190,23 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             mbar_init(smem_addr(&tail->acc_empty[s]), 4);
         }
         mbar_init(smem_addr(&tail->mma_done), 1);
-        mbar_init(smem_addr(&tail->xbar), 1);
+        mbar_init(smem_addr(&tail->xin), 1);
         tail->abort_flag = 0;
-        tail->bar_ok = 1;
         fence_mbar_init();
         tma_prefetch_desc(&tmCB);
     }
-    if (t < DM) tail->rowmax[t] = 0u;
+    if (t < DM) tail->pmax[t] = 0u;
     if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), 32);
+    // zero the operand (rows >= M and columns >= K must read as 0)
+    for (int i = t; i < a.kblocks * DBK * DM / 16; i += DTHREADS)
+        reinterpret_cast<uint4 *>(xq)[i] = make_uint4(0, 0, 0, 0);
     tc_fence_before();
-    __syncthreads();
+    // every CTA's barriers and zeroed buffers exist before a peer writes into them
+    cluster_barrier_all();
     tc_fence_after();
     const uint32_t tmem = tail->tmem_base;
     const BoundedWait wait{&tail->abort_flag, a.status, a.timeout_ns};
 
-    // weight stream state (the producer lane starts only once X is quantized: weight requests
-    // issued earlier would queue in front of X's loads and of the exchanges below)
     int stage = 0;
     uint32_t phase = 0, used = 0, last_parity = 0;
     int ptile = blockIdx.x, pit = 0;         // next (tile, k-block) to load
@@ -248,81 +231,81 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         return true;
     };
 
-    // ------------------------------------------------- quantize X across the grid ----
-    // pass 1 (own columns): outlier bits (OR over the 16 lanes = rows of a chunk) to the
-    // scratch, row maxima over the regular columns
     uint32_t fl[QKEEP];
-    float rm = 0.0f;
+    if (warp == 0) {
+        // the ring fill needs no free slot (they all start empty) and nothing from X; it
+        // waits for this CTA's X loads so as not to queue in front of them
+        if (lane == 0) {
+            drain_wait(smem_addr(&tail->xin), 0, a.status);
+            produce(S);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------- quantize X, this CTA's quarter of the columns ----
+        float rm = 0.0f;
 #pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        fl[i] = 0;
-        const int p = p0 + warp + i * DWARPS;
-        if (p < p1) {                        // uniform over the warp
-            float f[8];
-            unpack8(keep[i], f);
-            uint32_t b = outlier_bits(f, a.threshold);
+        for (int i = 0; i < QKEEP; ++i) {
+            fl[i] = 0;
+            const int p = p0 + qw + i * QWARPS;
+            if (p < p1) {                    // uniform over the warp
+                float f[8];
+                unpack8(keep[i], f);
+                uint32_t b = outlier_bits(f, a.threshold);
 #pragma unroll
-            for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
-            fl[i] = b;
-            if (m == 0) a.scr->flags[2 * p + half] = (uint8_t)b;
-            rm = masked_max(f, b, rm);
+                for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
+                fl[i] = b;
+                if (m == 0) {
+                    const uint32_t dst = smem_addr(&tail->flags[2 * p + half]);
+                    for (int r = 0; r < CL; ++r) st_cluster_u8(map_to_rank(dst, (uint32_t)r), b);
+                }
+                rm = masked_max(f, b, rm);
+            }
+        }
+        rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 16));
+        if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&tail->pmax[m], __float_as_uint(rm));
+        named_barrier(1, QTHREADS);
+        if (t == 32) mbar_arrive(smem_addr(&tail->xin));   // X is in: the ring may fill
+        if (t >= 32 && t < 32 + DM) {
+            const int q = t - 32;
+            const uint32_t dst = smem_addr(&tail->part[rank][q]);
+            for (int r = 0; r < CL; ++r)
+                st_cluster_u32(map_to_rank(dst, (uint32_t)r), tail->pmax[q]);
         }
     }
-    for (int p = p0 + warp + QKEEP * DWARPS; p < p1; p += DWARPS) {
-        const uint4 v = m < a.M ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
-                                : make_uint4(0, 0, 0, 0);
-        float f[8];
-        unpack8(v, f);
-        uint32_t b = outlier_bits(f, a.threshold);
-#pragma unroll
-        for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
-        if (m == 0) a.scr->flags[2 * p + half] = (uint8_t)b;
-        rm = masked_max(f, b, rm);
-    }
-    rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 16));
-    if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&tail->rowmax[m], __float_as_uint(rm));
-    __syncthreads();
-    if (t < DM) a.scr->part[blockIdx.x * DM + t] = __uint_as_float(tail->rowmax[t]);
-    grid_barrier(a.scr->arrived[0], a.epoch, tail, a.status);
+    // ---------------------------------- exchange 1: outlier bits and row maxima ----
+    __syncwarp();
+    cluster_barrier_all();
 
-    // every CTA: SCA (max over the CTAs' partial maxima), multipliers, ascending outlier list
-    if (t < DM) tail->rowmax[t] = 0u;
-    __syncthreads();
-    {
-        float r = 0.0f;
-        for (int i = t; i < (int)gridDim.x * DM; i += DTHREADS)   // DTHREADS % DM == 0
-            r = fmaxf(r, __ldcg(&a.scr->part[i]));
-        // lanes l and l + 16 hold the same row
-        r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, 16));
-        if (half == 0 && r > 0.0f) atomicMax(&tail->rowmax[m], __float_as_uint(r));
-    }
-    {
-        const int per = (nchunks + DTHREADS - 1) / DTHREADS;   // contiguous chunks per thread
-        const int c0 = t * per, c1 = min(nchunks, c0 + per);
-        uint32_t bits[(kDecodeMaxK / 8 + DTHREADS - 1) / DTHREADS];
-        int cnt = 0;
-#pragma unroll
-        for (int j = 0; j < (int)(sizeof(bits) / sizeof(bits[0])); ++j) {
-            bits[j] = (c0 + j < c1) ? (uint32_t)__ldcg(&a.scr->flags[c0 + j]) : 0u;
-            cnt += __popc(bits[j]);
+    if (warp > 0) {
+        const int q = t - 32;                // 0 .. QTHREADS-1
+        if (q < DM) {
+            float amax = 0.0f;
+            for (int r = 0; r < CL; ++r) amax = fmaxf(amax, tail->part[r][q]);
+            tail->sca[q] = amax;
+            tail->mult[q] = (q < a.M && amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
         }
+        // ascending outlier list: contiguous chunks per thread, scan over warps 1..15
+        const int per = (nchunks + QTHREADS - 1) / QTHREADS;
+        const int c0 = q * per, c1 = min(nchunks, c0 + per);
+        int cnt = 0;
+        for (int c = c0; c < c1; ++c) cnt += __popc(tail->flags[c]);
         int incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += y;
         }
-        if (lane == 31) tail->warp_tot[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            const int v0 = lane < DWARPS ? tail->warp_tot[lane] : 0;
+        if (lane == 31) tail->warp_tot[qw] = incl;
+        named_barrier(1, QTHREADS);
+        if (qw == 0) {
+            const int v0 = lane < QWARPS ? tail->warp_tot[lane] : 0;
             int x = v0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, x, o);
                 if (lane >= o) x += y;
             }
-            if (lane < DWARPS) tail->warp_tot[lane] = x - v0;
+            if (lane < QWARPS) tail->warp_tot[lane] = x - v0;
             if (lane == 31) {
                 tail->n_out = min(x, a.cap);
                 if (blockIdx.x == 0) {
@@ -331,74 +314,61 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 }
             }
         }
-        __syncthreads();
-        int pos = tail->warp_tot[warp] + incl - cnt;
-#pragma unroll
-        for (int j = 0; j < (int)(sizeof(bits) / sizeof(bits[0])); ++j) {
-            uint32_t b = bits[j];
+        named_barrier(1, QTHREADS);
+        int pos = tail->warp_tot[qw] + incl - cnt;
+        for (int c = c0; c < c1; ++c) {
+            uint32_t b = tail->flags[c];
             while (b) {
                 const int e = __ffs(b) - 1;
                 b &= b - 1;
-                if (pos < a.cap) tail->idx[pos] = (c0 + j) * 8 + e;
+                if (pos < a.cap) tail->idx[pos] = c * 8 + e;
                 ++pos;
             }
         }
-    }
-    if (t < DM) {
-        const float amax = __uint_as_float(tail->rowmax[t]);
-        tail->sca[t] = amax;
-        tail->mult[t] = (t < a.M && amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
-    }
-    __syncthreads();
+        named_barrier(1, QTHREADS);
 
-    // pass 2 (own columns): int8 codes into the operand image, all 16 rows
-    const float mul = tail->mult[m];
+        // int8 codes of this CTA's columns into every CTA's operand; X at outlier columns
+        const float mul = tail->mult[m];
+        const int n_out = tail->n_out;
+        const uint32_t xq_base = smem_addr(xq);
+        const uint32_t xo_base = smem_addr(tail->xo);
 #pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        const int p = p0 + warp + i * DWARPS;
-        if (p < p1) {
-            const int c = 2 * p + half;
-            uint2 q = make_uint2(0, 0);
-            if (mul > 0.0f) {
+        for (int i = 0; i < QKEEP; ++i) {
+            const int p = p0 + qw + i * QWARPS;
+            if (p < p1) {
+                const int c = 2 * p + half;
                 float f[8];
                 unpack8(keep[i], f);
-                q = quant8(f, mul, fl[i]);
+                if (mul > 0.0f) {
+                    const uint2 qv = quant8(f, mul, fl[i]);
+                    const uint32_t dst = xq_base + xq_offset(m, c * 8);
+                    for (int r = 0; r < CL; ++r) st_cluster_v2(map_to_rank(dst, (uint32_t)r), qv);
+                }
+                if (fl[i]) {
+                    // this chunk holds outlier columns: find their list positions
+                    for (int j = 0; j < n_out; ++j) {
+                        const int col = tail->idx[j];
+                        if ((col >> 3) == c) {
+                            const __half hv = __float2half_rn(m < a.M ? f[col & 7] : 0.0f);
+                            const uint32_t dst = xo_base + 2u * (uint32_t)(j * DM + m);
+                            for (int r = 0; r < CL; ++r)
+                                st_cluster_u16(map_to_rank(dst, (uint32_t)r),
+                                               __half_as_ushort(hv));
+                        }
+                    }
+                }
             }
-            *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8)) = q;
         }
     }
-    for (int p = p0 + warp + QKEEP * DWARPS; p < p1; p += DWARPS) {
-        const int c = 2 * p + half;
-        uint2 q = make_uint2(0, 0);
-        if (mul > 0.0f) {
-            float f[8];
-            unpack8(__ldg(X4 + (int64_t)m * nchunks + c), f);
-            q = quant8(f, mul, (uint32_t)__ldcg(&a.scr->flags[c]));
-        }
-        *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8)) = q;
-    }
-    if (blockIdx.x == 0) {
-        // the padding columns of the image
-        const int kpad_chunks = a.kblocks * (DBK / 8);
-        for (int i = t; i < (kpad_chunks - nchunks) * DM; i += DTHREADS)
-            *reinterpret_cast<uint2 *>(a.image + xq_offset(i % DM, (nchunks + i / DM) * 8)) =
-                make_uint2(0, 0);
-    }
-    // X at the outlier columns, [j][m]
+    // ------------------------------------------- exchange 2: the quantized operand ----
+    __syncwarp();
+    cluster_barrier_all();
     const int n_out = tail->n_out;
-    for (int i = t; i < n_out * DM; i += DTHREADS) {
-        const int j = i / DM, mm = i % DM;
-        tail->xo[i] = mm < a.M ? a.X[(int64_t)mm * a.K + tail->idx[j]] : __float2half_rn(0.0f);
-    }
-    // the image is read by other SMs' bulk copies (async proxy)
-    fence_proxy_async_global();
-    grid_barrier(a.scr->arrived[1], a.epoch, tail, a.status);
-    const bool run = tail->bar_ok != 0;
 
     if (warp == 0) {
         // --------------------------------------------------- weight stream (TMA) ----
         if (lane == 0) {
-            if (run) produce(1 << 30);
+            produce(1 << 30);
             for (int s = 0; s < S; ++s)
                 if (used & (1u << s))
                     drain_wait(smem_addr(&tail->full[s]), (last_parity >> s) & 1u, a.status);
@@ -406,20 +376,14 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issue ----
         if (lane == 0) {
-            // the whole quantized X, written by every CTA of the grid
-            const uint32_t xbar = smem_addr(&tail->xbar);
-            const uint32_t img_bytes = (uint32_t)(a.kblocks * DBK * DM);
-            fence_proxy_async_global();
-            mbar_arrive_expect_tx(xbar, img_bytes);
-            for (uint32_t off = 0; off < img_bytes; off += 16384)
-                bulk_load_1d(smem_addr(xq) + off, a.image + off, min(16384u, img_bytes - off),
-                             xbar);
-            const bool have_x = run && wait(xbar, 0);
+            // peers wrote the operand through the generic proxy; the tensor core reads it
+            // through the async proxy
+            fence_proxy_async_smem();
             const uint32_t idesc = idesc_i8(DBM, DM);
             const uint32_t xq_base = smem_addr(xq);
             int cs = 0, acc = 0;
             uint32_t cphase = 0, acc_phase = 0;
-            for (int tile = blockIdx.x; have_x && tile < a.tiles; tile += gridDim.x) {
+            for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
                 if (!wait(smem_addr(&tail->acc_empty[acc]), acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * DM);
@@ -448,7 +412,6 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
             }
-            if (!have_x) drain_wait(xbar, 0, a.status);   // the copies land before exit
             tc_commit(smem_addr(&tail->mma_done));
             drain_wait(smem_addr(&tail->mma_done), 0, a.status);
         }
@@ -459,7 +422,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         const float inv = 1.0f / 16129.0f;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; run && tile < a.tiles; tile += gridDim.x) {
+        for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
             int okw = 0;
             if (lane == 0) okw = wait(smem_addr(&tail->acc_full[acc]), acc_phase) ? 1 : 0;
             okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -535,25 +498,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     static std::mutex mu;
-    static int sms_cache[64] = {0};
+    static int max_clusters[64] = {0};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    int sms;
-    {
-        std::lock_guard<std::mutex> lk(mu);
-        if (sms_cache[dev] == 0) {
-            int n = 0;
-            err = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-            if (err != cudaSuccess) return err;
-            err = cudaFuncSetAttribute(llmint8_decode_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT);
-            if (err != cudaSuccess) return err;
-            sms_cache[dev] = n;
-        }
-        sms = sms_cache[dev];
-    }
 
     DArgs a;
     a.X = d.X;
@@ -564,10 +513,7 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     a.Y = d.Y;
     a.C_debug = d.C_debug;
     a.count = d.count;
-    a.scr = d.scratch;
-    a.image = reinterpret_cast<uint8_t *>(d.scratch) + sizeof(DecodeScratch);
     a.status = d.status;
-    a.epoch = d.status.tag >> 4;
     a.M = (int)d.M;
     a.N = (int)d.N;
     a.K = (int)d.K;
@@ -587,6 +533,38 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     const int smem = (int)(a.tail_off + sizeof(DTail) + 1024);
     if (smem > SMEM_LIMIT) return cudaErrorInvalidValue;
 
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(DTHREADS);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (max_clusters[dev] == 0) {
+            err = cudaFuncSetAttribute(llmint8_decode_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT);
+            if (err != cudaSuccess) return err;
+            cudaLaunchConfig_t qc = cfg;
+            qc.gridDim = dim3(CL);
+            qc.dynamicSmemBytes = (size_t)SMEM_LIMIT;
+            int n = 0;
+            err = cudaOccupancyMaxActiveClusters(&n, llmint8_decode_kernel, &qc);
+            if (err != cudaSuccess) return err;
+            if (n < 1) return cudaErrorInvalidConfiguration;
+            max_clusters[dev] = n;
+        }
+        clusters = max_clusters[dev];
+    }
+    clusters = std::min<int>(clusters, (int)ceil_div(a.tiles, CL));
+    cfg.gridDim = dim3((unsigned)(clusters * CL));
+
     auto enc = encoder();
     if (!enc) return cudaErrorInvalidValue;
     CUtensorMap tm;
@@ -598,19 +576,6 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-
-    // every CTA must be resident at once (they meet at grid barriers): cooperative launch,
-    // one CTA per SM (the shared memory allows no more)
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.gridDim = dim3((unsigned)std::min({a.tiles, sms, kDecodeMaxGrid}));
-    cfg.blockDim = dim3(DTHREADS);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     err = cudaLaunchKernelEx(&cfg, llmint8_decode_kernel, tm, a);
     note_launches(1);
     return err != cudaSuccess ? err : cudaGetLastError();

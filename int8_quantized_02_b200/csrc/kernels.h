@@ -63,28 +63,11 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s);
 
 namespace llmint8 {
 
-// Decode path (M <= kDecodeMaxM, K <= kDecodeMaxK): one cooperative weight-streaming
-// tcgen05 kernel; its CTAs quantize X together through workspace scratch while the weight
-// stream starts.
+// Decode path (M <= kDecodeMaxM, K <= kDecodeMaxK): one weight-streaming tcgen05 kernel in
+// clusters of CTAs that quantize X together through distributed shared memory.
 constexpr int kDecodeMaxM = 16;
 constexpr int kDecodeMaxK = 8192;
 constexpr int kDecodeMaxOutliers = 256;
-constexpr int kDecodeMaxGrid = 256;
-
-// Scratch the decode kernel's CTAs exchange through (global memory).
-struct DecodeScratch {
-    unsigned long long arrived[2][kDecodeMaxGrid];   // grid barriers: call epoch per CTA
-    float part[kDecodeMaxGrid * kDecodeMaxM];     // row maxima of each CTA's columns
-    uint8_t flags[kDecodeMaxK / 8];               // outlier bits of every 8-column chunk
-    // followed by the quantized-X image: 16 rows x K rounded up to 128, in 128-column blocks
-    // of two 1024-byte swizzled 8-row atoms (a byte copy of the tensor-core operand)
-};
-__host__ __device__ constexpr int64_t decode_image_bytes(int64_t K) {
-    return kDecodeMaxM * ((K + 127) / 128 * 128);
-}
-__host__ __device__ constexpr int64_t decode_scratch_bytes(int64_t K) {
-    return (int64_t)sizeof(DecodeScratch) + decode_image_bytes(K);
-}
 
 struct DecodeLaunch {
     const __half *X;         // [M, K]
@@ -95,7 +78,6 @@ struct DecodeLaunch {
     __half *Y;               // [M, N]
     int32_t *C_debug;        // [M, N] or null
     int32_t *count;          // device outlier count (workspace header)
-    DecodeScratch *scratch;  // decode_scratch_bytes(K), 1024-byte aligned
     StatusRef status;
     int64_t M, N, K, cap;
     float threshold;
