@@ -35,6 +35,7 @@ struct LinearLayout {
     ScanPlan plan;
     int64_t cap = 0, pitch = 0;
     size_t partial = 0, bitmap = 0, idx = 0, sca = 0, xq = 0, xo = 0, wo = 0, total = 0;
+    size_t dimage = 0, dtables = 0;   // decode path (shapes with M <= 16, K <= 8192 only)
 };
 
 LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t cap) {
@@ -55,6 +56,11 @@ LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t cap) {
     L.xq = take((size_t)(M * K));
     L.xo = take((size_t)(M * L.pitch) * 2);
     L.wo = take((size_t)(N * L.pitch) * 2);
+    if (M <= kDecodeMaxM && K <= kDecodeMaxK) {
+        off = (size_t)align_up((int64_t)off, 1024);
+        L.dimage = take((size_t)decode_image_bytes(K));
+        L.dtables = take(sizeof(DecodeTables));
+    }
     L.total = off;
     return L;
 }
@@ -94,7 +100,7 @@ cudaError_t record_profile_event(cudaEvent_t ev, cudaStream_t s) {
 
 llmint8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA; }
 
-// The decode path covers few activation rows and an X whose quantized form fits in shared
+// The decode path covers few activation rows and an X whose quantized image fits in shared
 // memory; threshold <= 0 (every column fp16) goes through the GEMM path.
 bool use_decode_path(int64_t M, int64_t K, float threshold, int64_t cap) {
     return M <= kDecodeMaxM && K <= kDecodeMaxK && threshold > 0.0f &&
@@ -212,7 +218,7 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     cudaError_t e;
 
     if (use_decode_path(M, K, threshold, max_outliers)) {
-        // one launch: X quantized inside each cluster while the weight stream starts
+        // quantize X once, then the weight-streaming tcgen05 kernel (programmatic dependent)
         DecodeLaunch d;
         d.X = Xh;
         d.CB = CB;
@@ -222,6 +228,8 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
         d.Y = reinterpret_cast<__half *>(Y);
         d.C_debug = C_debug;
         d.count = &h->n_outliers;
+        d.image = at<uint8_t>(ws, L.dimage);
+        d.tables = at<DecodeTables>(ws, L.dtables);
         d.status = status;
         d.M = M;
         d.N = N;

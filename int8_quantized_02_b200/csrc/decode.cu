@@ -1,35 +1,35 @@
 // Decode path of the LLM.int8() layer (few activation rows, M <= 16).
 //
-// At decode sizes the layer is bound by streaming the int8 weight CB from HBM once, and the
-// rest must hide under that stream.  One kernel in clusters of 4 CTAs (512 threads, one CTA
-// per SM, one 128-row weight tile per CTA, grid-stride when there are more tiles):
+// At decode sizes the layer is bound by streaming the int8 weight CB from HBM once, and
+// everything else must hide under that stream.  Two kernels:
 //
-//   warps 1..15   quantize X, each CTA of the cluster 1/4 of the columns: one lane per (row,
-//                 8-column chunk), each warp holding all 16 rows of two chunks, values in
-//                 registers.  The outlier bits of a chunk (|x| >= threshold in any row) are an
-//                 OR across its 16 lanes; the row maxima over the regular columns reduce in
-//                 registers and across warps.  Bits and partial maxima go to every CTA of the
-//                 cluster through distributed shared memory; after a cluster barrier each CTA
-//                 has SCA and the ascending outlier set, quantizes its columns and writes the
-//                 int8 codes straight into every CTA's operand buffer (128-byte swizzled
-//                 K-major, rows padded to 16, outlier columns 0), with X at its outlier
-//                 columns into their outlier tables; a second cluster barrier and every CTA
-//                 holds the whole quantized X.  Nothing of this goes through L2 or HBM but
-//                 the first load of X;
-//   warp 0        TMA producer: once its CTA's X loads have landed (weight requests issued
-//                 earlier would queue in front of them) it fills a ring of shared-memory
-//                 stages with 128-row x 128-byte tiles of CB (16 KB) - that needs nothing
-//                 from X - and keeps streaming after the barriers;
-//   warp 1        tcgen05.mma kind::i8 with the weight tile as the 128-row operand and the
-//                 quantized X as the 16-column operand: D[n, m] = sum_k CB[n, k] Xq[m, k] into
-//                 a 128 x 16 int32 TMEM accumulator (double-buffered over tiles);
+// llmint8_decode_quantize_kernel (one cluster of 8 CTAs x 1024 threads) quantizes X once:
+//   one thread per (row, 8-column chunk), each warp holding all 16 rows of two chunks, CTA r
+//   of the cluster 1/8 of the columns.  The outlier bits of a chunk (|x| >= threshold in any
+//   row) are an OR across 16 lanes; the row maxima over the regular columns reduce in
+//   registers, across warps, and across the cluster through distributed shared memory
+//   (one hardware cluster barrier); the int8 codes go into the workspace as a byte-exact
+//   image of the tensor-core operand (16 rows, 128-byte swizzled K-major blocks, outlier
+//   columns and padding 0), next to a table of SCA, the ascending outlier columns and X at
+//   those columns.  It lets its dependent launch at once.
+//
+// llmint8_decode_kernel (one CTA per 128-row weight tile, programmatic dependent launch):
+//   warp 0        TMA producer: streams 128-row x 128-byte tiles of CB (16 KB) through a ring
+//                 of shared-memory stages from its first cycle - it needs nothing from X - and
+//                 asks L2 for the rest of its first tile as well, so that HBM keeps streaming
+//                 while the MMA waits for the quantized X (every weight byte is still read
+//                 from HBM once per call; the later stage loads find it in L2);
+//   warp 1        waits until the quantize kernel publishes (an acquire on the call epoch it
+//                 stores last), bulk-copies the operand image and the table into shared
+//                 memory, then issues tcgen05.mma kind::i8
+//                 with the weight tile as the 128-row operand and the quantized X as the
+//                 16-column operand: D[n, m] = sum_k CB[n, k] Xq[m, k] into a 128 x 16 int32
+//                 TMEM accumulator (double-buffered over tiles);
 //   warps 4..7    epilogue: D -> registers; y = D * SCA_m * SCB_n / 127^2
 //                 + sum_{j in O} X[m, O_j] * W_o[n, O_j] + bias_n (the fp16 outlier part of
 //                 the decomposition, weights from the bytes of the outlier columns) -> fp16.
 // Same method and rounding as the GEMM path (LLM.int8() summary, sections الابتكار الثاني
-// and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded; every
-// thread of every CTA reaches each cluster barrier exactly once, with no wait in between
-// that depends on another CTA.
+// and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include <cstddef>
@@ -46,59 +46,17 @@ constexpr int DM = kDecodeMaxM;         // activation rows held (MMA N)
 constexpr int DBM = 128;                // weight rows per tile (MMA M)
 constexpr int DBK = 128;                // bytes of K per stage
 constexpr int DSTAGE = DBM * DBK;       // 16 KB
-constexpr int DTHREADS = 512;
-constexpr int DWARPS = DTHREADS / 32;
-constexpr int QWARPS = DWARPS - 1;      // warps 1..15 quantize X
-constexpr int QTHREADS = QWARPS * 32;
+constexpr int DTHREADS = 256;
 constexpr int DMAX_STAGES = 12;
-constexpr int DCAP = kDecodeMaxOutliers;
-constexpr int CL = 4;                   // CTAs per cluster
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
-// chunk pairs per quantization warp: every pair of this CTA's columns stays in registers
-constexpr int QKEEP = (kDecodeMaxK / 16 / CL + QWARPS - 1) / QWARPS;
-
-struct DTail {
-    uint64_t full[DMAX_STAGES];
-    uint64_t empty[DMAX_STAGES];
-    uint64_t acc_full[2];
-    uint64_t acc_empty[2];
-    uint64_t mma_done;
-    uint64_t xin;                        // this CTA's X loads have landed
-    uint32_t tmem_base;
-    int abort_flag;
-    int n_out;                           // outlier columns used (<= cap)
-    int pad0;
-    uint32_t pmax[DM];                   // this CTA's row maxima (float bits, >= 0)
-    float part[CL][DM];                  // row maxima of every CTA of the cluster
-    float sca[DM];
-    float mult[DM];                      // fl32(127 / sca), 0 for rows >= M or all-zero rows
-    int warp_tot[DWARPS];
-    alignas(16) uint8_t flags[kDecodeMaxK / 8];   // outlier bits of every 8-column chunk
-    int32_t idx[DCAP];                   // outlier columns (ascending)
-    alignas(16) __half xo[DCAP * DM];    // X at the outlier columns, [j][m] (read as uint4)
-};
-static_assert(offsetof(DTail, xo) % 16 == 0, "xo is read with 16-byte loads");
-static_assert(offsetof(DTail, xin) % 8 == 0, "mbarriers are 8-byte aligned");
-
-struct DArgs {
-    const __half *X;
-    const int8_t *CB;
-    const float *SCB;
-    const __half *W16;
-    const __half *bias;
-    __half *Y;
-    int32_t *C_debug;
-    int32_t *count;
-    StatusRef status;
-    int M, N, K, cap;
-    float threshold;
-    int stages;
-    int kblocks;
-    int tiles;
-    uint32_t xq_off;                     // byte offsets in shared memory
-    uint32_t tail_off;
-    uint64_t timeout_ns;
-};
+constexpr int QTHREADS = 1024;          // quantize kernel: one cluster of QCL CTAs
+constexpr int QWARPS = QTHREADS / 32;
+constexpr int QCL = 8;
+// chunk pairs (16 columns) per warp: K <= kDecodeMaxK keeps every item in registers
+constexpr int QKEEP = (kDecodeMaxK / 16 / QCL + QWARPS - 1) / QWARPS;
+// k-blocks of a CTA's first tile requested into L2 ahead of the stage ring, so that HBM keeps
+// streaming while the first MMA waits for the quantized X
+constexpr int kPrefetchBlocks = 64;
 
 __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&v);
@@ -147,10 +105,194 @@ __device__ __forceinline__ uint2 quant8(const float *f, float mul, uint32_t skip
     return make_uint2(lo, hi);
 }
 
-__device__ __forceinline__ void st_cluster_v2(uint32_t addr, const uint2 &v) {
-    asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y)
-                 : "memory");
+struct QArgs {
+    const __half *X;
+    int M, K, cap;
+    float threshold;
+    uint8_t *image;
+    DecodeTables *tables;
+    int32_t *count;
+    StatusRef status;
+    unsigned long long epoch;
+};
+
+// One cluster of QCL CTAs.  CTA r owns the chunk pairs [r*PP, (r+1)*PP); one thread per
+// (row, chunk) item, its values kept in registers between the two passes.
+__global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(const QArgs a) {
+    // launched as a programmatic dependent of whatever precedes it in the stream: wait for it
+    // before touching X or the workspace, then let the weight-streaming kernel launch
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ float part[QCL][DM];          // row maxima of every CTA of the cluster
+    __shared__ uint32_t pmax[DM];            // this CTA's (float bits, >= 0: int order)
+    __shared__ float mult[DM];
+    __shared__ uint8_t flags_all[kDecodeMaxK / 8];   // CTA 0: outlier bits of every chunk
+    __shared__ int n_out_s;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int m = lane & 15;                 // the row this thread handles
+    const int half = lane >> 4;              // which chunk of the warp's pair
+    const uint32_t r = cluster_ctarank();
+    const int nchunks = a.K / 8;
+    const int npairs = nchunks / 2;          // K is a multiple of 16
+    const int pp = (npairs + QCL - 1) / QCL;
+    const int p0 = (int)r * pp, p1 = min(npairs, p0 + pp);
+    const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
+
+    uint4 v[QKEEP];
+#pragma unroll
+    for (int i = 0; i < QKEEP; ++i) {
+        const int p = p0 + warp + i * QWARPS;
+        v[i] = (p < p1 && m < a.M) ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
+                                   : make_uint4(0, 0, 0, 0);
+    }
+    if (t < DM) pmax[t] = 0u;
+    __syncthreads();
+
+    // pass 1: outlier bits of each chunk (OR over its 16 lanes = rows), published to CTA 0;
+    // row maxima over the regular columns
+    uint32_t fl[QKEEP];
+    float rm = 0.0f;
+    const uint32_t flags0 = map_to_rank(smem_addr(flags_all), 0);
+#pragma unroll
+    for (int i = 0; i < QKEEP; ++i) {
+        fl[i] = 0;
+        const int p = p0 + warp + i * QWARPS;
+        if (p < p1) {                        // uniform over the warp
+            float f[8];
+            unpack8(v[i], f);
+            uint32_t b = outlier_bits(f, a.threshold);
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
+            fl[i] = b;
+            if (m == 0) st_cluster_u8(flags0 + (uint32_t)(2 * p + half), b);
+            rm = masked_max(f, b, rm);
+        }
+    }
+    rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 16));
+    if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&pmax[m], __float_as_uint(rm));
+    __syncthreads();
+    if (t < DM) {
+        const uint32_t dst = smem_addr(&part[r][t]);
+        for (int rr = 0; rr < QCL; ++rr) st_cluster_u32(map_to_rank(dst, (uint32_t)rr), pmax[t]);
+    }
+    // every CTA's flags and partial maxima are in place after this
+    cluster_barrier_all();
+
+    if (t < DM) {
+        float amax = 0.0f;
+        for (int rr = 0; rr < QCL; ++rr) amax = fmaxf(amax, part[rr][t]);
+        mult[t] = (t < a.M && amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
+        if (r == 0) a.tables->sca[t] = amax;
+    }
+    __syncthreads();
+
+    // pass 2: every (row, chunk) of this CTA into the operand image; rows >= M, all-zero rows
+    // and outlier columns are written as 0
+    const float mul = mult[m];
+#pragma unroll
+    for (int i = 0; i < QKEEP; ++i) {
+        const int p = p0 + warp + i * QWARPS;
+        if (p < p1) {
+            const int c = 2 * p + half;
+            uint2 q = make_uint2(0, 0);
+            if (mul > 0.0f) {
+                float f[8];
+                unpack8(v[i], f);
+                q = quant8(f, mul, fl[i]);
+            }
+            *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8)) = q;
+        }
+    }
+    // every CTA's part of the image is written before CTA 0 publishes it
+    __threadfence();
+    __syncwarp();
+    cluster_barrier_all();
+    if (r != 0) return;   // nothing of this CTA is read by its peers any more
+
+    // CTA 0: padding columns of the image, ascending outlier list, count, status, X there
+    const int kpad_chunks = (a.K + 127) / 128 * 16;
+    for (int i = t; i < (kpad_chunks - nchunks) * DM; i += QTHREADS) {
+        const int c = nchunks + i / DM, mm = i % DM;
+        *reinterpret_cast<uint2 *>(a.image + xq_offset(mm, c * 8)) = make_uint2(0, 0);
+    }
+    if (warp == 0) {
+        const int per = (nchunks + 31) / 32;
+        const int c0 = lane * per, c1 = min(nchunks, c0 + per);
+        int cnt = 0;
+        for (int c = c0; c < c1; ++c) cnt += __popc(flags_all[c]);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int pos = incl - cnt;
+        for (int c = c0; c < c1; ++c) {
+            uint32_t b = flags_all[c];
+            while (b) {
+                const int e = __ffs(b) - 1;
+                b &= b - 1;
+                if (pos < a.cap) a.tables->idx[pos] = c * 8 + e;
+                ++pos;
+            }
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        if (lane == 0) {
+            n_out_s = min(total, a.cap);
+            a.tables->n_out = n_out_s;
+            *a.count = total;
+            a.status.set(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
+        }
+    }
+    __syncthreads();
+    const int n_out = n_out_s;
+    for (int i = t; i < n_out * DM; i += QTHREADS) {
+        const int j = i / DM, mm = i % DM;
+        a.tables->xo[i] = mm < a.M ? a.X[(int64_t)mm * a.K + a.tables->idx[j]]
+                                   : __float2half_rn(0.0f);
+    }
+    // publish: the image and table are complete (the dependent kernel bulk-copies them)
+    __threadfence();
+    fence_proxy_async_global();
+    __syncthreads();
+    if (t == 0)
+        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&a.tables->ready), "l"(a.epoch)
+                     : "memory");
 }
+
+struct DTail {
+    uint64_t full[DMAX_STAGES];
+    uint64_t empty[DMAX_STAGES];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t mma_done;
+    uint64_t xbar;                       // operand image and table have landed
+    uint32_t tmem_base;
+    int abort_flag;
+    alignas(16) DecodeTables tab;
+};
+static_assert(offsetof(DTail, tab) % 16 == 0, "the table is a bulk-copy destination");
+static_assert(offsetof(DTail, xbar) % 8 == 0, "mbarriers are 8-byte aligned");
+
+struct DArgs {
+    unsigned long long epoch;
+    const int8_t *CB;
+    const float *SCB;
+    const __half *W16;
+    const __half *bias;
+    __half *Y;
+    int32_t *C_debug;
+    const uint8_t *image;
+    const DecodeTables *tables;
+    StatusRef status;
+    int M, N, K;
+    int stages;
+    int kblocks;
+    int tiles;
+    uint32_t xq_off;                     // byte offsets in shared memory
+    uint32_t tail_off;
+    uint64_t timeout_ns;
+};
 
 __global__ void __launch_bounds__(DTHREADS, 1)
 llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
@@ -159,28 +301,10 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     DTail *tail = reinterpret_cast<DTail *>(smem + a.tail_off);
     uint8_t *xq = smem + a.xq_off;
-    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = a.stages;
-    const uint32_t rank = cluster_ctarank();
-    const int m = lane & 15;                 // quantization: the row this lane handles
-    const int half = lane >> 4;              //               which chunk of the warp's pair
-    const int qw = warp - 1;                 // quantization warp index (warps 1..15)
-    const int nchunks = a.K / 8;
-    const int npairs = nchunks / 2;          // K is a multiple of 16
-    const int pp = (npairs + CL - 1) / CL;
-    const int p0 = (int)rank * pp, p1 = min(npairs, p0 + pp);   // this CTA's pairs
-    const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
 
-    // this CTA's columns of X, first of all memory traffic
-    uint4 keep[QKEEP];
-#pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        const int p = p0 + qw + i * QWARPS;
-        keep[i] = (warp > 0 && p < p1 && m < a.M)
-                      ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
-                      : make_uint4(0, 0, 0, 0);
-    }
-    if (t == 0) {
+    if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(smem_addr(&tail->full[s]), 1);
             mbar_init(smem_addr(&tail->empty[s]), 1);
@@ -190,185 +314,49 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             mbar_init(smem_addr(&tail->acc_empty[s]), 4);
         }
         mbar_init(smem_addr(&tail->mma_done), 1);
-        mbar_init(smem_addr(&tail->xin), 1);
+        mbar_init(smem_addr(&tail->xbar), 1);
         tail->abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmCB);
     }
-    if (t < DM) tail->pmax[t] = 0u;
     if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), 32);
-    // zero the operand (rows >= M and columns >= K must read as 0)
-    for (int i = t; i < a.kblocks * DBK * DM / 16; i += DTHREADS)
-        reinterpret_cast<uint4 *>(xq)[i] = make_uint4(0, 0, 0, 0);
+    // the next call's first kernel may launch now (it waits for this grid before it reads)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     tc_fence_before();
-    // every CTA's barriers and zeroed buffers exist before a peer writes into them
-    cluster_barrier_all();
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tail->tmem_base;
     const BoundedWait wait{&tail->abort_flag, a.status, a.timeout_ns};
 
-    int stage = 0;
-    uint32_t phase = 0, used = 0, last_parity = 0;
-    int ptile = blockIdx.x, pit = 0;         // next (tile, k-block) to load
-    auto produce = [&](int limit) -> bool {  // issue up to `limit` stage loads
-        for (int n = 0; n < limit && ptile < a.tiles; ++n) {
-            if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) return false;
-            const uint32_t full = smem_addr(&tail->full[stage]);
-            mbar_arrive_expect_tx(full, DSTAGE);
-            tma_load_2d(smem_addr(smem + stage * DSTAGE), &tmCB,
-                        rotated_kblock(pit, ptile, a.kblocks) * DBK, ptile * DBM, full);
-            used |= 1u << stage;
-            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-            if (++stage == S) {
-                stage = 0;
-                phase ^= 1;
-            }
-            if (++pit == a.kblocks) {
-                pit = 0;
-                ptile += gridDim.x;
-            }
-        }
-        return true;
-    };
-
-    uint32_t fl[QKEEP];
-    if (warp == 0) {
-        // the ring fill needs no free slot (they all start empty) and nothing from X; it
-        // waits for this CTA's X loads so as not to queue in front of them
-        if (lane == 0) {
-            drain_wait(smem_addr(&tail->xin), 0, a.status);
-            produce(S);
-        }
-        __syncwarp();
-    } else {
-        // ------------------------------- quantize X, this CTA's quarter of the columns ----
-        float rm = 0.0f;
-#pragma unroll
-        for (int i = 0; i < QKEEP; ++i) {
-            fl[i] = 0;
-            const int p = p0 + qw + i * QWARPS;
-            if (p < p1) {                    // uniform over the warp
-                float f[8];
-                unpack8(keep[i], f);
-                uint32_t b = outlier_bits(f, a.threshold);
-#pragma unroll
-                for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
-                fl[i] = b;
-                if (m == 0) {
-                    const uint32_t dst = smem_addr(&tail->flags[2 * p + half]);
-                    for (int r = 0; r < CL; ++r) st_cluster_u8(map_to_rank(dst, (uint32_t)r), b);
-                }
-                rm = masked_max(f, b, rm);
-            }
-        }
-        rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 16));
-        if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&tail->pmax[m], __float_as_uint(rm));
-        named_barrier(1, QTHREADS);
-        if (t == 32) mbar_arrive(smem_addr(&tail->xin));   // X is in: the ring may fill
-        if (t >= 32 && t < 32 + DM) {
-            const int q = t - 32;
-            const uint32_t dst = smem_addr(&tail->part[rank][q]);
-            for (int r = 0; r < CL; ++r)
-                st_cluster_u32(map_to_rank(dst, (uint32_t)r), tail->pmax[q]);
-        }
-    }
-    // ---------------------------------- exchange 1: outlier bits and row maxima ----
-    __syncwarp();
-    cluster_barrier_all();
-
-    if (warp > 0) {
-        const int q = t - 32;                // 0 .. QTHREADS-1
-        if (q < DM) {
-            float amax = 0.0f;
-            for (int r = 0; r < CL; ++r) amax = fmaxf(amax, tail->part[r][q]);
-            tail->sca[q] = amax;
-            tail->mult[q] = (q < a.M && amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
-        }
-        // ascending outlier list: contiguous chunks per thread, scan over warps 1..15
-        const int per = (nchunks + QTHREADS - 1) / QTHREADS;
-        const int c0 = q * per, c1 = min(nchunks, c0 + per);
-        int cnt = 0;
-        for (int c = c0; c < c1; ++c) cnt += __popc(tail->flags[c]);
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        if (lane == 31) tail->warp_tot[qw] = incl;
-        named_barrier(1, QTHREADS);
-        if (qw == 0) {
-            const int v0 = lane < QWARPS ? tail->warp_tot[lane] : 0;
-            int x = v0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            if (lane < QWARPS) tail->warp_tot[lane] = x - v0;
-            if (lane == 31) {
-                tail->n_out = min(x, a.cap);
-                if (blockIdx.x == 0) {
-                    *a.count = x;
-                    a.status.set(x > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
-                }
-            }
-        }
-        named_barrier(1, QTHREADS);
-        int pos = tail->warp_tot[qw] + incl - cnt;
-        for (int c = c0; c < c1; ++c) {
-            uint32_t b = tail->flags[c];
-            while (b) {
-                const int e = __ffs(b) - 1;
-                b &= b - 1;
-                if (pos < a.cap) tail->idx[pos] = c * 8 + e;
-                ++pos;
-            }
-        }
-        named_barrier(1, QTHREADS);
-
-        // int8 codes of this CTA's columns into every CTA's operand; X at outlier columns
-        const float mul = tail->mult[m];
-        const int n_out = tail->n_out;
-        const uint32_t xq_base = smem_addr(xq);
-        const uint32_t xo_base = smem_addr(tail->xo);
-#pragma unroll
-        for (int i = 0; i < QKEEP; ++i) {
-            const int p = p0 + qw + i * QWARPS;
-            if (p < p1) {
-                const int c = 2 * p + half;
-                float f[8];
-                unpack8(keep[i], f);
-                if (mul > 0.0f) {
-                    const uint2 qv = quant8(f, mul, fl[i]);
-                    const uint32_t dst = xq_base + xq_offset(m, c * 8);
-                    for (int r = 0; r < CL; ++r) st_cluster_v2(map_to_rank(dst, (uint32_t)r), qv);
-                }
-                if (fl[i]) {
-                    // this chunk holds outlier columns: find their list positions
-                    for (int j = 0; j < n_out; ++j) {
-                        const int col = tail->idx[j];
-                        if ((col >> 3) == c) {
-                            const __half hv = __float2half_rn(m < a.M ? f[col & 7] : 0.0f);
-                            const uint32_t dst = xo_base + 2u * (uint32_t)(j * DM + m);
-                            for (int r = 0; r < CL; ++r)
-                                st_cluster_u16(map_to_rank(dst, (uint32_t)r),
-                                               __half_as_ushort(hv));
-                        }
-                    }
-                }
-            }
-        }
-    }
-    // ------------------------------------------- exchange 2: the quantized operand ----
-    __syncwarp();
-    cluster_barrier_all();
-    const int n_out = tail->n_out;
-
     if (warp == 0) {
         // --------------------------------------------------- weight stream (TMA) ----
         if (lane == 0) {
-            produce(1 << 30);
+            int stage = 0;
+            uint32_t phase = 0, used = 0, last_parity = 0;
+            for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
+                const int n0 = tile * DBM;
+                for (int it = 0; it < a.kblocks; ++it) {
+                    const int kb = rotated_kblock(it, tile, a.kblocks);
+                    if (tile == (int)blockIdx.x && it == S) {
+                        // the ring is full: request the rest of this first tile into L2
+                        const int last = min(a.kblocks, S + kPrefetchBlocks);
+                        for (int pf = S; pf < last; ++pf)
+                            tma_prefetch_l2_2d(&tmCB, rotated_kblock(pf, tile, a.kblocks) * DBK,
+                                               n0);
+                    }
+                    if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
+                    const uint32_t full = smem_addr(&tail->full[stage]);
+                    mbar_arrive_expect_tx(full, DSTAGE);
+                    tma_load_2d(smem_addr(smem + stage * DSTAGE), &tmCB, kb * DBK, n0, full);
+                    used |= 1u << stage;
+                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+        drain:
             for (int s = 0; s < S; ++s)
                 if (used & (1u << s))
                     drain_wait(smem_addr(&tail->full[s]), (last_parity >> s) & 1u, a.status);
@@ -376,35 +364,62 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issue ----
         if (lane == 0) {
-            // peers wrote the operand through the generic proxy; the tensor core reads it
-            // through the async proxy
-            fence_proxy_async_smem();
+            // the quantize kernel (already running: this grid is its programmatic dependent)
+            // publishes the image with a release store of the call's epoch
+            bool published = false;
+            {
+                const uint64_t t0 = global_timer_ns();
+                for (uint32_t it = 0;; ++it) {
+                    unsigned long long v;
+                    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];"
+                                 : "=l"(v)
+                                 : "l"(&a.tables->ready)
+                                 : "memory");
+                    if (v == a.epoch) {
+                        published = true;
+                        break;
+                    }
+                    if ((it & 63u) == 0u && (tail->abort_flag ||
+                                             global_timer_ns() - t0 > a.timeout_ns)) {
+                        tail->abort_flag = 1;
+                        a.status.timed_out();
+                        break;
+                    }
+                }
+            }
+            fence_proxy_async_global();
+            const uint32_t xbar = smem_addr(&tail->xbar);
+            const uint32_t img_bytes = (uint32_t)(a.kblocks * DBK * DM);
+            mbar_arrive_expect_tx(xbar, img_bytes + (uint32_t)sizeof(DecodeTables));
+            bulk_load_1d(smem_addr(xq), a.image, img_bytes, xbar);
+            bulk_load_1d(smem_addr(&tail->tab), a.tables, (uint32_t)sizeof(DecodeTables), xbar);
+            const bool have_x = published && wait(xbar, 0);
             const uint32_t idesc = idesc_i8(DBM, DM);
             const uint32_t xq_base = smem_addr(xq);
-            int cs = 0, acc = 0;
-            uint32_t cphase = 0, acc_phase = 0;
-            for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (int tile = blockIdx.x; have_x && tile < a.tiles; tile += gridDim.x) {
                 if (!wait(smem_addr(&tail->acc_empty[acc]), acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * DM);
                 bool good = true;
                 for (int it = 0; it < a.kblocks; ++it) {
                     const int kb = rotated_kblock(it, tile, a.kblocks);
-                    if (!wait(smem_addr(&tail->full[cs]), cphase)) {
+                    if (!wait(smem_addr(&tail->full[stage]), phase)) {
                         good = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_addr(smem + cs * DSTAGE);
+                    const uint32_t sa = smem_addr(smem + stage * DSTAGE);
                     const uint32_t sb = xq_base + (uint32_t)(kb * DM * 128);
 #pragma unroll
                     for (int k = 0; k < DBK / 32; ++k)
                         mma_i8(d, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
                                (it | k) != 0);
-                    tc_commit(smem_addr(&tail->empty[cs]));
-                    if (++cs == S) {
-                        cs = 0;
-                        cphase ^= 1;
+                    tc_commit(smem_addr(&tail->empty[stage]));
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
                     }
                 }
                 if (!good) break;
@@ -412,17 +427,22 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
             }
+            if (!have_x) drain_wait(xbar, 0, a.status);   // the copies land before exit
             tc_commit(smem_addr(&tail->mma_done));
             drain_wait(smem_addr(&tail->mma_done), 0, a.status);
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4) {
         // ------------------------------------------------------------------ epilogue ----
         const int qd = warp & 3;
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
         const float inv = 1.0f / 16129.0f;
+        int okx = 0;
+        if (lane == 0) okx = wait(smem_addr(&tail->xbar), 0) ? 1 : 0;   // the table is in
+        okx = __shfl_sync(0xffffffffu, okx, 0);
+        const int n_out = okx ? tail->tab.n_out : 0;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
+        for (int tile = blockIdx.x; okx && tile < a.tiles; tile += gridDim.x) {
             int okw = 0;
             if (lane == 0) okw = wait(smem_addr(&tail->acc_full[acc]), acc_phase) ? 1 : 0;
             okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -443,30 +463,30 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 const float b = a.bias ? __half2float(a.bias[n]) : 0.0f;
                 float o[DM];
 #pragma unroll
-                for (int r = 0; r < DM; ++r) o[r] = 0.0f;
+                for (int m = 0; m < DM; ++m) o[m] = 0.0f;
                 const int8_t *cbrow = a.CB + (int64_t)n * a.K;
                 for (int j = 0; j < n_out; ++j) {
-                    const int col = tail->idx[j];
+                    const int col = tail->tab.idx[j];
                     const float w = a.W16 ? __half2float(a.W16[(int64_t)n * a.K + col])
                                           : __half2float(__float2half_rn(__fdiv_rn(
                                                 __fmul_rn((float)cbrow[col], sb), 127.0f)));
-                    const uint4 *xv = reinterpret_cast<const uint4 *>(tail->xo + j * DM);
+                    const uint4 *xv = reinterpret_cast<const uint4 *>(tail->tab.xo + j * DM);
                     float f0[8], f1[8];
                     unpack8(xv[0], f0);
                     unpack8(xv[1], f1);
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        o[r] = fmaf(f0[r], w, o[r]);
-                        o[r + 8] = fmaf(f1[r], w, o[r + 8]);
+                    for (int m = 0; m < 8; ++m) {
+                        o[m] = fmaf(f0[m], w, o[m]);
+                        o[m + 8] = fmaf(f1[m], w, o[m + 8]);
                     }
                 }
 #pragma unroll
-                for (int r = 0; r < DM; ++r) {
-                    if (r < a.M) {
-                        const float y = fmaf((float)(int32_t)d[r], tail->sca[r] * inv * sb,
-                                             o[r] + b);
-                        a.Y[(int64_t)r * a.N + n] = __float2half_rn(y);
-                        if (a.C_debug) a.C_debug[(int64_t)r * a.N + n] = (int32_t)d[r];
+                for (int m = 0; m < DM; ++m) {
+                    if (m < a.M) {
+                        const float y = fmaf((float)(int32_t)d[m], tail->tab.sca[m] * inv * sb,
+                                             o[m] + b);
+                        a.Y[(int64_t)m * a.N + n] = __float2half_rn(y);
+                        if (a.C_debug) a.C_debug[(int64_t)m * a.N + n] = (int32_t)d[m];
                     }
                 }
             }
@@ -498,27 +518,73 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     static std::mutex mu;
-    static int max_clusters[64] = {0};
+    static int sms_cache[64] = {0};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int sms;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (sms_cache[dev] == 0) {
+            int n = 0;
+            err = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+            if (err != cudaSuccess) return err;
+            err = cudaFuncSetAttribute(llmint8_decode_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT);
+            if (err != cudaSuccess) return err;
+            sms_cache[dev] = n;
+        }
+        sms = sms_cache[dev];
+    }
 
+    // 1. quantize X once (one CTA)
+    QArgs q;
+    q.X = d.X;
+    q.M = (int)d.M;
+    q.K = (int)d.K;
+    q.cap = (int)d.cap;
+    q.threshold = d.threshold;
+    q.image = d.image;
+    q.tables = d.tables;
+    q.count = d.count;
+    q.status = d.status;
+    q.epoch = d.status.tag >> 4;
+    {
+        cudaLaunchConfig_t qc = {};
+        cudaLaunchAttribute qa[2];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = QCL;
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        qa[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        qa[1].val.programmaticStreamSerializationAllowed = 1;
+        qc.gridDim = dim3(QCL);
+        qc.blockDim = dim3(QTHREADS);
+        qc.dynamicSmemBytes = 0;
+        qc.stream = s;
+        qc.attrs = qa;
+        qc.numAttrs = 2;
+        err = cudaLaunchKernelEx(&qc, llmint8_decode_quantize_kernel, q);
+        note_launches(1);
+        if (err != cudaSuccess) return err;
+    }
+
+    // 2. the weight-streaming product, allowed to start before step 1 finishes
     DArgs a;
-    a.X = d.X;
+    a.epoch = d.status.tag >> 4;
     a.CB = d.CB;
     a.SCB = d.SCB;
     a.W16 = d.W16;
     a.bias = d.bias;
     a.Y = d.Y;
     a.C_debug = d.C_debug;
-    a.count = d.count;
+    a.image = d.image;
+    a.tables = d.tables;
     a.status = d.status;
     a.M = (int)d.M;
     a.N = (int)d.N;
     a.K = (int)d.K;
-    a.cap = (int)d.cap;
-    a.threshold = d.threshold;
     a.kblocks = (int)ceil_div(d.K, DBK);
     a.tiles = (int)ceil_div(d.N, DBM);
     a.timeout_ns = d.timeout_ns;
@@ -533,38 +599,6 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     const int smem = (int)(a.tail_off + sizeof(DTail) + 1024);
     if (smem > SMEM_LIMIT) return cudaErrorInvalidValue;
 
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(DTHREADS);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters;
-    {
-        std::lock_guard<std::mutex> lk(mu);
-        if (max_clusters[dev] == 0) {
-            err = cudaFuncSetAttribute(llmint8_decode_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT);
-            if (err != cudaSuccess) return err;
-            cudaLaunchConfig_t qc = cfg;
-            qc.gridDim = dim3(CL);
-            qc.dynamicSmemBytes = (size_t)SMEM_LIMIT;
-            int n = 0;
-            err = cudaOccupancyMaxActiveClusters(&n, llmint8_decode_kernel, &qc);
-            if (err != cudaSuccess) return err;
-            if (n < 1) return cudaErrorInvalidConfiguration;
-            max_clusters[dev] = n;
-        }
-        clusters = max_clusters[dev];
-    }
-    clusters = std::min<int>(clusters, (int)ceil_div(a.tiles, CL));
-    cfg.gridDim = dim3((unsigned)(clusters * CL));
-
     auto enc = encoder();
     if (!enc) return cudaErrorInvalidValue;
     CUtensorMap tm;
@@ -576,6 +610,18 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    // QCL SMs stay with the quantize kernel while this grid starts
+    cfg.gridDim = dim3((unsigned)std::min(a.tiles, std::max(1, sms - QCL)));
+    cfg.blockDim = dim3(DTHREADS);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     err = cudaLaunchKernelEx(&cfg, llmint8_decode_kernel, tm, a);
     note_launches(1);
     return err != cudaSuccess ? err : cudaGetLastError();

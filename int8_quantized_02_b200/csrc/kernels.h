@@ -63,11 +63,30 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s);
 
 namespace llmint8 {
 
-// Decode path (M <= kDecodeMaxM, K <= kDecodeMaxK): one weight-streaming tcgen05 kernel in
-// clusters of CTAs that quantize X together through distributed shared memory.
+// Decode path (M <= kDecodeMaxM, K <= kDecodeMaxK): a one-CTA kernel quantizes X into a
+// ready-to-copy image of the tensor-core operand plus small tables in the workspace; the
+// weight-streaming tcgen05 kernel, launched as its programmatic dependent, starts streaming
+// CB at once and waits for that image only before its first MMA.
 constexpr int kDecodeMaxM = 16;
 constexpr int kDecodeMaxK = 8192;
 constexpr int kDecodeMaxOutliers = 256;
+
+// Written by the decode quantize kernel, copied whole into every decode CTA.
+struct DecodeTables {
+    unsigned long long ready;                 // call epoch, stored last (release)
+    int32_t n_out;                            // outlier columns used (<= capacity)
+    int32_t pad;
+    float sca[kDecodeMaxM];                   // row absmax over the regular columns
+    int32_t idx[kDecodeMaxOutliers];          // outlier columns, ascending
+    __half xo[kDecodeMaxOutliers * kDecodeMaxM];   // X at the outlier columns, [j][m]
+};
+static_assert(sizeof(DecodeTables) % 16 == 0, "copied with a bulk copy");
+
+// Bytes of the quantized-X operand image: 16 rows x K rounded up to 128, in 128-column
+// blocks of two 1024-byte swizzled 8-row atoms.
+__host__ __device__ constexpr int64_t decode_image_bytes(int64_t K) {
+    return kDecodeMaxM * ((K + 127) / 128 * 128);
+}
 
 struct DecodeLaunch {
     const __half *X;         // [M, K]
@@ -78,6 +97,8 @@ struct DecodeLaunch {
     __half *Y;               // [M, N]
     int32_t *C_debug;        // [M, N] or null
     int32_t *count;          // device outlier count (workspace header)
+    uint8_t *image;          // workspace: decode_image_bytes(K), 1024-byte aligned
+    DecodeTables *tables;    // workspace
     StatusRef status;
     int64_t M, N, K, cap;
     float threshold;
