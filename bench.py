@@ -55,50 +55,73 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """SM clock and throttle reasons sampled (NVML, read-only) while the timed region runs."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
     def __init__(self, device_index: int):
-        self.idx = device_index
         self.samples = []
+        self.max_mhz = None
         self._stop = threading.Event()
         self._thread = None
+        self._nvml = None
+        self._handle = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            handle = None
+            uuid = getattr(props, "uuid", None)
+            if uuid is not None:
+                try:
+                    handle = pynvml.nvmlDeviceGetHandleByUUID(f"GPU-{uuid}")
+                except Exception:  # noqa: BLE001
+                    handle = None
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nvml, self._handle = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self._nvml = None
 
     def _run(self):
+        nv, h = self._nvml, self._handle
         while not self._stop.is_set():
             try:
-                out = subprocess.run(
-                    ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                     "--format=csv,noheader,nounits"], capture_output=True, text=True,
-                    timeout=5).stdout.strip()
-                parts = [p.strip() for p in out.split(",")]
-                if len(parts) == 6:
-                    self.samples.append(parts)
-            except Exception:  # noqa: BLE001 - sampling is best effort
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, reasons))
+            except Exception:  # noqa: BLE001
                 pass
-            self._stop.wait(0.1)
+            time.sleep(0.0005)
 
     def __enter__(self):
-        self._thread = threading.Thread(target=self._run, daemon=True)
-        self._thread.start()
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
         return self
 
     def __exit__(self, *exc):
         self._stop.set()
-        self._thread.join(timeout=10)
+        if self._thread is not None:
+            self._thread.join(timeout=10)
 
     def summary(self):
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        reasons = sorted({names[i] for s in self.samples for i in range(4)
-                          if s[2 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.samples)}
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable"}
+        active = set()
+        for _, r in self.samples:
+            for name, const in self.REASONS:
+                if r & getattr(self._nvml, const, 0):
+                    active.add(name)
+        sm = [s for s, _ in self.samples]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(active), "samples": len(sm)}
 
 
 def kernel_source_hash() -> str:
@@ -239,11 +262,16 @@ def run_ours(args, rank, world, local_rank):
         if st != L.OK:
             raise SystemExit(f"{c.name}: device status {L.status_string(st)}")
 
-    # ---- timed region: whole steps, inputs resident, CUDA events on the launching stream
+    # ---- timed region: whole steps, inputs resident, CUDA events on the launching stream.
+    # Prefill calls run for milliseconds, so a pair of profile events around each GEMM launch
+    # costs nothing measurable and gives the dominant kernel's own duration.  A decode call
+    # lasts about 20 us and an event pair adds about 5 us, so decode records no per-call
+    # events: its weight-streaming kernel spans the whole call (the quantize kernel runs under
+    # it as a programmatic dependent), and the call's duration is region time / calls.
     stream = torch.cuda.current_stream()
-    # per-call profile events around the product kernel
+    per_call_events = bound != "hbm"
     kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in calls] for _ in range(args.steps)]
+            for _ in calls] for _ in range(args.steps if per_call_events else 0)]
     # torch creates an event's CUDA handle on its first record(): record each once here so
     # the library can re-record the same handles around the product kernel
     for row in kev:
@@ -259,10 +287,12 @@ def run_ours(args, rank, world, local_rank):
         e0.record(stream)
         for s in range(args.steps):
             for j, c in enumerate(calls):
-                L.llmint8_set_profile_events(*kev[s][j])
+                if per_call_events:
+                    L.llmint8_set_profile_events(*kev[s][j])
                 c.run()
         e1.record(stream)
-        L.llmint8_set_profile_events(None, None)
+        if per_call_events:
+            L.llmint8_set_profile_events(None, None)
         torch.cuda.synchronize()
     barrier()
     launches = L.llmint8_kernel_launch_count() - launches0
@@ -271,9 +301,13 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     elapsed = float(t.item())
-    kern_s = sum(kev[s][j][0].elapsed_time(kev[s][j][1]) for s in range(args.steps)
-                 for j in range(len(calls))) / 1e3
-    kern_bytes = sum(c.kernel_bytes for c in calls) * args.steps
+    if per_call_events:
+        call_s = [sum(kev[s][j][0].elapsed_time(kev[s][j][1]) for s in range(args.steps))
+                  / 1e3 / args.steps for j in range(len(calls))]
+    else:
+        # no per-call split inside the region: each call gets its share of the step by units
+        call_s = [elapsed / args.steps * c.units / step_units for c in calls]
+    kern_s = sum(call_s) * args.steps
     for c in calls:
         st = L.llmint8_device_status(c.ws)
         if st != L.OK:
@@ -307,17 +341,20 @@ def run_ours(args, rank, world, local_rank):
     e2e_s = float(e2e_t.item())
 
     peaks = measured_peaks()
+    traffic = profiled_traffic(args.workload)
     if bound == "hbm":
-        achieved = kern_bytes / kern_s / 1e9
+        # algorithmic bytes of a call: N*K + 4N + 2MK + 2MN (weights, scales, X in, Y out)
+        achieved = step_units * args.steps / kern_s / 1e9
         peak = peaks["hbm_gbs"]
         roof_unit = "GB/s"
-        traffic = profiled_traffic(args.workload)
+        kernel_name = "llmint8_decode_kernel (+ llmint8_decode_quantize_kernel under it)"
+        timing = "device time of the timed region / calls (no per-call events)"
     else:
-        kern_ops = sum(c.units for c in calls) * args.steps
-        achieved = kern_ops / kern_s / 1e12
+        achieved = step_units * args.steps / kern_s / 1e12
         peak = 2.0 * peaks["bf16_tflops"]           # int8 dense = 2 x bf16 dense (nominal ratio)
         roof_unit = "TOPS"
-        traffic = profiled_traffic(args.workload)
+        kernel_name = "llmint8_gemm_kernel"
+        timing = "CUDA events around each GEMM launch, averaged over the timed region"
     result = {
         "metric": "LLM.int8 linear TOPS (prefill) / weight GB/s (decode); fraction of roofline",
         "value": unit_value(step_units * args.steps * world, elapsed, unit),
@@ -336,7 +373,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": achieved / peak,
                      "peak_source": f"{peaks['source']} "
                                     + ("hbm_gbs" if bound == "hbm" else "2 x bf16_tflops (burst)"),
-                     "kernel": "llmint8_gemm_kernel",
+                     "kernel": kernel_name, "timing": timing,
                      "traffic": traffic},
         "e2e": {"value": unit_value(step_units * e2e_steps * world, e2e_s, unit), "unit": unit,
                 "h2d_bytes_per_step": sum(c.h2d_bytes for c in calls),
@@ -345,13 +382,11 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "per_call": {c.name: None for c in calls},
     }
-    # per-call achieved figure of the product kernel
+    # per-call figure of the product kernel
     for j, c in enumerate(calls):
-        ks = sum(kev[s][j][0].elapsed_time(kev[s][j][1]) for s in range(args.steps)) / 1e3
-        v = (c.kernel_bytes / (ks / args.steps) / 1e9) if bound == "hbm" else \
-            (c.units / (ks / args.steps) / 1e12)
-        result["per_call"][c.name] = {"kernel_us": ks / args.steps * 1e6,
-                                      ("GB/s" if bound == "hbm" else "TOPS"): v}
+        v = c.units / call_s[j] / (1e9 if bound == "hbm" else 1e12)
+        result["per_call"][c.name] = {("call_us" if bound == "hbm" else "kernel_us"):
+                                      call_s[j] * 1e6, unit: v}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args.workload)
     return result
@@ -373,57 +408,70 @@ def workload_config(name, calls):
 # ------------------------------------------------------------------- oracle (CPU) ----
 
 def _oracle_sample(name):
-    """A bounded sample of the workload for the CPU oracle and its metric units."""
-    if name == "decode":
-        N, K, b = 16384, 4096, 16
-        rows = 2048                                   # 1/8 of the output channels
-        W = synth.weight(rows, K, 0.02, seed=0)
-        X = synth.decode(b).make_x()[0]
-        units = rows * K + 4 * rows + 2 * b * K + 2 * b * rows
-        desc = f"decode b={b}: X [16, 4096] against {rows} of the {N} output channels"
-        return X, W, 6.0, units, desc
-    wl = {"ffn6.7b": synth.FFN_W1, "proj175b": synth.PROJ_175B, "sweep": synth.sweep(6)}[name]
-    rows_x, rows_w = 256, 512
-    X = wl.make_x()[0][:rows_x].copy()
-    W = synth.weight(rows_w, wl.K, wl.w_std, seed=0)
-    units = 2 * rows_x * rows_w * wl.K
-    desc = f"{wl.name}: first {rows_x} rows of X against {rows_w} output channels"
-    return X, W, wl.threshold, units, desc
-
-
-def cpu_baseline(name, reps=None):
+    """A bounded sample of every call of the workload for the CPU oracle, and its metric units:
+    the same X rows and shapes, against a slice of the output channels (and, for prefill,
+    of the token rows)."""
     from oracle import oracle
-    X, W, t, units, desc = _oracle_sample(name)
-    CB, SCB = oracle.quantize_weight_colwise(W)
-    oracle.linear(X[:1], CB[:16], SCB[:16], threshold=t)   # load + warm
-    times = []
-    deadline = time.perf_counter() + 15.0
-    while True:
-        t0 = time.perf_counter()
+    pieces, units = [], 0
+    if name == "decode":
+        N, K = 16384, 4096
+        rows = 2048                                   # 1/8 of the output channels
+        CB, SCB = oracle.quantize_weight_colwise(synth.weight(rows, K, 0.02, seed=0))
+        for b in DECODE_BATCHES:
+            pieces.append((synth.decode(b).make_x()[0], CB, SCB, 6.0))
+            units += rows * K + 4 * rows + 2 * b * K + 2 * b * rows
+        desc = (f"decode b=1,8,16: X [b, {K}] against {rows} of the {N} output channels")
+        return pieces, units, desc
+    specs = {"ffn6.7b": [(synth.FFN_W1, 6.0), (synth.FFN_W2, 6.0)],
+             "proj175b": [(synth.PROJ_175B, 6.0)],
+             "sweep": [(synth.sweep(k), 6.0) for k in (0, 6, 64, 512)]
+             + [(synth.sweep(6, float("inf")), float("inf")), (synth.sweep(0, 0.0), 0.0)]}[name]
+    rows_x, rows_w = 128, 256
+    for wl, t in specs:
+        X = wl.make_x()[0][:rows_x].copy()
+        CB, SCB = oracle.quantize_weight_colwise(synth.weight(rows_w, wl.K, wl.w_std, seed=0))
+        pieces.append((X, CB, SCB, t))
+        units += 2 * rows_x * rows_w * wl.K
+    desc = (f"{name}: every call on the first {rows_x} rows of X against {rows_w} "
+            f"output channels")
+    return pieces, units, desc
+
+
+def _oracle_step(pieces):
+    from oracle import oracle
+    for X, CB, SCB, t in pieces:
         oracle.linear(X, CB, SCB, threshold=t)
+
+
+def _cores():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count()))
+
+
+def cpu_baseline(name, budget_s=15.0):
+    pieces, units, desc = _oracle_sample(name)
+    _oracle_step(pieces[:1])                                  # load + warm
+    times = []
+    deadline = time.perf_counter() + budget_s
+    while not times or time.perf_counter() < deadline:
+        t0 = time.perf_counter()
+        _oracle_step(pieces)
         times.append(time.perf_counter() - t0)
-        if (reps is not None and len(times) >= reps) or (reps is None and
-                                                           time.perf_counter() > deadline):
-            break
     unit = "GB/s" if name == "decode" else "TOPS"
     sec = statistics.median(times)
-    return {"value": unit_value(units, sec, unit), "unit": unit,
-            "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count())), "kind": "oracle",
-            "sample": f"{desc}; median of {len(times)} runs of {sec:.3f} s"}
+    return {"value": unit_value(units, sec, unit), "unit": unit, "cores": _cores(),
+            "kind": "oracle", "sample": f"{desc}; median of {len(times)} runs of {sec:.3f} s"}
 
 
 def run_reference(args, rank, world):
-    """The oracle timed on the host cores on a bounded sample of the same workload."""
+    """The oracle timed on the host cores, each step a bounded sample of the same workload."""
     if rank != 0:
         return None
-    from oracle import oracle
-    X, W, t, units, desc = _oracle_sample(args.workload)
-    CB, SCB = oracle.quantize_weight_colwise(W)
+    pieces, units, desc = _oracle_sample(args.workload)
     for _ in range(min(args.warmup, 1)):
-        oracle.linear(X, CB, SCB, threshold=t)
+        _oracle_step(pieces)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.linear(X, CB, SCB, threshold=t)
+        _oracle_step(pieces)
     sec = time.perf_counter() - t0
     unit = "GB/s" if args.workload == "decode" else "TOPS"
     value = unit_value(units * args.steps, sec, unit)
@@ -432,12 +480,11 @@ def run_reference(args, rank, world):
         "metric": "LLM.int8 linear TOPS (prefill) / weight GB/s (decode); fraction of roofline",
         "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "i8/i32 (fp16 in/out)",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle; int8 codes exact)",
         "data": "synthetic (seeded, int8_quantized_02_b200.synth)",
         "config": {"workload": args.workload, "sample": desc, "parallelism": "replicas"},
-        "cpu_baseline": {"value": value, "unit": unit,
-                         "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count())),
-                         "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": _cores(), "kind": "oracle",
+                         "sample": desc},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
