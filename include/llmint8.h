@@ -158,6 +158,40 @@ LLMINT8_API llmint8_status llmint8_set_wait_timeout_ns(uint64_t ns);
 LLMINT8_API llmint8_status llmint8_set_profile_events(void *start, void *stop);
 LLMINT8_API uint64_t llmint8_kernel_launch_count(void);
 
+/*
+ * llmint8_linear without a workspace argument.  The paper has no counterpart: this is a
+ * calling convenience.  It is for callers that cannot allocate device memory where they
+ * call the layer: a token-by-token decode loop that must not call cudaMalloc/cudaFree
+ * between steps (cudaFree waits for the whole device), or a plain C host without a device
+ * allocator of its own.  The call allocates nothing.  Its scratch is a fixed 160 KiB
+ * device array inside this library, one per device.
+ *   Arguments X, M, K, CB, SCB, N, bias, W_fp16, threshold, max_outliers, Y, stream: as
+ *     for llmint8_linear (same layouts, same output).  There is no C_debug output.
+ *   Covered shapes are those of the decode path: M <= 16, K <= 8192 (K, N multiples of
+ *     16), threshold > 0 and max_outliers <= 256.  Anything larger returns
+ *     LLMINT8_ERR_UNSUPPORTED_SHAPE before any CUDA call; use llmint8_linear there.
+ *   scratch_out  NULL, or receives the device address of the calling device's scratch.
+ *     The scratch begins with the same 256-byte header as an llmint8_linear workspace.
+ *     So llmint8_device_status(*scratch_out, stream) and
+ *     llmint8_workspace_outlier_count(*scratch_out, ...) report the device status and the
+ *     outlier count of the last call on that device.
+ *   Set-up: the first call on each device looks up the scratch's address
+ *     (cudaGetSymbolAddress, with the device current), which may load this library's
+ *     device code.  Make that first call before any stream capture.
+ *   The scratch starts zero-filled when the module loads.  Nothing in it needs clearing
+ *     between calls.
+ *   Calls on one stream, in order, are safe.  Calls that overlap on one device share its
+ *     scratch and race, with undefined outputs.  Overlap means two streams, or host
+ *     threads without stream order between them.
+ * Returns LLMINT8_ERR_INVALID_ARG for NULL or misaligned pointers (16 bytes) or a NaN
+ * threshold, and LLMINT8_ERR_CUDA if the set-up or a launch fails.
+ */
+LLMINT8_API llmint8_status llmint8_linear_noalloc(const uint16_t *X, int64_t M, int64_t K,
+                                      const int8_t *CB, const float *SCB, int64_t N,
+                                      const uint16_t *bias, const uint16_t *W_fp16,
+                                      float threshold, int64_t max_outliers, uint16_t *Y,
+                                      void *stream, void **scratch_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -306,6 +307,111 @@ llmint8_status llmint8_workspace_outlier_count(const void *ws, void *stream, int
     if (cudaMemcpy(count, &h->n_outliers, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     return LLMINT8_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ no-allocation call ----
+//
+// llmint8_linear_noalloc runs the decode path (the X-quantize kernel and the weight-streaming
+// kernel) on scratch that lives in this file-scope device array instead of a caller
+// workspace.  It is meant for callers that cannot allocate device memory at the call site: a
+// token-by-token decode loop that must not call cudaMalloc or cudaFree between steps (cudaFree
+// waits for the whole device), and plain C hosts that hold no device allocator of their own.
+// Nothing here allocates: no cudaMalloc, cudaFree or allocating library routine.
+//
+// Layout of the scratch (one copy per device; the module zero-fills it when it loads):
+//   [0, 256)                         WsHeader: status words and outlier count of the last call
+//   [first 1024-aligned address ...) quantized-X operand image, decode_image_bytes(K) bytes
+//   [next 256-aligned address ...)   DecodeTables
+// Nothing in it must be zeroed between calls: every call tags the words it hands from one
+// kernel to the other, and its status words, with a fresh call epoch (the counter only grows
+// and starts above zero).  Calls in stream order are safe: the X-quantize kernel of a call
+// waits for the previous grid on its stream to finish before it writes the scratch.  Calls
+// that overlap - on two streams, or from two host threads without stream order between them -
+// share the one scratch of their device and race; their outputs are undefined.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 160 * 1024;
+
+constexpr size_t noalloc_image_offset_bound() { return 1024; }   // header + worst alignment pad
+constexpr size_t noalloc_need_bound() {
+    return noalloc_image_offset_bound() + (size_t)decode_image_bytes(kDecodeMaxK) + 256 +
+           sizeof(DecodeTables);
+}
+static_assert(noalloc_need_bound() <= kNoAllocScratchBytes,
+              "the no-allocation scratch holds the decode path's largest shape");
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Set-up, once per device, with that device current: the scratch's device address.
+cudaError_t noalloc_scratch(void **ptr) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+llmint8_status llmint8_linear_noalloc(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
+                                      const float *SCB, int64_t N, const uint16_t *bias,
+                                      const uint16_t *W_fp16, float threshold,
+                                      int64_t max_outliers, uint16_t *Y, void *stream,
+                                      void **scratch_out) {
+    if (!X || !CB || !SCB || !Y) return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(CB) || !aligned16(SCB) || !aligned16(Y) ||
+        (bias && !aligned16(bias)) || (W_fp16 && !aligned16(W_fp16)))
+        return LLMINT8_ERR_INVALID_ARG;
+    if (isnan(threshold)) return LLMINT8_ERR_INVALID_ARG;
+    if (!shape_ok_mk(M, K) || !shape_ok_n(N)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    if (max_outliers < 0 || max_outliers > K) return LLMINT8_ERR_INVALID_ARG;
+    // only what the decode path covers fits the fixed scratch
+    if (!use_decode_path(M, K, threshold, max_outliers)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+
+    void *base = nullptr;
+    if (noalloc_scratch(&base) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    const uintptr_t b = reinterpret_cast<uintptr_t>(base);
+    const size_t image = (size_t)(align_up((int64_t)(b + sizeof(WsHeader)), 1024) - (int64_t)b);
+    const size_t tables = (size_t)align_up((int64_t)(image + decode_image_bytes(K)), 256);
+    if (tables + sizeof(DecodeTables) > kNoAllocScratchBytes) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+
+    WsHeader *h = at<WsHeader>(base, 0);
+    DecodeLaunch d;
+    d.X = reinterpret_cast<const __half *>(X);
+    d.CB = CB;
+    d.SCB = SCB;
+    d.W16 = reinterpret_cast<const __half *>(W_fp16);
+    d.bias = reinterpret_cast<const __half *>(bias);
+    d.Y = reinterpret_cast<__half *>(Y);
+    d.C_debug = nullptr;
+    d.count = &h->n_outliers;
+    d.image = at<uint8_t>(base, image);
+    d.tables = at<DecodeTables>(base, tables);
+    d.status = next_status(h);
+    d.M = M;
+    d.N = N;
+    d.K = K;
+    d.cap = max_outliers;
+    d.threshold = threshold;
+    d.timeout_ns = g_timeout_ns.load();
+    if (scratch_out) *scratch_out = base;
+    return from_cuda(launch_decode(d, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

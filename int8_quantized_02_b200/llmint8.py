@@ -43,6 +43,8 @@ PROTOTYPES = {
     "llmint8_set_wait_timeout_ns": (ctypes.c_int, [_U64]),
     "llmint8_set_profile_events": (ctypes.c_int, [_P, _P]),
     "llmint8_kernel_launch_count": (_U64, []),
+    "llmint8_linear_noalloc": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _F32, _I64,
+                                              _P, _P, ctypes.POINTER(ctypes.c_void_p)]),
 }
 
 
@@ -232,3 +234,29 @@ def llmint8_set_profile_events(start=None, stop=None) -> None:
 
 def llmint8_kernel_launch_count() -> int:
     return int(load().llmint8_kernel_launch_count())
+
+
+def llmint8_linear_noalloc(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor, Y: torch.Tensor,
+                           bias=None, W_fp16=None, threshold: float = 6.0,
+                           max_outliers: int = 64, stream=None) -> int:
+    """llmint8_linear on the library's fixed per-device scratch: no workspace, nothing
+    allocated (the caller passes Y).  Decode shapes only (M <= 16, K <= 8192, threshold > 0,
+    max_outliers <= 256).  Returns the device address of the scratch, whose header
+    llmint8_device_status / llmint8_workspace_outlier_count read through the C ABI."""
+    M, K = X.shape
+    N = CB.shape[0]
+    _want(X, torch.float16, (M, K), "X")
+    _want(CB, torch.int8, (N, K), "CB")
+    _want(SCB, torch.float32, (N,), "SCB")
+    _want(Y, torch.float16, (M, N), "Y")
+    if bias is not None:
+        _want(bias, torch.float16, (N,), "bias")
+    if W_fp16 is not None:
+        _want(W_fp16, torch.float16, (N, K), "W_fp16")
+    scratch = ctypes.c_void_p(0)
+    _check(load().llmint8_linear_noalloc(_ptr(X), M, K, _ptr(CB), _ptr(SCB), N, _ptr(bias),
+                                         _ptr(W_fp16), ctypes.c_float(threshold),
+                                         int(max_outliers), _ptr(Y), _stream(stream),
+                                         ctypes.byref(scratch)),
+           "llmint8_linear_noalloc")
+    return int(scratch.value or 0)
