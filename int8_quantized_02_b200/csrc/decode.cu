@@ -10,8 +10,8 @@
 //   registers, across warps, and across the cluster through distributed shared memory
 //   (one hardware cluster barrier); the int8 codes go into the workspace as a byte-exact
 //   image of the tensor-core operand (16 rows, 128-byte swizzled K-major blocks, outlier
-//   columns and padding 0), next to a table of SCA, the ascending outlier columns and X at
-//   those columns.  It lets its dependent launch at once.
+//   columns and padding 0), next to a table of SCA and the ascending outlier columns.  It
+//   lets its dependent launch as soon as the work before it in the stream is complete.
 //
 // llmint8_decode_kernel (one CTA per 128-row weight tile, programmatic dependent launch):
 //   warp 0        TMA producer: streams 128-row x 128-byte tiles of CB (16 KB) through a ring
@@ -25,9 +25,11 @@
 //                 with the weight tile as the 128-row operand and the quantized X as the
 //                 16-column operand: D[n, m] = sum_k CB[n, k] Xq[m, k] into a 128 x 16 int32
 //                 TMEM accumulator (double-buffered over tiles);
-//   warps 4..7    epilogue: D -> registers; y = D * SCA_m * SCB_n / 127^2
-//                 + sum_{j in O} X[m, O_j] * W_o[n, O_j] + bias_n (the fp16 outlier part of
-//                 the decomposition, weights from the bytes of the outlier columns) -> fp16.
+//   warps 4..7    epilogue: while the weights stream, each thread (one output row n) builds
+//                 sum_{j in O} X[m, O_j] * W_o[n, O_j] + bias_n (the fp16 outlier part of the
+//                 decomposition, weights from the bytes of the outlier columns) and its scale;
+//                 after the tile's last MMA: D -> registers, y = D * SCA_m * SCB_n / 127^2 +
+//                 that part -> fp16.
 // Same method and rounding as the GEMM path (LLM.int8() summary, sections الابتكار الثاني
 // and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded.
 #include <cudaTypedefs.h>
@@ -127,7 +129,6 @@ __global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(co
     __shared__ uint32_t pmax[DM];            // this CTA's (float bits, >= 0: int order)
     __shared__ float mult[DM];
     __shared__ uint8_t flags_all[kDecodeMaxK / 8];   // CTA 0: outlier bits of every chunk
-    __shared__ int n_out_s;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int m = lane & 15;                 // the row this thread handles
     const int half = lane >> 4;              // which chunk of the warp's pair
@@ -238,18 +239,10 @@ __global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(co
         }
         const int total = __shfl_sync(0xffffffffu, incl, 31);
         if (lane == 0) {
-            n_out_s = min(total, a.cap);
-            a.tables->n_out = n_out_s;
+            a.tables->n_out = min(total, a.cap);
             *a.count = total;
             a.status.set(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
         }
-    }
-    __syncthreads();
-    const int n_out = n_out_s;
-    for (int i = t; i < n_out * DM; i += QTHREADS) {
-        const int j = i / DM, mm = i % DM;
-        a.tables->xo[i] = mm < a.M ? a.X[(int64_t)mm * a.K + a.tables->idx[j]]
-                                   : __float2half_rn(0.0f);
     }
     // publish: the image and table are complete (the dependent kernel bulk-copies them)
     __threadfence();
@@ -270,12 +263,14 @@ struct DTail {
     uint32_t tmem_base;
     int abort_flag;
     alignas(16) DecodeTables tab;
+    alignas(16) __half xo[kDecodeMaxOutliers * DM];   // X at the outlier columns, [j][m]
 };
 static_assert(offsetof(DTail, tab) % 16 == 0, "the table is a bulk-copy destination");
 static_assert(offsetof(DTail, xbar) % 8 == 0, "mbarriers are 8-byte aligned");
 
 struct DArgs {
     unsigned long long epoch;
+    const __half *X;
     const int8_t *CB;
     const float *SCB;
     const __half *W16;
@@ -433,16 +428,56 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------------ epilogue ----
+        // Everything of an output row except the int8 product - its scale, bias and fp16
+        // outlier part - is computed while the MMAs still stream the weights; after the last
+        // MMA of a tile only the accumulator read, one FMA per value and the stores remain.
         const int qd = warp & 3;
+        const int et = threadIdx.x - 128;                 // 0..127 over the epilogue warps
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
         const float inv = 1.0f / 16129.0f;
         int okx = 0;
         if (lane == 0) okx = wait(smem_addr(&tail->xbar), 0) ? 1 : 0;   // the table is in
         okx = __shfl_sync(0xffffffffu, okx, 0);
         const int n_out = okx ? tail->tab.n_out : 0;
+        // X at the outlier columns (an input of the call, complete before this grid launched)
+        for (int i = et; i < n_out * DM; i += 128) {
+            const int j = i / DM, mm = i % DM;
+            tail->xo[i] = mm < a.M ? a.X[(int64_t)mm * a.K + tail->tab.idx[j]]
+                                   : __float2half_rn(0.0f);
+        }
+        named_barrier(1, 128);
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; okx && tile < a.tiles; tile += gridDim.x) {
+            const int n = tile * DBM + qd * 32 + lane;
+            const bool live = n < a.N;
+            float o[DM];
+            float scale = 0.0f;
+#pragma unroll
+            for (int m = 0; m < DM; ++m) o[m] = 0.0f;
+            if (live) {
+                const float sb = a.SCB[n];
+                const float b = a.bias ? __half2float(a.bias[n]) : 0.0f;
+                scale = sb * inv;
+                const int8_t *cbrow = a.CB + (int64_t)n * a.K;
+                for (int j = 0; j < n_out; ++j) {
+                    const int col = tail->tab.idx[j];
+                    const float w = a.W16 ? __half2float(a.W16[(int64_t)n * a.K + col])
+                                          : __half2float(__float2half_rn(__fdiv_rn(
+                                                __fmul_rn((float)cbrow[col], sb), 127.0f)));
+                    const uint4 *xv = reinterpret_cast<const uint4 *>(tail->xo + j * DM);
+                    float f0[8], f1[8];
+                    unpack8(xv[0], f0);
+                    unpack8(xv[1], f1);
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {
+                        o[m] = fmaf(f0[m], w, o[m]);
+                        o[m + 8] = fmaf(f1[m], w, o[m + 8]);
+                    }
+                }
+#pragma unroll
+                for (int m = 0; m < DM; ++m) o[m] += b;
+            }
             int okw = 0;
             if (lane == 0) okw = wait(smem_addr(&tail->acc_full[acc]), acc_phase) ? 1 : 0;
             okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -456,35 +491,11 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             if (lane == 0) mbar_arrive(smem_addr(&tail->acc_empty[acc]));
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
-
-            const int n = tile * DBM + qd * 32 + lane;
-            if (n < a.N) {
-                const float sb = a.SCB[n];
-                const float b = a.bias ? __half2float(a.bias[n]) : 0.0f;
-                float o[DM];
-#pragma unroll
-                for (int m = 0; m < DM; ++m) o[m] = 0.0f;
-                const int8_t *cbrow = a.CB + (int64_t)n * a.K;
-                for (int j = 0; j < n_out; ++j) {
-                    const int col = tail->tab.idx[j];
-                    const float w = a.W16 ? __half2float(a.W16[(int64_t)n * a.K + col])
-                                          : __half2float(__float2half_rn(__fdiv_rn(
-                                                __fmul_rn((float)cbrow[col], sb), 127.0f)));
-                    const uint4 *xv = reinterpret_cast<const uint4 *>(tail->tab.xo + j * DM);
-                    float f0[8], f1[8];
-                    unpack8(xv[0], f0);
-                    unpack8(xv[1], f1);
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        o[m] = fmaf(f0[m], w, o[m]);
-                        o[m + 8] = fmaf(f1[m], w, o[m + 8]);
-                    }
-                }
+            if (live) {
 #pragma unroll
                 for (int m = 0; m < DM; ++m) {
                     if (m < a.M) {
-                        const float y = fmaf((float)(int32_t)d[m], tail->tab.sca[m] * inv * sb,
-                                             o[m] + b);
+                        const float y = fmaf((float)(int32_t)d[m], tail->tab.sca[m] * scale, o[m]);
                         a.Y[(int64_t)m * a.N + n] = __float2half_rn(y);
                         if (a.C_debug) a.C_debug[(int64_t)m * a.N + n] = (int32_t)d[m];
                     }
@@ -573,6 +584,7 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     // 2. the weight-streaming product, allowed to start before step 1 finishes
     DArgs a;
     a.epoch = d.status.tag >> 4;
+    a.X = d.X;
     a.CB = d.CB;
     a.SCB = d.SCB;
     a.W16 = d.W16;

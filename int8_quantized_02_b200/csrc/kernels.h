@@ -63,7 +63,7 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s);
 
 namespace llmint8 {
 
-// Decode path (M <= kDecodeMaxM, K <= kDecodeMaxK): a one-CTA kernel quantizes X into a
+// Decode path (M <= kDecodeMaxM, K <= kDecodeMaxK): a cluster of CTAs quantizes X into a
 // ready-to-copy image of the tensor-core operand plus small tables in the workspace; the
 // weight-streaming tcgen05 kernel, launched as its programmatic dependent, starts streaming
 // CB at once and waits for that image only before its first MMA.
@@ -78,7 +78,6 @@ struct DecodeTables {
     int32_t pad;
     float sca[kDecodeMaxM];                   // row absmax over the regular columns
     int32_t idx[kDecodeMaxOutliers];          // outlier columns, ascending
-    __half xo[kDecodeMaxOutliers * kDecodeMaxM];   // X at the outlier columns, [j][m]
 };
 static_assert(sizeof(DecodeTables) % 16 == 0, "copied with a bulk copy");
 

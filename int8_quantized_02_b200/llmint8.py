@@ -193,6 +193,47 @@ def llmint8_linear(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor, bias=No
     return Y
 
 
+class LinearPlan:
+    """One llmint8_linear call with its arguments checked and marshalled once.
+
+    Calling the plan launches the same C entry point with the same tensors, so a loop that
+    runs the layer on fixed buffers (a decode loop) pays the Python-side argument handling
+    only once.  The tensors must stay alive and keep their storage while the plan is used."""
+
+    def __init__(self, X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor, bias=None,
+                 W_fp16=None, threshold: float = 6.0, max_outliers: int | None = None, Y=None,
+                 workspace=None, C_debug=None, stream=None):
+        M, K = X.shape
+        N = CB.shape[0]
+        _want(X, torch.float16, (M, K), "X")
+        _want(CB, torch.int8, (N, K), "CB")
+        _want(SCB, torch.float32, (N,), "SCB")
+        if bias is not None:
+            _want(bias, torch.float16, (N,), "bias")
+        if W_fp16 is not None:
+            _want(W_fp16, torch.float16, (N, K), "W_fp16")
+        if C_debug is not None:
+            _want(C_debug, torch.int32, (M, N), "C_debug")
+        cap = default_max_outliers(K, threshold) if max_outliers is None else int(max_outliers)
+        self.Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+        _want(self.Y, torch.float16, (M, N), "Y")
+        if workspace is None:
+            workspace = torch.empty((llmint8_linear_workspace_size(M, N, K, cap),),
+                                    dtype=torch.uint8, device=X.device)
+        self.workspace = workspace
+        self._keep = (X, CB, SCB, bias, W_fp16, C_debug)
+        self._fn = load().llmint8_linear
+        self._args = (_ptr(X), M, K, _ptr(CB), _ptr(SCB), N, _ptr(bias), _ptr(W_fp16),
+                      ctypes.c_float(threshold), cap, _ptr(self.Y), _ptr(workspace),
+                      workspace.numel(), _stream(stream), _ptr(C_debug))
+
+    def __call__(self) -> torch.Tensor:
+        code = self._fn(*self._args)
+        if code != OK:
+            raise LLMInt8Error(code, "llmint8_linear")
+        return self.Y
+
+
 def llmint8_dequant(CB: torch.Tensor, SCB: torch.Tensor, out=None, stream=None):
     """(CB int8 [N, K], SCB fp32 [N]) -> fp16 [N, K] = (CB * SCB) / 127."""
     N, K = CB.shape

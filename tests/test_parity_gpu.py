@@ -292,3 +292,16 @@ def test_decode_bounded_wait_timeout_is_reported():
     assert L.ERR_TIMEOUT in seen
     assert seen <= {L.OK, L.ERR_TIMEOUT}
     _check_linear(X, W, 6.0, cap=64)
+
+
+def test_linear_plan_matches_the_call():
+    X = _x(16, 4096, 6, lo=6.0, hi=60.0, row_frac=1.0, seed=31)
+    W = synth.weight(1024, 4096, 0.02, seed=31)
+    CB, SCB = L.llmint8_quantize_weight_colwise(dev(W))
+    Xd = dev(X)
+    ref = host(L.llmint8_linear(Xd, CB, SCB, threshold=6.0, max_outliers=64))
+    plan = L.LinearPlan(Xd, CB, SCB, threshold=6.0, max_outliers=64)
+    for _ in range(2):
+        got = host(plan())
+        assert np.array_equal(got, ref)
+    assert L.llmint8_device_status(plan.workspace) == L.OK
