@@ -15,9 +15,15 @@
 //               (64 fp16 of K each) - both fill the same 48 KB shared-memory stages;
 //   warp 1      TMEM allocator and MMA issuer (one thread);
 //   warps 2..5  epilogue: TMEM -> registers -> dequantize, add P and bias -> fp16 -> global.
-// TMEM (512 columns): with no outlier columns the int32 accumulator is double-buffered
-// (2 x 256 columns) so the epilogue of a tile overlaps the main loop of the next; with
-// outlier columns the second half holds the fp32 outlier accumulator P instead.
+// TMEM (512 columns): the int32 accumulator is double-buffered (2 x 256 columns) so the
+// epilogue of a tile overlaps the main loop of the next.  The outlier product P takes one of
+// two routes:
+//   few outlier columns (n_out <= kRegOutliers, the usual case: a handful of feature
+//   dimensions) - the epilogue warps form P on the CUDA cores (fp32 FMAs) from their rows of
+//   Xo (registers) and the tile's slice of Wo (shared memory), both loaded while the main
+//   loop of the tile runs;
+//   more - P is a tcgen05 kind::f16 product appended to the k-loop, accumulated in fp32 in
+//   the second half of TMEM, and the int32 accumulator is single-buffered.
 // Every wait is bounded (BoundedWait); a timeout records LLMINT8_ERR_TIMEOUT, drains the
 // copies and MMAs in flight, frees TMEM and returns.
 #include <cudaTypedefs.h>
@@ -40,6 +46,11 @@ constexpr int B_BYTES = BN * BKB;       // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
+constexpr int kRegOutliers = 32;        // outlier columns formed in the epilogue at most
+// the tile's column slice, staged once per tile by the four epilogue warps together:
+// Wo [o][n] fp16, SCB [n] and bias [n] as fp32
+constexpr int SL_W_BYTES = kRegOutliers * BN * 2;
+constexpr int SL_BYTES = SL_W_BYTES + BN * 4 + BN * 4;
 
 struct Tail {
     uint64_t full[STAGES];
@@ -47,12 +58,18 @@ struct Tail {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t mma_done;
+    uint64_t slice_full;                // the four epilogue warps staged the column slice
+    uint64_t slice_empty;               // ... and are done reading it
     uint32_t tmem_base;
     int abort_flag;
 };
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + (int)sizeof(Tail);
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SL_BYTES + 1024 + (int)sizeof(Tail);
+static_assert(SMEM_BYTES <= 232448, "fits the opt-in shared memory of one CTA");
 
 struct Args {
+    const __half *Xo;        // [M, pitch]
+    const __half *Wo;        // [N, pitch]
+    int pitch;
     const int32_t *count;
     int64_t cap;
     const float *SCA;
@@ -79,13 +96,17 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Tail *tail = reinterpret_cast<Tail *>(smem + STAGES * STAGE_BYTES);
+    __half *sl_w = reinterpret_cast<__half *>(smem + STAGES * STAGE_BYTES);
+    float *sl_scb = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + SL_W_BYTES);
+    float *sl_bias = sl_scb + BN;
+    Tail *tail = reinterpret_cast<Tail *>(smem + STAGES * STAGE_BYTES + SL_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // Outlier configuration of this call (uniform over the grid).
     const int n_out = (int)min((int64_t)*a.count, a.cap);
-    const int nob = (n_out + 63) / 64;                 // fp16 k-blocks of 64 columns
     const bool all_outliers = n_out >= a.K;            // then C == 0: skip the int8 blocks
+    const bool reg_out = n_out > 0 && n_out <= kRegOutliers && !all_outliers;
+    const int nob = reg_out ? 0 : (n_out + 63) / 64;   // fp16 k-blocks of 64 columns
     const int nkb = all_outliers ? 0 : a.num_kb;
     const int acc_stages = nob > 0 ? 1 : 2;
     const int total_tiles = a.tiles_m * a.tiles_n;
@@ -100,6 +121,8 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             mbar_init(smem_addr(&tail->acc_empty[s]), 4);
         }
         mbar_init(smem_addr(&tail->mma_done), 1);
+        mbar_init(smem_addr(&tail->slice_full), 4);
+        mbar_init(smem_addr(&tail->slice_empty), 4);
         tail->abort_flag = 0;
         fence_mbar_init();
     }
@@ -210,19 +233,73 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // ----------------------------------------------------------------- epilogue ----
         const int q = warp & 3;                        // TMEM lane quadrant of this warp
         const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+        const int wq = warp - 2;                       // this warp's quarter of the slice
         int acc = 0;
-        uint32_t acc_phase = 0;
+        uint32_t acc_phase = 0, sl_phase = 0;
+        bool first = true;
         for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+            const int m0 = (tile % a.tiles_m) * BM;
+            const int n0 = (tile / a.tiles_m) * BN;
+            // The tile's column slice (SCB, bias and, with few outlier columns, Wo), staged
+            // while the tensor cores still work on the tile: each warp one quarter of it,
+            // after every warp is done with the previous tile's slice.
+            {
+                int okq = 1;
+                if (lane == 0 && !first)
+                    okq = wait(smem_addr(&tail->slice_empty), sl_phase ^ 1) ? 1 : 0;
+                okq = __shfl_sync(0xffffffffu, okq, 0);
+                if (!okq) break;
+                for (int cc = wq * 64 + lane; cc < wq * 64 + 64; cc += 32) {
+                    const int n = n0 + cc;
+                    const bool in = n < a.N;
+                    sl_scb[cc] = in ? __ldg(a.SCB + n) : 0.0f;
+                    sl_bias[cc] = (in && a.bias) ? __half2float(a.bias[n]) : 0.0f;
+                    if (reg_out) {
+#pragma unroll
+                        for (int o8 = 0; o8 < kRegOutliers; o8 += 8) {
+                            if (o8 < n_out) {
+                                uint4 v = make_uint4(0, 0, 0, 0);
+                                if (in)
+                                    v = __ldg(reinterpret_cast<const uint4 *>(
+                                        a.Wo + (int64_t)n * a.pitch + o8));
+                                const __half *h = reinterpret_cast<const __half *>(&v);
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    if (o8 + e < n_out) sl_w[(o8 + e) * BN + cc] = h[e];
+                            }
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&tail->slice_full));
+                int okf = 0;
+                if (lane == 0) okf = wait(smem_addr(&tail->slice_full), sl_phase) ? 1 : 0;
+                okf = __shfl_sync(0xffffffffu, okf, 0);
+                if (!okf) break;
+                first = false;
+            }
+            // this thread's row of Xo (the outlier columns of X)
+            float xo[kRegOutliers];
+            if (reg_out) {
+                const int r = m0 + q * 32 + lane;
+#pragma unroll
+                for (int o8 = 0; o8 < kRegOutliers; o8 += 8) {
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (o8 < n_out && r < a.M)
+                        v = __ldg(reinterpret_cast<const uint4 *>(a.Xo + (int64_t)r * a.pitch + o8));
+                    const __half *h = reinterpret_cast<const __half *>(&v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) xo[o8 + e] = __half2float(h[e]);
+                }
+            }
+            const int row = m0 + q * 32 + lane;
+            const bool row_ok = row < a.M;
+            const float rs = row_ok ? a.SCA[row] * (1.0f / 16129.0f) : 0.0f;
             int ok = 0;
             if (lane == 0) ok = wait(smem_addr(&tail->acc_full[acc]), acc_phase) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
-            const int m0 = (tile % a.tiles_m) * BM;
-            const int n0 = (tile / a.tiles_m) * BN;
-            const int row = m0 + q * 32 + lane;
-            const bool row_ok = row < a.M;
-            const float rs = row_ok ? a.SCA[row] * (1.0f / 16129.0f) : 0.0f;
             for (int c = 0; c < BN / 32; ++c) {
                 const int nb = n0 + c * 32;
                 if (nb >= a.N) break;
@@ -235,8 +312,33 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int j = 0; j < 32; ++j) ci[j] = 0u;
                 }
                 if (nob == 0) {
+                    float p[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) pf[j] = 0u;
+                    for (int j = 0; j < 32; ++j) p[j] = 0.0f;
+                    if (reg_out) {
+                        // P[row, nb + j] = sum_o Xo[row, o] * Wo[nb + j, o], o ascending
+#pragma unroll
+                        for (int o = 0; o < kRegOutliers; ++o) {
+                            if (o < n_out) {
+                                const uint4 *wv =
+                                    reinterpret_cast<const uint4 *>(sl_w + o * BN + c * 32);
+#pragma unroll
+                                for (int v = 0; v < 4; ++v) {
+                                    const uint4 w8 = wv[v];
+                                    const __half2 *h = reinterpret_cast<const __half2 *>(&w8);
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const float2 wf = __half22float2(h[e]);
+                                        p[v * 8 + 2 * e] = fmaf(xo[o], wf.x, p[v * 8 + 2 * e]);
+                                        p[v * 8 + 2 * e + 1] =
+                                            fmaf(xo[o], wf.y, p[v * 8 + 2 * e + 1]);
+                                    }
+                                }
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) pf[j] = __float_as_uint(p[j]);
                 }
                 const int groups = min(32, a.N - nb) / 16;   // 1 or 2 groups of 16 columns
                 if (row_ok) {
@@ -248,18 +350,10 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             uint32_t packed[8];
 #pragma unroll
                             for (int j4 = 0; j4 < 4; ++j4) {
-                                const float4 sb = __ldg(reinterpret_cast<const float4 *>(
-                                    a.SCB + nb + g * 16 + j4 * 4));
-                                float b[4] = {0.f, 0.f, 0.f, 0.f};
-                                if (a.bias) {
-                                    const uint2 bb = __ldg(reinterpret_cast<const uint2 *>(
-                                        a.bias + nb + g * 16 + j4 * 4));
-                                    const float2 b01 = __half22float2(
-                                        *reinterpret_cast<const __half2 *>(&bb.x));
-                                    const float2 b23 = __half22float2(
-                                        *reinterpret_cast<const __half2 *>(&bb.y));
-                                    b[0] = b01.x; b[1] = b01.y; b[2] = b23.x; b[3] = b23.y;
-                                }
+                                const int cj = c * 32 + g * 16 + j4 * 4;
+                                const float4 sb = *reinterpret_cast<const float4 *>(sl_scb + cj);
+                                const float4 bv = *reinterpret_cast<const float4 *>(sl_bias + cj);
+                                const float b[4] = {bv.x, bv.y, bv.z, bv.w};
                                 const float sbv[4] = {sb.x, sb.y, sb.z, sb.w};
                                 float y[4];
 #pragma unroll
@@ -288,7 +382,11 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&tail->acc_empty[acc]));
+            if (lane == 0) {
+                mbar_arrive(smem_addr(&tail->acc_empty[acc]));
+                mbar_arrive(smem_addr(&tail->slice_empty));
+            }
+            sl_phase ^= 1;
             if (++acc == acc_stages) {
                 acc = 0;
                 acc_phase ^= 1;
@@ -373,6 +471,9 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s) {
                       BKB / 2, BN);
     if (!ok) return cudaErrorInvalidValue;
     Args a;
+    a.Xo = g.Xo;
+    a.Wo = g.Wo;
+    a.pitch = (int)g.pitch;
     a.count = g.count;
     a.cap = g.cap;
     a.SCA = g.SCA;

@@ -143,6 +143,11 @@ LINEAR_CASES = {
     "two_outlier_blocks": (96, 1024, 320, 70, 6.0, True, False),
     "single_tile_exact": (128, 128, 256, 6, 6.0, False, False),
     "many_tiles": (520, 768, 1296, 6, 6.0, True, False),
+    # outlier part formed in the GEMM epilogue (<= 16 columns) or by the tensor cores (more)
+    "outliers_16_epilogue": (200, 1024, 528, 16, 6.0, True, False),
+    "outliers_17_tensor_cores": (200, 1024, 528, 17, 6.0, True, False),
+    "outliers_9_fp16_w": (150, 512, 272, 9, 6.0, True, True),
+    "K32_half_outliers": (40, 32, 64, 16, 6.0, False, False),
 }
 
 
@@ -186,11 +191,12 @@ def test_linear_capacity_overflow_reports_status():
 
 def test_linear_bounded_wait_timeout_is_reported():
     """A wait limit of 1 ns makes the GEMM's pipeline waits give up: the kernel must record
-    LLMINT8_ERR_TIMEOUT, wind down and return; later calls are unaffected."""
-    X = _x(256, 2048, 6, seed=13)
-    W = synth.weight(512, 2048, 0.02, seed=13)
+    LLMINT8_ERR_TIMEOUT, wind down and return; later calls are unaffected.  One 128 x 256 tile
+    with K = 16384 keeps the epilogue waiting for the accumulator for tens of microseconds."""
+    X = _x(128, 16384, 6, seed=13)
+    W = synth.weight(256, 16384, 0.02, seed=13)
     CB, SCB = L.llmint8_quantize_weight_colwise(dev(W))
-    ws = torch.empty((L.llmint8_linear_workspace_size(256, 512, 2048, 64),), dtype=torch.uint8,
+    ws = torch.empty((L.llmint8_linear_workspace_size(128, 256, 16384, 64),), dtype=torch.uint8,
                      device="cuda")
     seen = set()
     try:
