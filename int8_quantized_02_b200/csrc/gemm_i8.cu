@@ -20,8 +20,8 @@
 // two routes:
 //   few outlier columns (n_out <= kRegOutliers, the usual case: a handful of feature
 //   dimensions) - the epilogue warps form P on the CUDA cores (fp32 FMAs) from their rows of
-//   Xo (registers) and the tile's slice of Wo (shared memory), both loaded while the main
-//   loop of the tile runs;
+//   Xo and the tile's slice of Wo, both staged in shared memory while the main loop of the
+//   tile runs;
 //   more - P is a tcgen05 kind::f16 product appended to the k-loop, accumulated in fp32 in
 //   the second half of TMEM, and the int32 accumulator is single-buffered.
 // Every wait is bounded (BoundedWait); a timeout records LLMINT8_ERR_TIMEOUT, drains the
@@ -46,11 +46,13 @@ constexpr int B_BYTES = BN * BKB;       // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int kRegOutliers = 32;        // outlier columns formed in the epilogue at most
+constexpr int kRegOutliers = 16;        // outlier columns formed in the epilogue at most
 // the tile's column slice, staged once per tile by the four epilogue warps together:
-// Wo [o][n] fp16, SCB [n] and bias [n] as fp32
+// Wo [o][n] fp16, SCB [n] and bias [n] as fp32; and per epilogue warp its rows of Xo,
+// [o][lane] fp32
 constexpr int SL_W_BYTES = kRegOutliers * BN * 2;
-constexpr int SL_BYTES = SL_W_BYTES + BN * 4 + BN * 4;
+constexpr int SL_XO_WARP = kRegOutliers * 32 * 4;
+constexpr int SL_BYTES = SL_W_BYTES + BN * 4 + BN * 4 + 4 * SL_XO_WARP;
 
 struct Tail {
     uint64_t full[STAGES];
@@ -99,6 +101,7 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     __half *sl_w = reinterpret_cast<__half *>(smem + STAGES * STAGE_BYTES);
     float *sl_scb = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + SL_W_BYTES);
     float *sl_bias = sl_scb + BN;
+    float *sl_xo = sl_bias + BN;
     Tail *tail = reinterpret_cast<Tail *>(smem + STAGES * STAGE_BYTES + SL_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -278,18 +281,17 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (!okf) break;
                 first = false;
             }
-            // this thread's row of Xo (the outlier columns of X)
-            float xo[kRegOutliers];
+            // this thread's row of Xo (the outlier columns of X), [o][lane] in this warp's part
+            float *xo_s = sl_xo + wq * (kRegOutliers * 32);
             if (reg_out) {
                 const int r = m0 + q * 32 + lane;
-#pragma unroll
-                for (int o8 = 0; o8 < kRegOutliers; o8 += 8) {
+                for (int o8 = 0; o8 < n_out; o8 += 8) {
                     uint4 v = make_uint4(0, 0, 0, 0);
-                    if (o8 < n_out && r < a.M)
+                    if (r < a.M)
                         v = __ldg(reinterpret_cast<const uint4 *>(a.Xo + (int64_t)r * a.pitch + o8));
                     const __half *h = reinterpret_cast<const __half *>(&v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) xo[o8 + e] = __half2float(h[e]);
+                    for (int e = 0; e < 8; ++e) xo_s[(o8 + e) * 32 + lane] = __half2float(h[e]);
                 }
             }
             const int row = m0 + q * 32 + lane;
@@ -317,22 +319,19 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int j = 0; j < 32; ++j) p[j] = 0.0f;
                     if (reg_out) {
                         // P[row, nb + j] = sum_o Xo[row, o] * Wo[nb + j, o], o ascending
+#pragma unroll 1
+                        for (int o = 0; o < n_out; ++o) {
+                            const float xv = xo_s[o * 32 + lane];
+                            const uint4 *wv = reinterpret_cast<const uint4 *>(sl_w + o * BN + c * 32);
 #pragma unroll
-                        for (int o = 0; o < kRegOutliers; ++o) {
-                            if (o < n_out) {
-                                const uint4 *wv =
-                                    reinterpret_cast<const uint4 *>(sl_w + o * BN + c * 32);
+                            for (int v = 0; v < 4; ++v) {
+                                const uint4 w8 = wv[v];
+                                const __half2 *h = reinterpret_cast<const __half2 *>(&w8);
 #pragma unroll
-                                for (int v = 0; v < 4; ++v) {
-                                    const uint4 w8 = wv[v];
-                                    const __half2 *h = reinterpret_cast<const __half2 *>(&w8);
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        const float2 wf = __half22float2(h[e]);
-                                        p[v * 8 + 2 * e] = fmaf(xo[o], wf.x, p[v * 8 + 2 * e]);
-                                        p[v * 8 + 2 * e + 1] =
-                                            fmaf(xo[o], wf.y, p[v * 8 + 2 * e + 1]);
-                                    }
+                                for (int e = 0; e < 4; ++e) {
+                                    const float2 wf = __half22float2(h[e]);
+                                    p[v * 8 + 2 * e] = fmaf(xv, wf.x, p[v * 8 + 2 * e]);
+                                    p[v * 8 + 2 * e + 1] = fmaf(xv, wf.y, p[v * 8 + 2 * e + 1]);
                                 }
                             }
                         }
