@@ -236,6 +236,14 @@ def check_brute_force(lib):
                                  threshold=t, want_C=True, lib=lib)
             assert np.array_equal(C.astype(np.int64), ref["C"]), idx
             assert np.array_equal(Y, ref["Y"]), (idx, keep)
+            # the sampled form of the layer, every position once in a shuffled order
+            M, N = X.shape[0], W.shape[0]
+            flat = rng.permutation(M * N)
+            rows, cols = flat // N, flat % N
+            Ys, Cs = oracle.linear_sampled(X, CB, SCB, rows, cols, bias=bias,
+                                           W_fp16=W if keep else None, threshold=t, lib=lib)
+            assert np.array_equal(Cs.astype(np.int64), ref["C"][rows, cols]), idx
+            assert np.array_equal(Ys, ref["Y"][rows, cols]), (idx, keep)
 
 
 def check_invariants(lib):
@@ -326,6 +334,8 @@ MUTANTS = [
     ("half_exponent_bias", r"ldexp\(\(double\)\(m \+ 1024\), e - 25\)",
      "ldexp((double)(m + 1024), e - 24)"),
     ("stores_multiplier_not_absmax", r"SCB\[n\] = amax;", "SCB[n] = 127.0f / amax;"),
+    ("sampled_rows_and_cols_swapped", r"Xq, SCA, rows\[s\], cols\[s\],",
+     "Xq, SCA, cols[s] % M, rows[s] % N,"),
 ]
 
 
