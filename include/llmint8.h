@@ -128,6 +128,8 @@ LLMINT8_API llmint8_status llmint8_dequant(const int8_t *CB, const float *SCB, i
  * Synchronizes `stream` and returns the device status word of a workspace used by the
  * last llmint8_linear / llmint8_quantize_rows_and_find_outliers call on it
  * (LLMINT8_OK, LLMINT8_ERR_OUTLIER_CAPACITY or LLMINT8_ERR_TIMEOUT), or LLMINT8_ERR_CUDA.
+ * The result is meaningful only for a workspace that at least one call has used; a
+ * zero-filled one reads LLMINT8_OK.
  */
 LLMINT8_API llmint8_status llmint8_device_status(const void *ws, void *stream);
 

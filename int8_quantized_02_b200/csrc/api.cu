@@ -295,7 +295,8 @@ llmint8_status llmint8_device_status(const void *ws, void *stream) {
     unsigned long long words[2] = {0, 0};   // status, timeout
     if (cudaMemcpy(words, ws, sizeof(words), cudaMemcpyDeviceToHost) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    if ((words[1] >> 4) == (words[0] >> 4)) return LLMINT8_ERR_TIMEOUT;
+    // epochs start at 1: a zero-filled header has recorded no call and no timeout
+    if ((words[0] >> 4) != 0 && (words[1] >> 4) == (words[0] >> 4)) return LLMINT8_ERR_TIMEOUT;
     return static_cast<llmint8_status>(words[0] & 0xFull);
 }
 
