@@ -239,6 +239,23 @@ def unit_value(units, seconds, unit):
     return units / seconds / 1e9 if unit == "GB/s" else units / seconds / 1e12
 
 
+def max_over_ranks(seconds: float, world: int, device=None) -> float:
+    """The slowest rank's time (every rank calls this at the same point)."""
+    if world <= 1:
+        return float(seconds)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(seconds)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(units_per_step: float, steps: int, world: int, seconds: float,
+                    unit: str) -> float:
+    """Units all ranks processed (replicas: the same per rank) / the max-over-ranks time."""
+    return unit_value(units_per_step * steps * world, seconds, unit)
+
+
 # ------------------------------------------------------------------------ our arm ----
 
 def run_ours(args, rank, world, local_rank):
@@ -303,11 +320,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     barrier()
     launches = L.llmint8_kernel_launch_count() - launches0
-    elapsed = e0.elapsed_time(e1) / 1e3
-    t = torch.tensor([elapsed], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed = float(t.item())
+    elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, device="cuda")
     if per_call_events:
         call_s = [sum(kev[s][j][0].elapsed_time(kev[s][j][1]) for s in range(args.steps))
                   / 1e3 / args.steps for j in range(len(calls))]
@@ -343,10 +356,7 @@ def run_ours(args, rank, world, local_rank):
     a1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_t = torch.tensor([a0.elapsed_time(a1) / 1e3], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_s = float(e2e_t.item())
+    e2e_s = max_over_ranks(a0.elapsed_time(a1) / 1e3, world, device="cuda")
 
     peaks = measured_peaks()
     traffic = profiled_traffic(args.workload)
@@ -365,7 +375,7 @@ def run_ours(args, rank, world, local_rank):
         timing = "CUDA events around each GEMM launch, averaged over the timed region"
     result = {
         "metric": "LLM.int8 linear TOPS (prefill) / weight GB/s (decode); fraction of roofline",
-        "value": unit_value(step_units * args.steps * world, elapsed, unit),
+        "value": whole_job_value(step_units, args.steps, world, elapsed, unit),
         "unit": unit,
         "n_gpus": world,
         "steps": args.steps,
@@ -383,7 +393,7 @@ def run_ours(args, rank, world, local_rank):
                                     + ("hbm_gbs" if bound == "hbm" else "2 x bf16_tflops (burst)"),
                      "kernel": kernel_name, "timing": timing,
                      "traffic": traffic},
-        "e2e": {"value": unit_value(step_units * e2e_steps * world, e2e_s, unit), "unit": unit,
+        "e2e": {"value": whole_job_value(step_units, e2e_steps, world, e2e_s, unit), "unit": unit,
                 "h2d_bytes_per_step": sum(c.h2d_bytes for c in calls),
                 "d2h_bytes_per_step": sum(c.d2h_bytes for c in calls)},
         "gpu_launches": int(launches),
