@@ -59,6 +59,11 @@ constexpr int QKEEP = (kDecodeMaxK / 16 / QCL + QWARPS - 1) / QWARPS;
 // k-blocks of a CTA's first tile requested into L2 ahead of the stage ring, so that HBM keeps
 // streaming while the first MMA waits for the quantized X
 constexpr int kPrefetchBlocks = 64;
+// Independent int32 accumulators per tile: k-block it accumulates into sub-accumulator
+// it % DSUB, so consecutive MMAs do not wait on each other's result (a 128 x 16 MMA is too
+// short to hide the accumulate dependency); the epilogue adds them (exact in int32).
+constexpr int DSUB = 4;
+constexpr uint32_t DTMEM_COLS = 2 * DSUB * kDecodeMaxM;   // double-buffered over tiles
 
 __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&v);
@@ -314,7 +319,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         fence_mbar_init();
         tma_prefetch_desc(&tmCB);
     }
-    if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), 32);
+    if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), DTMEM_COLS);
     // the next call's first kernel may launch now (it waits for this grid before it reads)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     tc_fence_before();
@@ -396,7 +401,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             for (int tile = blockIdx.x; have_x && tile < a.tiles; tile += gridDim.x) {
                 if (!wait(smem_addr(&tail->acc_empty[acc]), acc_phase ^ 1)) break;
                 tc_fence_after();
-                const uint32_t d = tmem + (uint32_t)(acc * DM);
+                const uint32_t d = tmem + (uint32_t)(acc * DSUB * DM);
                 bool good = true;
                 for (int it = 0; it < a.kblocks; ++it) {
                     const int kb = rotated_kblock(it, tile, a.kblocks);
@@ -407,10 +412,11 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                     tc_fence_after();
                     const uint32_t sa = smem_addr(smem + stage * DSTAGE);
                     const uint32_t sb = xq_base + (uint32_t)(kb * DM * 128);
+                    const uint32_t dsub = d + (uint32_t)((it % DSUB) * DM);
 #pragma unroll
                     for (int k = 0; k < DBK / 32; ++k)
-                        mma_i8(d, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
-                               (it | k) != 0);
+                        mma_i8(dsub, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
+                               (it >= DSUB) || k != 0);
                     tc_commit(smem_addr(&tail->empty[stage]));
                     if (++stage == S) {
                         stage = 0;
@@ -484,7 +490,15 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             if (!okw) break;
             tc_fence_after();
             uint32_t d[DM];
-            tmem_ld_32x16(tl + (uint32_t)(acc * DM), d);
+            tmem_ld_32x16(tl + (uint32_t)(acc * DSUB * DM), d);
+            for (int u = 1; u < DSUB; ++u) {
+                if (u >= a.kblocks) break;               // sub-accumulators never written
+                uint32_t e[DM];
+                tmem_ld_32x16(tl + (uint32_t)((acc * DSUB + u) * DM), e);
+                tmem_wait_ld();
+#pragma unroll
+                for (int m = 0; m < DM; ++m) d[m] += e[m];
+            }
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -508,7 +522,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 32);
+        tmem_dealloc(tmem, DTMEM_COLS);
     }
 }
 
