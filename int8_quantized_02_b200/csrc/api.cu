@@ -193,7 +193,7 @@ llmint8_status llmint8_quantize_rows_and_find_outliers(const uint16_t *X, int64_
                                           bitmap, outlier_idx, cap, n_outliers, next_status(h), s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     return from_cuda(launch_quantize_rows(Xh, M, K, bitmap, outlier_idx, n_outliers, cap, 0, Xq,
-                                          SCA, nullptr, s));
+                                          SCA, nullptr, nullptr, nullptr, nullptr, 0, nullptr, s));
 }
 
 llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
@@ -256,13 +256,10 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
                               idx, max_outliers, &h->n_outliers, status, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     e = launch_quantize_rows(Xh, M, K, bitmap, idx, &h->n_outliers, max_outliers, L.pitch, Xq, SCA,
-                             max_outliers > 0 ? Xo : nullptr, s);
+                             max_outliers > 0 ? Xo : nullptr, CB, SCB,
+                             reinterpret_cast<const __half *>(W_fp16), N,
+                             max_outliers > 0 ? Wo : nullptr, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-    if (max_outliers > 0) {
-        e = launch_gather_outlier_w(CB, SCB, reinterpret_cast<const __half *>(W_fp16), N, K, idx,
-                                    &h->n_outliers, max_outliers, L.pitch, Wo, s);
-        if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-    }
     GemmLaunch g;
     g.Xq = Xq;
     g.CB = CB;

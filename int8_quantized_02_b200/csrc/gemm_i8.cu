@@ -105,15 +105,8 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     Tail *tail = reinterpret_cast<Tail *>(smem + STAGES * STAGE_BYTES + SL_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // Outlier configuration of this call (uniform over the grid).
-    const int n_out = (int)min((int64_t)*a.count, a.cap);
-    const bool all_outliers = n_out >= a.K;            // then C == 0: skip the int8 blocks
-    const bool reg_out = n_out > 0 && n_out <= kRegOutliers && !all_outliers;
-    const int nob = reg_out ? 0 : (n_out + 63) / 64;   // fp16 k-blocks of 64 columns
-    const int nkb = all_outliers ? 0 : a.num_kb;
-    const int acc_stages = nob > 0 ? 1 : 2;
-    const int total_tiles = a.tiles_m * a.tiles_n;
-
+    // Prologue: nothing here reads global memory that the kernels before this one write, so
+    // it overlaps their tail (this grid is their programmatic dependent).
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_addr(&tail->full[s]), 1);
@@ -132,12 +125,25 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
-        if (nob > 0) {
+        if (a.cap > 0) {
             tma_prefetch_desc(&tmXo);
             tma_prefetch_desc(&tmWo);
         }
     }
     if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), TMEM_COLS);
+    // the quantized operands, scales and outlier list of this call are complete after this
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // Outlier configuration of this call (uniform over the grid).
+    const int n_out = (int)min((int64_t)*a.count, a.cap);
+    const bool all_outliers = n_out >= a.K;            // then C == 0: skip the int8 blocks
+    const bool reg_out = n_out > 0 && n_out <= kRegOutliers && !all_outliers;
+    const int nob = reg_out ? 0 : (n_out + 63) / 64;   // fp16 k-blocks of 64 columns
+    const int nkb = all_outliers ? 0 : a.num_kb;
+    const int acc_stages = nob > 0 ? 1 : 2;
+    const int total_tiles = a.tiles_m * a.tiles_n;
+
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -490,9 +496,19 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s) {
     a.timeout_ns = g.timeout_ns;
     const int tiles = a.tiles_m * a.tiles_n;
     const int grid = std::min(tiles, sms);
-    llmint8_gemm_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmXo, tmWo, a);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, llmint8_gemm_kernel, tmA, tmB, tmXo, tmWo, a);
     note_launches(1);
-    return cudaGetLastError();
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace llmint8

@@ -26,14 +26,14 @@ cudaError_t launch_outlier_detect(const __half *X, int64_t M, int64_t K, float t
                                   const ScanPlan &plan, uint32_t *partial, uint32_t *bitmap,
                                   int32_t *idx, int64_t cap, int32_t *count, StatusRef status,
                                   cudaStream_t s);
+// Row quantization of X (and, with Wo non-null, the gather of the outlier weights Wo
+// [N, xo_pitch] from CB/SCB or W16, in the same launch).  The scan, compaction and this
+// kernel are programmatic dependents of whatever precedes them in the stream.
 cudaError_t launch_quantize_rows(const __half *X, int64_t M, int64_t K, const uint32_t *bitmap,
                                  const int32_t *idx, const int32_t *count, int64_t cap,
                                  int64_t xo_pitch, int8_t *Xq, float *SCA, __half *Xo,
-                                 cudaStream_t s);
-cudaError_t launch_gather_outlier_w(const int8_t *CB, const float *SCB, const __half *W16,
-                                    int64_t N, int64_t K, const int32_t *idx,
-                                    const int32_t *count, int64_t cap, int64_t pitch, __half *Wo,
-                                    cudaStream_t s);
+                                 const int8_t *CB, const float *SCB, const __half *W16, int64_t N,
+                                 __half *Wo, cudaStream_t s);
 cudaError_t launch_quantize_weight(const __half *W, int64_t N, int64_t K, int8_t *CB, float *SCB,
                                    cudaStream_t s);
 cudaError_t launch_dequant(const int8_t *CB, const float *SCB, int64_t N, int64_t K,

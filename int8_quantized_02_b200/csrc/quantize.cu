@@ -4,8 +4,8 @@
 //   outlier_compact   - OR of the row-split bitmaps, ascending index list, count, status;
 //   quantize_rows     - row absmax over the regular columns, absmax quantization to int8
 //                       (outlier columns zeroed) and the compact gather of the fp16 outlier
-//                       columns Xo;
-//   gather_outlier_w  - the fp16 weights of the outlier columns, Wo[n, j];
+//                       columns Xo; the CTAs past the last row gather the fp16 weights of the
+//                       outlier columns, Wo[n, j];
 //   quantize_weight   - per-output-channel absmax quantization of W (one-time setup);
 //   dequant           - (CB * SCB) / 127 back to fp16.
 // Rounding follows the definition exactly: multiplier = fl32(127 / absmax) (IEEE division),
@@ -18,6 +18,15 @@ namespace llmint8 {
 namespace {
 
 constexpr int kThreads = 256;
+
+// Programmatic dependent launch: every kernel of a layer call is launched so that its CTAs
+// may start while the previous kernel in the stream finishes.  Each waits for that kernel
+// (and so for everything before it) before it touches global memory, and lets the next one
+// launch right away.
+__device__ __forceinline__ void pdl_wait_then_release() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&v);
@@ -66,6 +75,7 @@ __device__ __forceinline__ float block_max(float v, float *red) {
 __global__ void __launch_bounds__(kThreads)
 outlier_scan_kernel(const __half *__restrict__ X, int64_t M, int64_t K, float threshold,
                     int64_t rows_per_split, uint32_t *__restrict__ partial, int64_t nwords) {
+    pdl_wait_then_release();
     const int64_t chunk = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     const int64_t nchunks = K / 8;
     const int64_t r0 = (int64_t)blockIdx.y * rows_per_split;
@@ -104,7 +114,9 @@ outlier_scan_kernel(const __half *__restrict__ X, int64_t M, int64_t K, float th
 }
 
 // One CTA of 1024 threads: OR over the row splits, popcount, exclusive scan, ascending
-// index list.  Also writes the workspace status word (resetting it for this call).
+// index list.  Also writes the workspace status word (resetting it for this call).  The OR
+// over the splits is spread over every thread: thread t takes word t % nwords' share of
+// the splits when nwords < 1024, and the shares meet in shared memory.
 constexpr int kCompactThreads = 1024;
 constexpr int kMaxWordsPerThread = 4;   // nwords <= 4096 (K <= 131072)
 
@@ -112,8 +124,37 @@ __global__ void __launch_bounds__(kCompactThreads)
 outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t nwords,
                        int32_t *__restrict__ idx, int64_t cap, int32_t *__restrict__ count_out,
                        uint32_t *__restrict__ bitmap_out, StatusRef status) {
+    pdl_wait_then_release();
     __shared__ int warp_tot[32];
+    __shared__ uint32_t merged[kCompactThreads];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (nwords < kCompactThreads) {
+        // parts of the split range per word
+        const int parts = kCompactThreads / (int)nwords;
+        const int wi = tid % (int)nwords, part = tid / (int)nwords;
+        uint32_t v = 0;
+        if (part < parts) {
+            const int s0 = (int)((int64_t)splits * part / parts);
+            const int s1 = (int)((int64_t)splits * (part + 1) / parts);
+            int sp = s0;
+            for (; sp + 4 <= s1; sp += 4) {
+                const uint32_t a0 = partial[(int64_t)sp * nwords + wi];
+                const uint32_t a1 = partial[(int64_t)(sp + 1) * nwords + wi];
+                const uint32_t a2 = partial[(int64_t)(sp + 2) * nwords + wi];
+                const uint32_t a3 = partial[(int64_t)(sp + 3) * nwords + wi];
+                v |= a0 | a1 | a2 | a3;
+            }
+            for (; sp < s1; ++sp) v |= partial[(int64_t)sp * nwords + wi];
+        }
+        merged[tid] = v;
+        __syncthreads();
+        if (tid < nwords) {
+            uint32_t o = 0;
+            for (int pp = 0; pp < parts; ++pp) o |= merged[pp * (int)nwords + tid];
+            merged[tid] = o;      // only threads < nwords write, after every read above
+        }
+        __syncthreads();
+    }
     const int wpt = (int)ceil_div(nwords, kCompactThreads);
     const int64_t w0 = (int64_t)tid * wpt;
     uint32_t w[kMaxWordsPerThread];
@@ -124,7 +165,11 @@ outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t
         const int64_t wi = w0 + i;
         if (i < wpt && wi < nwords) {
             uint32_t v = 0;
-            for (int s = 0; s < splits; ++s) v |= partial[(int64_t)s * nwords + wi];
+            if (nwords < kCompactThreads) {
+                v = merged[wi];
+            } else {
+                for (int sp = 0; sp < splits; ++sp) v |= partial[(int64_t)sp * nwords + wi];
+            }
             w[i] = v;
             bitmap_out[wi] = v;
             cnt += __popc(v);
@@ -167,16 +212,55 @@ outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t
     }
 }
 
-// One CTA per row.  Row values stay in registers for K <= 8 * 256 * kCache.
+// The fp16 weights of the outlier columns for weight row n (one warp).
+__device__ __forceinline__ void gather_w_row(const int8_t *__restrict__ CB,
+                                             const float *__restrict__ SCB,
+                                             const __half *__restrict__ W16, int64_t n, int64_t K,
+                                             const int32_t *__restrict__ idx, int64_t n_o,
+                                             int64_t pitch, __half *__restrict__ Wo, int lane) {
+    const int64_t n_o64 = align_up(n_o, 64);
+    const float scb = SCB[n];
+    for (int64_t j = lane; j < n_o64; j += 32) {
+        __half v = __float2half_rn(0.0f);
+        if (j < n_o) {
+            const int64_t col = idx[j];
+            if (W16 != nullptr)
+                v = W16[n * K + col];
+            else
+                v = __float2half_rn(__fdiv_rn(__fmul_rn((float)CB[n * K + col], scb), 127.0f));
+        }
+        Wo[n * pitch + j] = v;
+    }
+}
+
+struct GatherW {
+    const int8_t *CB;
+    const float *SCB;
+    const __half *W16;
+    __half *Wo;          // null: no gather
+    int64_t N;
+};
+
+// One CTA per row of X; CTAs past the last row gather Wo, one warp per weight row.
+// Row values stay in registers for K <= 8 * 256 * kCache.
 constexpr int kCache = 8;
 
 __global__ void __launch_bounds__(kThreads)
-quantize_rows_kernel(const __half *__restrict__ X, int64_t K, const uint32_t *__restrict__ bitmap,
-                     const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
-                     int64_t cap, int64_t xo_pitch, int8_t *__restrict__ Xq,
-                     float *__restrict__ SCA, __half *__restrict__ Xo) {
+quantize_rows_kernel(const __half *__restrict__ X, int64_t M, int64_t K,
+                     const uint32_t *__restrict__ bitmap, const int32_t *__restrict__ idx,
+                     const int32_t *__restrict__ count, int64_t cap, int64_t xo_pitch,
+                     int8_t *__restrict__ Xq, float *__restrict__ SCA, __half *__restrict__ Xo,
+                     const GatherW gw) {
+    pdl_wait_then_release();
     __shared__ float red[32];
     const int64_t row = blockIdx.x;
+    if (row >= M) {
+        const int64_t n = (row - M) * (kThreads / 32) + (threadIdx.x >> 5);
+        if (n < gw.N)
+            gather_w_row(gw.CB, gw.SCB, gw.W16, n, K, idx, min((int64_t)*count, cap), xo_pitch,
+                         gw.Wo, threadIdx.x & 31);
+        return;
+    }
     const int64_t nchunks = K / 8;
     const uint4 *xr = reinterpret_cast<const uint4 *>(X + row * K);
     uint4 cache[kCache];
@@ -232,31 +316,6 @@ quantize_rows_kernel(const __half *__restrict__ X, int64_t K, const uint32_t *__
         const __half *x = X + row * K;
         for (int64_t j = threadIdx.x; j < n_o64; j += kThreads)
             Xo[row * xo_pitch + j] = j < n_o ? x[idx[j]] : __float2half_rn(0.0f);
-    }
-}
-
-// One warp per output channel n.
-__global__ void __launch_bounds__(kThreads)
-gather_outlier_w_kernel(const int8_t *__restrict__ CB, const float *__restrict__ SCB,
-                        const __half *__restrict__ W16, int64_t N, int64_t K,
-                        const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
-                        int64_t cap, int64_t pitch, __half *__restrict__ Wo) {
-    const int64_t n = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (n >= N) return;
-    const int64_t n_o = min((int64_t)*count, cap);
-    const int64_t n_o64 = align_up(n_o, 64);
-    const float scb = SCB[n];
-    for (int64_t j = lane; j < n_o64; j += 32) {
-        __half v = __float2half_rn(0.0f);
-        if (j < n_o) {
-            const int64_t col = idx[j];
-            if (W16 != nullptr)
-                v = W16[n * K + col];
-            else
-                v = __float2half_rn(__fdiv_rn(__fmul_rn((float)CB[n * K + col], scb), 127.0f));
-        }
-        Wo[n * pitch + j] = v;
     }
 }
 
@@ -350,38 +409,60 @@ ScanPlan scan_plan(int64_t M, int64_t K) {
     return p;
 }
 
+namespace {
+
+// Launch with the programmatic-stream-serialization attribute (see pdl_wait_then_release).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t s,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+}  // namespace
+
 cudaError_t launch_outlier_detect(const __half *X, int64_t M, int64_t K, float threshold,
                                   const ScanPlan &plan, uint32_t *partial, uint32_t *bitmap,
                                   int32_t *idx, int64_t cap, int32_t *count, StatusRef status,
                                   cudaStream_t s) {
     dim3 grid((unsigned)plan.col_blocks, (unsigned)plan.splits);
-    outlier_scan_kernel<<<grid, kThreads, 0, s>>>(X, M, K, threshold, plan.rows_per_split,
-                                                  partial, plan.nwords);
-    outlier_compact_kernel<<<1, kCompactThreads, 0, s>>>(partial, (int)plan.splits, plan.nwords,
-                                                         idx, cap, count, bitmap, status);
-    note_launches(2);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(outlier_scan_kernel, grid, dim3(kThreads), s, X, M, K, threshold,
+                               plan.rows_per_split, partial, plan.nwords);
+    note_launches(1);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(outlier_compact_kernel, dim3(1), dim3(kCompactThreads), s,
+                   (const uint32_t *)partial, (int)plan.splits, plan.nwords, idx, cap, count,
+                   bitmap, status);
+    note_launches(1);
+    return e;
 }
 
 cudaError_t launch_quantize_rows(const __half *X, int64_t M, int64_t K, const uint32_t *bitmap,
                                  const int32_t *idx, const int32_t *count, int64_t cap,
                                  int64_t xo_pitch, int8_t *Xq, float *SCA, __half *Xo,
-                                 cudaStream_t s) {
-    quantize_rows_kernel<<<(unsigned)M, kThreads, 0, s>>>(X, K, bitmap, idx, count, cap, xo_pitch,
-                                                          Xq, SCA, Xo);
+                                 const int8_t *CB, const float *SCB, const __half *W16, int64_t N,
+                                 __half *Wo, cudaStream_t s) {
+    GatherW gw;
+    gw.CB = CB;
+    gw.SCB = SCB;
+    gw.W16 = W16;
+    gw.Wo = Wo;
+    gw.N = Wo != nullptr ? N : 0;
+    const int64_t gather_ctas = ceil_div(gw.N, kThreads / 32);
+    const cudaError_t e = launch_pdl(quantize_rows_kernel, dim3((unsigned)(M + gather_ctas)),
+                                     dim3(kThreads), s, X, M, K, bitmap, idx, count, cap,
+                                     xo_pitch, Xq, SCA, Xo, gw);
     note_launches(1);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_gather_outlier_w(const int8_t *CB, const float *SCB, const __half *W16,
-                                    int64_t N, int64_t K, const int32_t *idx,
-                                    const int32_t *count, int64_t cap, int64_t pitch, __half *Wo,
-                                    cudaStream_t s) {
-    const unsigned blocks = (unsigned)ceil_div(N, kThreads / 32);
-    gather_outlier_w_kernel<<<blocks, kThreads, 0, s>>>(CB, SCB, W16, N, K, idx, count, cap,
-                                                        pitch, Wo);
-    note_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_quantize_weight(const __half *W, int64_t N, int64_t K, int8_t *CB, float *SCB,
