@@ -287,8 +287,9 @@ def run_ours(args, rank, world, local_rank):
             raise SystemExit(f"{c.name}: device status {L.status_string(st)}")
 
     # ---- timed region: whole steps, inputs resident, CUDA events on the launching stream.
-    # Prefill calls run for milliseconds, so a pair of profile events around each GEMM launch
-    # costs nothing measurable and gives the dominant kernel's own duration.  A decode call
+    # Prefill calls run for a tenth of a millisecond or more, so a pair of profile events
+    # around each GEMM launch costs little (the GEMM then starts after its quantize kernel
+    # instead of overlapping its tail) and gives the dominant kernel's own duration.  A decode call
     # lasts about 20 us and an event pair adds about 5 us, so decode records no per-call
     # events: its weight-streaming kernel spans the whole call (the quantize kernel runs under
     # it as a programmatic dependent), and the call's duration is region time / calls.
