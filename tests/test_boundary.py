@@ -98,3 +98,15 @@ def test_argument_errors_before_any_launch(lib):
                               ctypes.c_float(6.0), 0, None, None, 0, None, None) == \
         llmint8.ERR_INVALID_ARG
     assert lib.llmint8_dequant(None, None, 16, 16, None, None) == llmint8.ERR_INVALID_ARG
+
+
+def test_empty_and_out_of_range_shapes_are_rejected_before_any_launch(lib):
+    fake = ctypes.c_void_p(1 << 20)      # aligned, never dereferenced
+    for M, K, N in ((0, 1024, 1024), (16, 0, 1024), (16, 1024, 0), (16, 262144, 1024),
+                    (16, 1000, 1024), (16, 1024, 1000)):
+        assert lib.llmint8_linear(fake, M, K, fake, fake, N, None, None, ctypes.c_float(6.0),
+                                  0, fake, fake, 1 << 20, None, None) == \
+            llmint8.ERR_UNSUPPORTED_SHAPE, (M, K, N)
+    assert lib.llmint8_quantize_weight_colwise(fake, 0, 1024, fake, fake, None) == \
+        llmint8.ERR_UNSUPPORTED_SHAPE
+    assert lib.llmint8_dequant(fake, fake, 16, 8, fake, None) == llmint8.ERR_UNSUPPORTED_SHAPE

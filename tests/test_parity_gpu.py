@@ -311,3 +311,23 @@ def test_linear_plan_matches_the_call():
         got = host(plan())
         assert np.array_equal(got, ref)
     assert L.llmint8_device_status(plan.workspace) == L.OK
+
+
+def test_maximum_K_accumulator_bound():
+    # K = 131072, the largest K accepted: every |Xq| and |CB| code is 127, so each int32
+    # accumulator reaches K * 127^2 = 2,114,060,288, within 2 % of the int32 limit
+    K = 131072
+    X = np.ones((20, K), np.float16)
+    X[1] *= -1
+    X[3, :] = 0.5
+    W = np.full((48, K), 0.25, np.float16)
+    W[5] *= -1
+    Y_gpu, _ = _check_linear(X, W, 6.0, cap=64)
+    assert np.isfinite(Y_gpu).all()
+
+
+def test_decode_path_limits_K8192_cap256():
+    # the decode path's largest K and outlier capacity, with 200 outlier columns
+    X = _x(16, 8192, 200, lo=6.0, hi=60.0, row_frac=1.0, seed=41)
+    W = synth.weight(512, 8192, 0.02, seed=41)
+    _check_linear(X, W, 6.0, cap=256)
