@@ -193,6 +193,18 @@ def llmint8_linear(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor, bias=No
     return Y
 
 
+def llmint8_linear_fp16_weight(X: torch.Tensor, W: torch.Tensor, bias=None,
+                               threshold: float = 6.0, max_outliers: int | None = None, Y=None,
+                               workspace=None, CB=None, SCB=None, stream=None):
+    """The layer with fp16 weights kept (the blog's has_fp16_weights=True, section 用法):
+    every call quantizes W per output channel (CB, SCB) and the outlier columns use the
+    original fp16 rows of W.  Two calls of the C ABI, both on the GPU:
+    llmint8_quantize_weight_colwise, then llmint8_linear with W_fp16 = W."""
+    CB, SCB = llmint8_quantize_weight_colwise(W, CB, SCB, stream)
+    return llmint8_linear(X, CB, SCB, bias=bias, W_fp16=W, threshold=threshold,
+                          max_outliers=max_outliers, Y=Y, workspace=workspace, stream=stream)
+
+
 class LinearPlan:
     """One llmint8_linear call with its arguments checked and marshalled once.
 

@@ -331,3 +331,30 @@ def test_decode_path_limits_K8192_cap256():
     X = _x(16, 8192, 200, lo=6.0, hi=60.0, row_frac=1.0, seed=41)
     W = synth.weight(512, 8192, 0.02, seed=41)
     _check_linear(X, W, 6.0, cap=256)
+
+
+@pytest.mark.parametrize("M", [8, 96])          # decode path, GEMM path
+def test_fp16_weight_forward_matches_oracle(M):
+    X = _x(M, 1024, 5, lo=6.0, hi=30.0, row_frac=1.0, seed=51 + M)
+    W = synth.weight(272, 1024, 0.02, seed=51)
+    b = synth.bias(272, seed=51)
+    Y = L.llmint8_linear_fp16_weight(dev(X), dev(W), bias=dev(b), threshold=6.0,
+                                     max_outliers=64)
+    CB_o, SCB_o = oracle.quantize_weight_colwise(W)
+    Y_o = oracle.linear(X, CB_o, SCB_o, bias=b, W_fp16=W, threshold=6.0)
+    assert_y_close(host(Y), Y_o)
+
+
+def test_saved_state_reloads_to_the_same_output(tmp_path):
+    from int8_quantized_02_b200 import state
+    X = _x(16, 2048, 6, lo=6.0, hi=60.0, row_frac=1.0, seed=61)
+    W = synth.weight(512, 2048, 0.02, seed=61)
+    b = synth.bias(512, seed=61)
+    CB, SCB = L.llmint8_quantize_weight_colwise(dev(W))
+    Y0 = host(L.llmint8_linear(dev(X), CB, SCB, bias=dev(b), threshold=6.0, max_outliers=64))
+    path = str(tmp_path / "layer.llmint8")
+    state.save_int8_weight(path, CB, SCB, threshold=6.0, bias=dev(b))
+    st = state.load_int8_weight(path, device="cuda")
+    Y1 = host(L.llmint8_linear(dev(X), st["CB"], st["SCB"], bias=st["bias"],
+                               threshold=st["threshold"], max_outliers=64))
+    assert np.array_equal(Y0, Y1)
