@@ -76,12 +76,33 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
 }
 
 // Byte offset of Xq[m, k0 ..] (k0 a multiple of 8) in the 128-byte-swizzled K-major layout:
-// per 128-column block, 16 rows of 128 bytes in two 8-row atoms of 1024 bytes; the 16-byte
-// chunk index within a row is XORed with (row mod 8).
-__device__ __forceinline__ uint32_t xq_offset(int m, int k0) {
+// per 128-column block, `rows` (16, or 8 when M <= 8) rows of 128 bytes in 8-row atoms of
+// 1024 bytes; the 16-byte chunk index within a row is XORed with (row mod 8).  With 8 rows
+// the MMA's second 8-row group is one shared all-zero atom after the last block (see
+// image_desc), so the image takes half the shared memory and the weight ring two more stages.
+__device__ __forceinline__ uint32_t xq_offset(int m, int k0, int rows) {
     const int kb = k0 >> 7, c = k0 & 127;
-    return (uint32_t)(kb * (DM * 128) + (m >> 3) * 1024 + (m & 7) * 128 +
+    return (uint32_t)(kb * (rows * 128) + (m >> 3) * 1024 + (m & 7) * 128 +
                       ((((c >> 4) ^ (m & 7)) << 4) | (c & 15)));
+}
+
+__host__ __device__ constexpr int image_rows(int M) { return M <= 8 ? 8 : kDecodeMaxM; }
+// Bytes of the image: the blocks, plus the shared zero atom when it has 8 rows.
+__host__ __device__ constexpr int image_bytes(int kblocks, int rows) {
+    return kblocks * rows * 128 + (rows == 8 ? 1024 : 0);
+}
+
+// Descriptor of the image's block at `saddr` (+ k offset) for the 16-column MMA operand: the
+// two 8-row groups are `sbo` bytes apart (1024 in the 16-row image; in the 8-row image the
+// distance to the zero atom, so that rows 8..15 read as zeros).
+__device__ __forceinline__ uint64_t image_desc(uint32_t saddr, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);      // start address / 16
+    d |= (uint64_t)1u << 16;                      // leading byte offset (unused, 16 B)
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;  // stride byte offset between 8-row groups
+    d |= (uint64_t)1u << 46;                      // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                      // swizzle: 128 B
+    return d;
 }
 
 __device__ __forceinline__ uint32_t outlier_bits(const float *f, float threshold) {
@@ -121,6 +142,7 @@ struct QArgs {
     int32_t *count;
     StatusRef status;
     unsigned long long epoch;
+    int rows;                                // image rows: 16, or 8 when M <= 8
 };
 
 // One cluster of QCL CTAs.  CTA r owns the chunk pairs [r*PP, (r+1)*PP); one thread per
@@ -206,7 +228,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(co
                 unpack8(v[i], f);
                 q = quant8(f, mul, fl[i]);
             }
-            *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8)) = q;
+            if (m < a.rows) *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8, a.rows)) = q;
         }
     }
     // every CTA's part of the image is written before CTA 0 publishes it
@@ -215,12 +237,15 @@ __global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(co
     cluster_barrier_all();
     if (r != 0) return;   // nothing of this CTA is read by its peers any more
 
-    // CTA 0: padding columns of the image, ascending outlier list, count, status, X there
+    // CTA 0: padding columns of the image (and its zero atom), ascending outlier list, count,
+    // status
     const int kpad_chunks = (a.K + 127) / 128 * 16;
-    for (int i = t; i < (kpad_chunks - nchunks) * DM; i += QTHREADS) {
-        const int c = nchunks + i / DM, mm = i % DM;
-        *reinterpret_cast<uint2 *>(a.image + xq_offset(mm, c * 8)) = make_uint2(0, 0);
+    for (int i = t; i < (kpad_chunks - nchunks) * a.rows; i += QTHREADS) {
+        const int c = nchunks + i / a.rows, mm = i % a.rows;
+        *reinterpret_cast<uint2 *>(a.image + xq_offset(mm, c * 8, a.rows)) = make_uint2(0, 0);
     }
+    if (a.rows == 8 && t < 128)
+        reinterpret_cast<uint2 *>(a.image + (kpad_chunks / 16) * 1024)[t] = make_uint2(0, 0);
     if (warp == 0) {
         const int per = (nchunks + 31) / 32;
         const int c0 = lane * per, c1 = min(nchunks, c0 + per);
@@ -292,6 +317,7 @@ struct DArgs {
     uint32_t xq_off;                     // byte offsets in shared memory
     uint32_t tail_off;
     uint64_t timeout_ns;
+    int rows;                            // image rows: 16, or 8 when M <= 8
 };
 
 __global__ void __launch_bounds__(DTHREADS, 1)
@@ -389,7 +415,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             }
             fence_proxy_async_global();
             const uint32_t xbar = smem_addr(&tail->xbar);
-            const uint32_t img_bytes = (uint32_t)(a.kblocks * DBK * DM);
+            const uint32_t img_bytes = (uint32_t)image_bytes(a.kblocks, a.rows);
             mbar_arrive_expect_tx(xbar, img_bytes + (uint32_t)sizeof(DecodeTables));
             bulk_load_1d(smem_addr(xq), a.image, img_bytes, xbar);
             bulk_load_1d(smem_addr(&tail->tab), a.tables, (uint32_t)sizeof(DecodeTables), xbar);
@@ -411,11 +437,13 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                     }
                     tc_fence_after();
                     const uint32_t sa = smem_addr(smem + stage * DSTAGE);
-                    const uint32_t sb = xq_base + (uint32_t)(kb * DM * 128);
+                    const uint32_t sb = xq_base + (uint32_t)(kb * a.rows * 128);
+                    const uint32_t sbo =
+                        a.rows == 8 ? (uint32_t)((a.kblocks - kb) * 1024) : 1024u;
                     const uint32_t dsub = d + (uint32_t)((it % DSUB) * DM);
 #pragma unroll
                     for (int k = 0; k < DBK / 32; ++k)
-                        mma_i8(dsub, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
+                        mma_i8(dsub, sw128_desc(sa + 32 * k), image_desc(sb + 32 * k, sbo), idesc,
                                (it >= DSUB) || k != 0);
                     tc_commit(smem_addr(&tail->empty[stage]));
                     if (++stage == S) {
@@ -575,6 +603,7 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     q.count = d.count;
     q.status = d.status;
     q.epoch = d.status.tag >> 4;
+    q.rows = image_rows((int)d.M);
     {
         cudaLaunchConfig_t qc = {};
         cudaLaunchAttribute qa[2];
@@ -615,7 +644,8 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     a.tiles = (int)ceil_div(d.N, DBM);
     a.timeout_ns = d.timeout_ns;
     // shared memory: [stages][quantized X][tail], 1024-byte aligned pieces
-    const int xq_bytes = a.kblocks * DBK * DM;
+    a.rows = image_rows((int)d.M);
+    const int xq_bytes = (int)align_up(image_bytes(a.kblocks, a.rows), 1024);
     const int tail_bytes = (int)align_up(sizeof(DTail), 1024);
     const int room = SMEM_LIMIT - 1024 - xq_bytes - tail_bytes;
     a.stages = std::min(DMAX_STAGES, room / DSTAGE);
