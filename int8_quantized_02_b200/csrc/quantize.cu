@@ -72,6 +72,8 @@ __device__ __forceinline__ float block_max(float v, float *red) {
 }
 
 // grid (ceil(K/8/256), splits); thread = 8 consecutive columns, loops over its row split.
+// Plain cached loads: X is read again right after by the row quantization, from L2 when it
+// fits there.
 __global__ void __launch_bounds__(kThreads)
 outlier_scan_kernel(const __half *__restrict__ X, int64_t M, int64_t K, float threshold,
                     int64_t rows_per_split, uint32_t *__restrict__ partial, int64_t nwords) {
@@ -87,7 +89,7 @@ outlier_scan_kernel(const __half *__restrict__ X, int64_t M, int64_t K, float th
         for (; r + 4 <= r1; r += 4) {
             uint4 v[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = __ldcs(p + u * nchunks);
+            for (int u = 0; u < 4; ++u) v[u] = __ldg(p + u * nchunks);
             p += 4 * nchunks;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -99,7 +101,7 @@ outlier_scan_kernel(const __half *__restrict__ X, int64_t M, int64_t K, float th
         }
         for (; r < r1; ++r) {
             float f[8];
-            unpack8(__ldcs(p), f);
+            unpack8(__ldg(p), f);
             p += nchunks;
 #pragma unroll
             for (int e = 0; e < 8; ++e) bits |= (fabsf(f[e]) >= threshold ? 1u : 0u) << e;
