@@ -88,15 +88,18 @@ class ClockSampler:
         except Exception:  # noqa: BLE001 - clocks are reported as unavailable
             self._nvml = None
 
-    def _run(self):
+    def _sample(self):
         nv, h = self._nvml, self._handle
+        try:
+            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.samples.append((sm, reasons))
+        except Exception:  # noqa: BLE001
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.samples.append((sm, reasons))
-            except Exception:  # noqa: BLE001
-                pass
+            self._sample()
             time.sleep(0.005)
 
     def __enter__(self):
@@ -109,6 +112,7 @@ class ClockSampler:
         self._stop.set()
         if self._thread is not None:
             self._thread.join(timeout=10)
+            self._sample()              # the clocks as the region ends
 
     def summary(self):
         if self._nvml is None:
@@ -385,7 +389,8 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "i8/i32 (fp16 in/out, fp16 outlier product)",
+        "dtype": "i8",
+        "dtype_note": "int8 x int8 -> int32 product; fp16 in/out; fp16 x fp16 -> fp32 outlier part",
         "data": "synthetic (seeded, int8_quantized_02_b200.synth)",
         "config": workload_config(args.workload, calls),
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": roof_unit,
