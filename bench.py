@@ -504,7 +504,7 @@ def run_reference(args, rank, world):
         "metric": "LLM.int8 linear TOPS (prefill) / weight GB/s (decode); fraction of roofline",
         "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle; int8 codes exact)",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, int8_quantized_02_b200.synth)",
         "config": {"workload": args.workload, "sample": desc, "parallelism": "replicas"},
         "cpu_baseline": {"value": value, "unit": unit, "cores": _cores(), "kind": "oracle",
