@@ -1,6 +1,10 @@
 // The LLM.int8() product on the 5th-generation tensor cores of sm_100a.
 //
-// One persistent CTA per SM computes 128 x 256 output tiles of
+// One persistent CTA per SM computes 128 x 256 output tiles (or, for M > 128, a pair of CTAs in
+// a cluster computes 256 x 256 tiles with tcgen05.mma.cta_group::2: each CTA holds its 128
+// rows of Xq and 128 of the 256 weight rows of a stage, and its TMEM the 128 x 256 result of
+// its rows; the pair halves the weight bytes each SM brings in per MAC and fits six stages)
+// of
 //     Y = fp16( C * SCA_i * SCB_n / 127^2 + P + bias_n ),
 //     C = Xq . CB^T    (int8 x int8 -> int32, tcgen05.mma kind::i8, exact)
 //     P = Xo . Wo^T    (fp16 x fp16 -> fp32, tcgen05.mma kind::f16, the outlier columns)
@@ -12,8 +16,9 @@
 //
 // Warp roles (192 threads):
 //   warp 0      TMA producer: k-blocks of Xq / CB (128 B of K each), then of Xo / Wo
-//               (64 fp16 of K each) - both fill the same 48 KB shared-memory stages;
-//   warp 1      TMEM allocator and MMA issuer (one thread);
+//               (64 fp16 of K each) - both fill the same shared-memory stages (48 KB, or
+//               32 KB per CTA of a pair, whose loads complete on the pair leader's barrier);
+//   warp 1      TMEM allocator and MMA issuer (one thread; of a pair, the leader's only);
 //   warps 2..5  epilogue: TMEM -> registers -> dequantize, add P and bias -> fp16 -> global.
 // TMEM (512 columns): the int32 accumulator is double-buffered (2 x 256 columns) so the
 // epilogue of a tile overlaps the main loop of the next.  The outlier product P takes one of
@@ -25,7 +30,9 @@
 //   more - P is a tcgen05 kind::f16 product appended to the k-loop, accumulated in fp32 in
 //   the second half of TMEM, and the int32 accumulator is single-buffered.
 // Every wait is bounded (BoundedWait); a timeout records LLMINT8_ERR_TIMEOUT, drains the
-// copies and MMAs in flight, frees TMEM and returns.
+// copies and MMAs in flight, frees TMEM and returns.  A pair's CTAs exit only after the
+// leader has drained the loads of both and the second CTA has made its last arrive on the
+// leader's barriers.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -37,14 +44,22 @@ namespace llmint8 {
 
 namespace {
 
-constexpr int BM = 128;                 // tile rows (M)
+constexpr int BM = 128;                 // tile rows (M) held by one CTA
 constexpr int BN = 256;                 // tile columns (N)
 constexpr int BKB = 128;                // bytes of K per stage row (128 int8 or 64 fp16)
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BKB;       // 16 KB
-constexpr int B_BYTES = BN * BKB;       // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
+
+// Single CTA (PAIR = false): 128 x 256 tiles, 4 stages of 16 + 32 KB.  CTA pair: 256 x 256
+// tiles, each CTA 6 stages of 16 KB (its Xq rows) + 16 KB (its half of the weight rows).
+template <bool PAIR>
+struct Cfg {
+    static constexpr int STAGES = PAIR ? 6 : 4;
+    static constexpr int B_ROWS = PAIR ? BN / 2 : BN;
+    static constexpr int TILE_M = PAIR ? 2 * BM : BM;
+    static constexpr int A_BYTES = BM * BKB;
+    static constexpr int B_BYTES = B_ROWS * BKB;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+};
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int kRegOutliers = 16;        // outlier columns formed in the epilogue at most
 // the tile's column slice, staged once per tile by the four epilogue warps together:
@@ -54,19 +69,27 @@ constexpr int SL_W_BYTES = kRegOutliers * BN * 2;
 constexpr int SL_XO_WARP = kRegOutliers * 32 * 4;
 constexpr int SL_BYTES = SL_W_BYTES + BN * 4 + BN * 4 + 4 * SL_XO_WARP;
 
+template <int NSTAGES>
 struct Tail {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[NSTAGES];
+    uint64_t empty[NSTAGES];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t mma_done;
     uint64_t slice_full;                // the four epilogue warps staged the column slice
     uint64_t slice_empty;               // ... and are done reading it
+    uint64_t loads_drained;             // pair, second CTA: the leader drained every load
+    uint64_t peer_exit;                 // pair, leader: the second CTA made its last arrive
     uint32_t tmem_base;
     int abort_flag;
 };
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SL_BYTES + 1024 + (int)sizeof(Tail);
-static_assert(SMEM_BYTES <= 232448, "fits the opt-in shared memory of one CTA");
+template <bool PAIR>
+constexpr int smem_bytes() {
+    return Cfg<PAIR>::STAGES * Cfg<PAIR>::STAGE_BYTES + SL_BYTES + 1024 +
+           (int)sizeof(Tail<Cfg<PAIR>::STAGES>);
+}
+static_assert(smem_bytes<false>() <= 232448, "fits the opt-in shared memory of one CTA");
+static_assert(smem_bytes<true>() <= 232448, "fits the opt-in shared memory of one CTA");
 
 struct Args {
     const __half *Xo;        // [M, pitch]
@@ -86,15 +109,68 @@ struct Args {
     uint64_t timeout_ns;
 };
 
+// ---- CTA-pair forms (tcgen05 cta_group::2).  The pair's leader (rank 0) issues the MMAs;
+// operand addresses are the same shared-memory offsets in both CTAs.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *tm, int x,
+                                                 int y, uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+__device__ __forceinline__ void mma_i8_pair(uint32_t d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_f16_pair(uint32_t d, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on the barrier at `bar` in both CTAs of the pair once the pair's MMAs issued so far
+// by this thread have completed.
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\t"
+        "mov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], m;\n\t}" ::"r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
     __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmXo,
-                    const __grid_constant__ CUtensorMap tmWo, const Args a) {
+template <bool PAIR>
+__device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensorMap &tmB,
+                                          const CUtensorMap &tmXo, const CUtensorMap &tmWo,
+                                          const Args &a) {
+    using C = Cfg<PAIR>;
+    constexpr int STAGES = C::STAGES;
+    constexpr int STAGE_BYTES = C::STAGE_BYTES;
+    constexpr int A_BYTES = C::A_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -102,8 +178,13 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     float *sl_scb = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + SL_W_BYTES);
     float *sl_bias = sl_scb + BN;
     float *sl_xo = sl_bias + BN;
-    Tail *tail = reinterpret_cast<Tail *>(smem + STAGES * STAGE_BYTES + SL_BYTES);
+    Tail<STAGES> *tail = reinterpret_cast<Tail<STAGES> *>(smem + STAGES * STAGE_BYTES + SL_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the pair: rank 0 is the leader; tiles are numbered per pair
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     // Prologue: nothing here reads global memory that the kernels before this one write, so
     // it overlaps their tail (this grid is their programmatic dependent).
@@ -114,11 +195,14 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&tail->acc_full[s]), 1);
-            mbar_init(smem_addr(&tail->acc_empty[s]), 4);
+            // the epilogue warps of this CTA (and of the second CTA of a pair) release it
+            mbar_init(smem_addr(&tail->acc_empty[s]), PAIR ? 8 : 4);
         }
         mbar_init(smem_addr(&tail->mma_done), 1);
         mbar_init(smem_addr(&tail->slice_full), 4);
         mbar_init(smem_addr(&tail->slice_empty), 4);
+        mbar_init(smem_addr(&tail->loads_drained), 1);
+        mbar_init(smem_addr(&tail->peer_exit), 1);
         tail->abort_flag = 0;
         fence_mbar_init();
     }
@@ -130,7 +214,12 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tma_prefetch_desc(&tmWo);
         }
     }
-    if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), TMEM_COLS);
+    if (warp == 1) {
+        if (PAIR) tmem_alloc_pair(smem_addr(&tail->tmem_base), TMEM_COLS);
+        else tmem_alloc(smem_addr(&tail->tmem_base), TMEM_COLS);
+    }
+    // a pair's barriers are initialized in both CTAs before either may use the other's
+    if (PAIR) cluster_barrier_all();
     // the quantized operands, scales and outlier list of this call are complete after this
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -156,22 +245,35 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             int stage = 0;
             uint32_t phase = 0;
             uint32_t used = 0, last_parity = 0;   // per stage: issued at least once / parity
-            for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-                const int m0 = (tile % a.tiles_m) * BM;
-                const int n0 = (tile / a.tiles_m) * BN;
+            for (int tile = unit; tile < total_tiles; tile += units) {
+                // this CTA's rows of X and of the weight tile
+                const int m0 = (tile % a.tiles_m) * C::TILE_M + (int)rank * BM;
+                const int n0 = (tile / a.tiles_m) * BN + (int)rank * C::B_ROWS;
                 for (int kb = 0; kb < nkb + nob; ++kb) {
                     if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
                     const uint32_t full = smem_addr(&tail->full[stage]);
                     const uint32_t sa = smem_addr(smem + stage * STAGE_BYTES);
-                    mbar_arrive_expect_tx(full, STAGE_BYTES);
+                    if (!PAIR || leader)   // the leader's barrier counts the bytes of both CTAs
+                        mbar_arrive_expect_tx(full, PAIR ? 2 * STAGE_BYTES : STAGE_BYTES);
+                    const uint32_t fbar = PAIR ? map_to_rank(full, 0) : full;
                     if (kb < nkb) {
                         const int kr = rotated_kblock(kb, tile / a.tiles_m, nkb);
-                        tma_load_2d(sa, &tmA, kr * BKB, m0, full);
-                        tma_load_2d(sa + A_BYTES, &tmB, kr * BKB, n0, full);
+                        if (PAIR) {
+                            tma_load_2d_pair(sa, &tmA, kr * BKB, m0, fbar);
+                            tma_load_2d_pair(sa + A_BYTES, &tmB, kr * BKB, n0, fbar);
+                        } else {
+                            tma_load_2d(sa, &tmA, kr * BKB, m0, full);
+                            tma_load_2d(sa + A_BYTES, &tmB, kr * BKB, n0, full);
+                        }
                     } else {
                         const int x = (kb - nkb) * (BKB / 2);
-                        tma_load_2d(sa, &tmXo, x, m0, full);
-                        tma_load_2d(sa + A_BYTES, &tmWo, x, n0, full);
+                        if (PAIR) {
+                            tma_load_2d_pair(sa, &tmXo, x, m0, fbar);
+                            tma_load_2d_pair(sa + A_BYTES, &tmWo, x, n0, fbar);
+                        } else {
+                            tma_load_2d(sa, &tmXo, x, m0, full);
+                            tma_load_2d(sa + A_BYTES, &tmWo, x, n0, full);
+                        }
                     }
                     used |= 1u << stage;
                     last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -182,21 +284,25 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
             }
         drain:
-            // wait for every copy this thread issued to land before the CTA may exit
-            for (int s = 0; s < STAGES; ++s)
-                if (used & (1u << s))
-                    drain_wait(smem_addr(&tail->full[s]), (last_parity >> s) & 1u, a.status);
+            // wait for every copy this thread issued to land before the CTA may exit (a pair's
+            // leader waits for the copies of both CTAs, then tells the second CTA)
+            if (!PAIR || leader) {
+                for (int s = 0; s < STAGES; ++s)
+                    if (used & (1u << s))
+                        drain_wait(smem_addr(&tail->full[s]), (last_parity >> s) & 1u, a.status);
+                if (PAIR) mbar_arrive_cluster(map_to_rank(smem_addr(&tail->loads_drained), 1));
+            }
         }
     } else if (warp == 1) {
         // --------------------------------------------------------------- MMA issuer ----
-        if (lane == 0) {
-            const uint32_t id_i8 = idesc_i8(BM, BN);
-            const uint32_t id_f16 = idesc_f16(BM, BN);
+        if (lane == 0 && (!PAIR || leader)) {
+            const uint32_t id_i8 = idesc_i8(C::TILE_M, BN);
+            const uint32_t id_f16 = idesc_f16(C::TILE_M, BN);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+            for (int tile = unit; tile < total_tiles; tile += units) {
                 if (!wait(smem_addr(&tail->acc_empty[acc]), acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_i32 = tmem + (uint32_t)(acc * 256);
@@ -212,30 +318,50 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const uint32_t sb = sa + A_BYTES;
                     if (kb < nkb) {
 #pragma unroll
-                        for (int k = 0; k < BKB / 32; ++k)
-                            mma_i8(d_i32, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), id_i8,
-                                   (kb | k) != 0);
+                        for (int k = 0; k < BKB / 32; ++k) {
+                            if (PAIR)
+                                mma_i8_pair(d_i32, sw128_desc(sa + 32 * k),
+                                            sw128_desc(sb + 32 * k), id_i8, (kb | k) != 0);
+                            else
+                                mma_i8(d_i32, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k),
+                                       id_i8, (kb | k) != 0);
+                        }
                     } else {
 #pragma unroll
-                        for (int k = 0; k < BKB / 32; ++k)
-                            mma_f16(d_f32, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k),
-                                    id_f16, ((kb - nkb) | k) != 0);
+                        for (int k = 0; k < BKB / 32; ++k) {
+                            if (PAIR)
+                                mma_f16_pair(d_f32, sw128_desc(sa + 32 * k),
+                                             sw128_desc(sb + 32 * k), id_f16,
+                                             ((kb - nkb) | k) != 0);
+                            else
+                                mma_f16(d_f32, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k),
+                                        id_f16, ((kb - nkb) | k) != 0);
+                        }
                     }
-                    tc_commit(smem_addr(&tail->empty[stage]));   // frees the stage
+                    // frees the stage (in both CTAs of a pair)
+                    if (PAIR) tc_commit_pair_both(smem_addr(&tail->empty[stage]));
+                    else tc_commit(smem_addr(&tail->empty[stage]));
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
                 if (!ok) break;
-                tc_commit(smem_addr(&tail->acc_full[acc]));      // accumulators ready
+                // accumulators ready (in both CTAs of a pair)
+                if (PAIR) tc_commit_pair_both(smem_addr(&tail->acc_full[acc]));
+                else tc_commit(smem_addr(&tail->acc_full[acc]));
                 if (++acc == acc_stages) {
                     acc = 0;
                     acc_phase ^= 1;
                 }
             }
             // every MMA issued by this thread has completed once mma_done arrives
-            tc_commit(smem_addr(&tail->mma_done));
+            if (PAIR) tc_commit_pair_both(smem_addr(&tail->mma_done));
+            else tc_commit(smem_addr(&tail->mma_done));
+            drain_wait(smem_addr(&tail->mma_done), 0, a.status);
+        } else if (lane == 0) {
+            // second CTA of a pair: its TMEM and shared memory are the leader's MMA operands
+            // until the leader's last MMA has completed
             drain_wait(smem_addr(&tail->mma_done), 0, a.status);
         }
     } else {
@@ -246,8 +372,8 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         int acc = 0;
         uint32_t acc_phase = 0, sl_phase = 0;
         bool first = true;
-        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-            const int m0 = (tile % a.tiles_m) * BM;
+        for (int tile = unit; tile < total_tiles; tile += units) {
+            const int m0 = (tile % a.tiles_m) * C::TILE_M + (int)rank * BM;   // this CTA's rows
             const int n0 = (tile / a.tiles_m) * BN;
             // The tile's column slice (SCB, bias and, with few outlier columns, Wo), staged
             // while the tensor cores still work on the tile: each warp one quarter of it,
@@ -388,7 +514,11 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(smem_addr(&tail->acc_empty[acc]));
+                // the accumulator buffer is free again (the leader's barrier for a pair)
+                if (PAIR && !leader)
+                    mbar_arrive_cluster(map_to_rank(smem_addr(&tail->acc_empty[acc]), 0));
+                else
+                    mbar_arrive(smem_addr(&tail->acc_empty[acc]));
                 mbar_arrive(smem_addr(&tail->slice_empty));
             }
             sl_phase ^= 1;
@@ -401,10 +531,37 @@ llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
+    if (PAIR && threadIdx.x == 0) {
+        if (leader) {
+            // the second CTA has made its last arrive on this CTA's barriers
+            drain_wait(smem_addr(&tail->peer_exit), 0, a.status);
+        } else {
+            // the leader has seen every copy of this CTA land; then release the leader
+            drain_wait(smem_addr(&tail->loads_drained), 0, a.status);
+            mbar_arrive_cluster(map_to_rank(smem_addr(&tail->peer_exit), 0));
+        }
+    }
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        if (PAIR) tmem_dealloc_pair(tmem, TMEM_COLS);
+        else tmem_dealloc(tmem, TMEM_COLS);
     }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmXo,
+                    const __grid_constant__ CUtensorMap tmWo, const Args a) {
+    gemm_body<false>(tmA, tmB, tmXo, tmWo, a);
+}
+
+// M > 128: clusters of two CTAs, 256 x 256 tiles.
+__global__ void __launch_bounds__(THREADS, 1)
+llmint8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmXo,
+                         const __grid_constant__ CUtensorMap tmWo, const Args a) {
+    gemm_body<true>(tmA, tmB, tmXo, tmWo, a);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -441,6 +598,9 @@ struct DeviceInfo {
     bool attr_set = false;
 };
 
+// The CTA-pair kernel takes every call with more than 128 rows of X.
+bool use_pair(int64_t M) { return M > BM; }
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s) {
@@ -458,22 +618,29 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s) {
             err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
             if (err != cudaSuccess) return err;
             err = cudaFuncSetAttribute(llmint8_gemm_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem_bytes<false>());
+            if (err != cudaSuccess) return err;
+            err = cudaFuncSetAttribute(llmint8_gemm_pair_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem_bytes<true>());
             if (err != cudaSuccess) return err;
             d.attr_set = true;
         }
         sms = d.sms;
     }
+    const bool pair = use_pair(g.M);
+    const uint32_t b_rows = pair ? (uint32_t)Cfg<true>::B_ROWS : (uint32_t)Cfg<false>::B_ROWS;
     CUtensorMap tmA, tmB, tmXo, tmWo;
     memset(&tmXo, 0, sizeof(tmXo));
     memset(&tmWo, 0, sizeof(tmWo));
     bool ok = make_map(&tmA, g.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.K, g.M, g.K, BKB, BM) &&
-              make_map(&tmB, g.CB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.K, g.N, g.K, BKB, BN);
+              make_map(&tmB, g.CB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.K, g.N, g.K, BKB, b_rows);
     if (ok && g.cap > 0)
         ok = make_map(&tmXo, g.Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, g.pitch, g.M, g.pitch,
                       BKB / 2, BM) &&
              make_map(&tmWo, g.Wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, g.pitch, g.N, g.pitch,
-                      BKB / 2, BN);
+                      BKB / 2, b_rows);
     if (!ok) return cudaErrorInvalidValue;
     Args a;
     a.Xo = g.Xo;
@@ -491,22 +658,28 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s) {
     a.N = (int)g.N;
     a.K = (int)g.K;
     a.num_kb = (int)ceil_div(g.K, BKB);
-    a.tiles_m = (int)ceil_div(g.M, BM);
+    a.tiles_m = (int)ceil_div(g.M, pair ? 2 * BM : BM);
     a.tiles_n = (int)ceil_div(g.N, BN);
     a.timeout_ns = g.timeout_ns;
     const int tiles = a.tiles_m * a.tiles_n;
-    const int grid = std::min(tiles, sms);
+    // one CTA (or one pair of CTAs) per tile, persistent beyond the SM count
+    const int grid = pair ? 2 * std::min(tiles, sms / 2) : std::min(tiles, sms);
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = (size_t)(pair ? smem_bytes<true>() : smem_bytes<false>());
     cfg.stream = s;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, llmint8_gemm_kernel, tmA, tmB, tmXo, tmWo, a);
+    cfg.numAttrs = pair ? 2 : 1;
+    err = pair ? cudaLaunchKernelEx(&cfg, llmint8_gemm_pair_kernel, tmA, tmB, tmXo, tmWo, a)
+               : cudaLaunchKernelEx(&cfg, llmint8_gemm_kernel, tmA, tmB, tmXo, tmWo, a);
     note_launches(1);
     return err != cudaSuccess ? err : cudaGetLastError();
 }
