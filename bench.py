@@ -376,7 +376,8 @@ def run_ours(args, rank, world, local_rank):
         achieved = step_units * args.steps / kern_s / 1e12
         peak = 2.0 * peaks["bf16_tflops"]           # int8 dense = 2 x bf16 dense (nominal ratio)
         roof_unit = "TOPS"
-        kernel_name = "llmint8_gemm_kernel"
+        kernel_name = ("llmint8_gemm_pair_kernel" if all(c.M > 128 for c in calls)
+                       else "llmint8_gemm_kernel")
         timing = "CUDA events around each GEMM launch, averaged over the timed region"
     result = {
         "metric": "LLM.int8 linear TOPS (prefill) / weight GB/s (decode); fraction of roofline",
