@@ -138,14 +138,15 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t d, uint64_t adesc, uint64_
         : "memory");
 }
 // Arrive on the barrier at `bar` in both CTAs of the pair once the pair's MMAs issued so far
-// by this thread have completed.
+// by this thread have completed: one commit for each CTA's barrier (a commit tracks every
+// earlier tcgen05 operation of the thread, so the two arrive at the same point).
 __device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .b16 m;\n\t"
-        "mov.b16 m, 3;\n\t"
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], m;\n\t}" ::"r"(bar)
-        : "memory");
+#pragma unroll
+    for (uint32_t r = 0; r < 2; ++r)
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                map_to_rank(bar, r))
+            : "memory");
 }
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
