@@ -108,6 +108,11 @@ LLMINT8_API size_t llmint8_quantize_workspace_size(int64_t M, int64_t K);
  *           evaluated in fp32 with int32 C.
  *   ws      device workspace of llmint8_linear_workspace_size(M, N, K, max_outliers) bytes.
  *   C_debug int32 [M, N] or NULL: when given, also receives the exact int8 accumulators C.
+ * Kernels (the results do not depend on the choice): M <= 16, K <= 8192, threshold > 0 and
+ * max_outliers <= 256 run two kernels, a row quantizer and a weight-streaming tcgen05 kernel
+ * launched as its programmatic dependent.  Other shapes run outlier detection, row
+ * quantization (with the gather of the outlier weight rows) and a persistent tcgen05 GEMM,
+ * on CTA pairs when M > 128.
  */
 LLMINT8_API llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
                               const float *SCB, int64_t N, const uint16_t *bias,
@@ -140,7 +145,7 @@ LLMINT8_API llmint8_status llmint8_workspace_outlier_count(const void *ws, void 
 LLMINT8_API const char *llmint8_status_string(llmint8_status status);
 
 /*
- * Upper bound, in nanoseconds, of every wait inside the GEMM kernels of later calls
+ * Upper bound, in nanoseconds, of every wait inside the GEMM and decode kernels of later calls
  * (process-wide; default 1e9).  A wait that runs out records LLMINT8_ERR_TIMEOUT in the
  * device status and the kernel winds down and returns.  Tests set a tiny bound to
  * exercise that path.  ns == 0 restores the default.
@@ -152,7 +157,8 @@ LLMINT8_API llmint8_status llmint8_set_wait_timeout_ns(uint64_t ns);
  * kernel of a call with CUDA events and count launches):
  *   llmint8_set_profile_events(start, stop): two cudaEvent_t.  While both are non-NULL,
  *     every llmint8_linear call records `start` on its stream immediately before its
- *     product kernel (the GEMM) and `stop` immediately after it.  NULL, NULL disables.
+ *     product kernel (the GEMM; on the decode path, the pair of decode kernels) and `stop`
+ *     immediately after it.  NULL, NULL disables.
  *     Process-wide; the caller owns the events and must keep them alive while set.
  *   llmint8_kernel_launch_count(): number of kernels this library has launched in the
  *     process so far.
