@@ -123,6 +123,29 @@ LLMINT8_API llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t 
 LLMINT8_API size_t llmint8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t max_outliers);
 
 /*
+ * llmint8_linear on HOST activations and outputs (a calling convenience with no counterpart
+ * on the pages: the layer itself is llmint8_linear).  On `stream`, in order: copy X_host
+ * [M, K] fp16 into the device buffer X_dev, run llmint8_linear(X_dev -> Y_dev), copy Y_dev
+ * [M, N] fp16 into Y_host.  No C_debug output.
+ *   X_host, Y_host  HOST pointers owned by the caller.  Page-locked (cudaHostAlloc /
+ *                   torch pin_memory) memory keeps the call asynchronous; pageable memory
+ *                   works, but CUDA then copies synchronously.  Y_host holds the output only
+ *                   after the stream has reached the end of the call (synchronize it).
+ *   X_dev, Y_dev    DEVICE buffers of M*K and M*N fp16 values, owned by the caller, 16-byte
+ *                   aligned; they hold X and Y afterwards.
+ *   CB, SCB, bias, W_fp16, threshold, max_outliers, ws, ws_bytes: as for llmint8_linear.
+ * Every argument check of llmint8_linear runs before the first copy, with the same codes;
+ * a NULL host pointer returns LLMINT8_ERR_INVALID_ARG.  A failed copy returns
+ * LLMINT8_ERR_CUDA.  Conditions found on the device go to the workspace's status word.
+ */
+LLMINT8_API llmint8_status llmint8_linear_host(const uint16_t *X_host, int64_t M, int64_t K,
+                                   const int8_t *CB, const float *SCB, int64_t N,
+                                   const uint16_t *bias, const uint16_t *W_fp16,
+                                   float threshold, int64_t max_outliers, uint16_t *Y_host,
+                                   uint16_t *X_dev, uint16_t *Y_dev, void *ws, size_t ws_bytes,
+                                   void *stream);
+
+/*
  * Weight dequantization W_out[n,k] = fp16(fl32(fl32(CB[n,k] * SCB[n]) / 127)) (blog
  * section 用法: the fp16 weights are recovered as (CB * SCB) / 127).
  */

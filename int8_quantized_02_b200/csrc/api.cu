@@ -196,11 +196,16 @@ llmint8_status llmint8_quantize_rows_and_find_outliers(const uint16_t *X, int64_
                                           SCA, nullptr, nullptr, nullptr, nullptr, 0, nullptr, s));
 }
 
-llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
-                              const float *SCB, int64_t N, const uint16_t *bias,
-                              const uint16_t *W_fp16, float threshold, int64_t max_outliers,
-                              uint16_t *Y, void *ws, size_t ws_bytes, void *stream,
-                              int32_t *C_debug) {
+}  // extern "C"
+
+namespace {
+
+// Every check of llmint8_linear that needs no CUDA call, in the order the header lists them.
+llmint8_status check_linear(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
+                            const float *SCB, int64_t N, const uint16_t *bias,
+                            const uint16_t *W_fp16, float threshold, int64_t max_outliers,
+                            const uint16_t *Y, const void *ws, size_t ws_bytes,
+                            const int32_t *C_debug) {
     if (!X || !CB || !SCB || !Y || !ws) return LLMINT8_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(CB) || !aligned16(SCB) || !aligned16(Y) || !aligned16(ws) ||
         (bias && !aligned16(bias)) || (W_fp16 && !aligned16(W_fp16)) ||
@@ -209,8 +214,24 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     if (isnan(threshold)) return LLMINT8_ERR_INVALID_ARG;
     if (!shape_ok_mk(M, K) || !shape_ok_n(N)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
     if (max_outliers < 0 || max_outliers > K) return LLMINT8_ERR_INVALID_ARG;
+    if (ws_bytes < linear_layout(M, N, K, max_outliers).total)
+        return LLMINT8_ERR_WORKSPACE_TOO_SMALL;
+    return LLMINT8_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
+                              const float *SCB, int64_t N, const uint16_t *bias,
+                              const uint16_t *W_fp16, float threshold, int64_t max_outliers,
+                              uint16_t *Y, void *ws, size_t ws_bytes, void *stream,
+                              int32_t *C_debug) {
+    const llmint8_status chk = check_linear(X, M, K, CB, SCB, N, bias, W_fp16, threshold,
+                                            max_outliers, Y, ws, ws_bytes, C_debug);
+    if (chk != LLMINT8_OK) return chk;
     const LinearLayout L = linear_layout(M, N, K, max_outliers);
-    if (ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsHeader *h = at<WsHeader>(ws, 0);
     const StatusRef status = next_status(h);
@@ -283,6 +304,26 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     if (ev1 && record_profile_event(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
     return LLMINT8_OK;
+}
+
+llmint8_status llmint8_linear_host(const uint16_t *X_host, int64_t M, int64_t K,
+                                   const int8_t *CB, const float *SCB, int64_t N,
+                                   const uint16_t *bias, const uint16_t *W_fp16, float threshold,
+                                   int64_t max_outliers, uint16_t *Y_host, uint16_t *X_dev,
+                                   uint16_t *Y_dev, void *ws, size_t ws_bytes, void *stream) {
+    if (!X_host || !Y_host) return LLMINT8_ERR_INVALID_ARG;
+    const llmint8_status chk = check_linear(X_dev, M, K, CB, SCB, N, bias, W_fp16, threshold,
+                                            max_outliers, Y_dev, ws, ws_bytes, nullptr);
+    if (chk != LLMINT8_OK) return chk;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(X_dev, X_host, (size_t)(M * K) * 2, cudaMemcpyHostToDevice, s) !=
+        cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    const llmint8_status st = llmint8_linear(X_dev, M, K, CB, SCB, N, bias, W_fp16, threshold,
+                                             max_outliers, Y_dev, ws, ws_bytes, stream, nullptr);
+    if (st != LLMINT8_OK) return st;
+    return from_cuda(
+        cudaMemcpyAsync(Y_host, Y_dev, (size_t)(M * N) * 2, cudaMemcpyDeviceToHost, s));
 }
 
 llmint8_status llmint8_device_status(const void *ws, void *stream) {

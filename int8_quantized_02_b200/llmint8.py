@@ -45,6 +45,8 @@ PROTOTYPES = {
     "llmint8_kernel_launch_count": (_U64, []),
     "llmint8_linear_noalloc": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _F32, _I64,
                                               _P, _P, ctypes.POINTER(ctypes.c_void_p)]),
+    "llmint8_linear_host": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _F32, _I64, _P,
+                                           _P, _P, _P, _SZ, _P]),
 }
 
 
@@ -99,6 +101,14 @@ def _ptr(t: torch.Tensor | None):
         return None
     if not t.is_cuda:
         raise ValueError("llmint8 tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("llmint8 tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(t: torch.Tensor):
+    if t.is_cuda:
+        raise ValueError("host buffers must be CPU tensors")
     if not t.is_contiguous():
         raise ValueError("llmint8 tensors must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
@@ -244,6 +254,70 @@ class LinearPlan:
         if code != OK:
             raise LLMInt8Error(code, "llmint8_linear")
         return self.Y
+
+
+class LinearHostPlan:
+    """llmint8_linear_host on fixed buffers: host X in, host Y out, marshalled once.
+
+    Each call copies X_host to the device, runs the layer and copies Y back into Y_host, all
+    on the stream; Y_host holds the result once the stream has been synchronized.  Pinned
+    host tensors (``pin_memory()``) keep the call asynchronous.  The device staging buffers
+    and the workspace are allocated here unless given."""
+
+    def __init__(self, X_host: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
+                 Y_host: torch.Tensor | None = None, bias=None, W_fp16=None,
+                 threshold: float = 6.0, max_outliers: int | None = None, X_dev=None,
+                 Y_dev=None, workspace=None, stream=None):
+        M, K = X_host.shape
+        N = CB.shape[0]
+        dev = CB.device
+        _want(X_host, torch.float16, (M, K), "X_host")
+        _want(CB, torch.int8, (N, K), "CB")
+        _want(SCB, torch.float32, (N,), "SCB")
+        if bias is not None:
+            _want(bias, torch.float16, (N,), "bias")
+        if W_fp16 is not None:
+            _want(W_fp16, torch.float16, (N, K), "W_fp16")
+        cap = default_max_outliers(K, threshold) if max_outliers is None else int(max_outliers)
+        self.Y_host = torch.empty((M, N), dtype=torch.float16).pin_memory() \
+            if Y_host is None else Y_host
+        _want(self.Y_host, torch.float16, (M, N), "Y_host")
+        self.X_dev = torch.empty((M, K), dtype=torch.float16, device=dev) if X_dev is None \
+            else X_dev
+        self.Y_dev = torch.empty((M, N), dtype=torch.float16, device=dev) if Y_dev is None \
+            else Y_dev
+        _want(self.X_dev, torch.float16, (M, K), "X_dev")
+        _want(self.Y_dev, torch.float16, (M, N), "Y_dev")
+        if workspace is None:
+            workspace = torch.empty((llmint8_linear_workspace_size(M, N, K, cap),),
+                                    dtype=torch.uint8, device=dev)
+        self.workspace = workspace
+        self._keep = (X_host, CB, SCB, bias, W_fp16)
+        self._fn = load().llmint8_linear_host
+        self._args = (_host_ptr(X_host), M, K, _ptr(CB), _ptr(SCB), N, _ptr(bias),
+                      _ptr(W_fp16), ctypes.c_float(threshold), cap, _host_ptr(self.Y_host),
+                      _ptr(self.X_dev), _ptr(self.Y_dev), _ptr(workspace), workspace.numel(),
+                      _stream(stream))
+
+    def __call__(self) -> torch.Tensor:
+        code = self._fn(*self._args)
+        if code != OK:
+            raise LLMInt8Error(code, "llmint8_linear_host")
+        return self.Y_host
+
+
+def llmint8_linear_host(X_host: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
+                        Y_host=None, bias=None, W_fp16=None, threshold: float = 6.0,
+                        max_outliers: int | None = None, X_dev=None, Y_dev=None, workspace=None,
+                        stream=None, synchronize: bool = True) -> torch.Tensor:
+    """The layer on a host X fp16 [M, K]: Y fp16 [M, N] in host memory (by default the stream
+    is synchronized before returning, so Y is ready)."""
+    plan = LinearHostPlan(X_host, CB, SCB, Y_host, bias, W_fp16, threshold, max_outliers,
+                          X_dev, Y_dev, workspace, stream)
+    Y = plan()
+    if synchronize:
+        (torch.cuda.current_stream() if stream is None else stream).synchronize()
+    return Y
 
 
 def llmint8_dequant(CB: torch.Tensor, SCB: torch.Tensor, out=None, stream=None):

@@ -110,3 +110,28 @@ def test_empty_and_out_of_range_shapes_are_rejected_before_any_launch(lib):
     assert lib.llmint8_quantize_weight_colwise(fake, 0, 1024, fake, fake, None) == \
         llmint8.ERR_UNSUPPORTED_SHAPE
     assert lib.llmint8_dequant(fake, fake, 16, 8, fake, None) == llmint8.ERR_UNSUPPORTED_SHAPE
+
+
+def test_host_entry_checks_run_before_any_copy(lib):
+    # llmint8_linear_host: null host pointers, bad shapes and a short workspace are rejected on
+    # the host with llmint8_linear's codes, before the first copy
+    fake = ctypes.c_void_p(1 << 20)      # aligned, never dereferenced
+    f6 = ctypes.c_float(6.0)
+    assert lib.llmint8_linear_host(None, 16, 1024, fake, fake, 1024, None, None, f6, 0, fake,
+                                   fake, fake, fake, 1 << 30, None) == llmint8.ERR_INVALID_ARG
+    assert lib.llmint8_linear_host(fake, 16, 1024, fake, fake, 1024, None, None, f6, 0, None,
+                                   fake, fake, fake, 1 << 30, None) == llmint8.ERR_INVALID_ARG
+    assert lib.llmint8_linear_host(fake, 16, 1024, fake, fake, 1024, None, None, f6, 0, fake,
+                                   None, fake, fake, 1 << 30, None) == llmint8.ERR_INVALID_ARG
+    assert lib.llmint8_linear_host(fake, 16, 1024, fake, fake, 1024, None, None, f6, 0, fake,
+                                   ctypes.c_void_p((1 << 20) + 8), fake, fake, 1 << 30,
+                                   None) == llmint8.ERR_INVALID_ARG       # X_dev misaligned
+    assert lib.llmint8_linear_host(fake, 16, 1000, fake, fake, 1024, None, None, f6, 0, fake,
+                                   fake, fake, fake, 1 << 30, None) == \
+        llmint8.ERR_UNSUPPORTED_SHAPE
+    assert lib.llmint8_linear_host(fake, 16, 1024, fake, fake, 1024, None, None, f6, 0, fake,
+                                   fake, fake, fake, 256, None) == \
+        llmint8.ERR_WORKSPACE_TOO_SMALL
+    assert lib.llmint8_linear_host(fake, 16, 1024, fake, fake, 1024, None, None,
+                                   ctypes.c_float(float("nan")), 0, fake, fake, fake, fake,
+                                   1 << 30, None) == llmint8.ERR_INVALID_ARG
