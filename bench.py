@@ -181,11 +181,11 @@ class Call:
                                   max_outliers=self.cap, Y=self.Y, workspace=self.ws)
                 for i in range(len(self.CBs))]
 
-    def host_plan(self, X_host, Y_host, X_dev):
-        """Prepared host-buffer calls (llmint8_linear_host), one per weight copy."""
+    def host_plan(self, X_host, Y_host, X_dev, stream):
+        """Prepared host-buffer calls (llmint8_linear_host) on `stream`, one per weight copy."""
         return [self.L.LinearHostPlan(X_host, self.CBs[i], self.SCBs[i], Y_host=Y_host,
                                       threshold=self.t, max_outliers=self.cap, X_dev=X_dev,
-                                      Y_dev=self.Y, workspace=self.ws)
+                                      Y_dev=self.Y, workspace=self.ws, stream=stream)
                 for i in range(len(self.CBs))]
 
     def run(self, plans=None):
@@ -362,26 +362,46 @@ def run_ours(args, rank, world, local_rank):
                                           device="cuda"))
 
     # ---- end to end through the C ABI's host-buffer call: every call copies its X from pinned
-    # host memory, runs the layer and copies Y back into pinned host memory
+    # host memory, runs the layer and copies Y back into pinned host memory.  The calls of a
+    # step share no buffer (own X, Y and workspace), so each runs on a stream of its own and
+    # one call's copies overlap the others' kernels; a call's steps stay in order.
     hosts = [(c.X.cpu().pin_memory(),
               torch.empty((c.M, c.N), dtype=torch.float16).pin_memory()) for c in calls]
     xd = [torch.empty_like(c.X) for c in calls]
-    e2e_plans = [c.host_plan(hosts[j][0], hosts[j][1], xd[j]) for j, c in enumerate(calls)]
+    e2e_streams = [torch.cuda.Stream() for _ in calls]
+    e2e_plans = [c.host_plan(hosts[j][0], hosts[j][1], xd[j], e2e_streams[j])
+                 for j, c in enumerate(calls)]
     e2e_steps = max(1, min(args.steps, 50))
-    for _ in range(2):
-        for j, c in enumerate(calls):
-            c.run(e2e_plans[j])
+
+    def e2e_run(n):
+        start = torch.cuda.Event()
+        start.record(stream)
+        for st in e2e_streams:
+            st.wait_event(start)
+        for _ in range(n):
+            for j, c in enumerate(calls):
+                c.run(e2e_plans[j])
+        for st in e2e_streams:
+            done = torch.cuda.Event()
+            done.record(st)
+            stream.wait_event(done)
+
+    e2e_run(2)
     barrier()
     a0 = torch.cuda.Event(enable_timing=True)
     a1 = torch.cuda.Event(enable_timing=True)
     a0.record(stream)
-    for _ in range(e2e_steps):
-        for j, c in enumerate(calls):
-            c.run(e2e_plans[j])
+    e2e_run(e2e_steps)
     a1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_s = max_over_ranks(a0.elapsed_time(a1) / 1e3, world, device="cuda")
+    for j, c in enumerate(calls):
+        st = L.llmint8_device_status(c.ws)
+        if st != L.OK:
+            raise SystemExit(f"{c.name} (end to end): device status {L.status_string(st)}")
+        if not torch.equal(hosts[j][1], c.Y.cpu()):
+            raise SystemExit(f"{c.name} (end to end): host Y differs from the device Y")
 
     peaks = measured_peaks()
     traffic = profiled_traffic(args.workload)
