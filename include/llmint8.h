@@ -123,6 +123,43 @@ LLMINT8_API llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t 
 LLMINT8_API size_t llmint8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t max_outliers);
 
 /*
+ * Token-parallel (M-split) layers.  When the rows of X are split over ranks, the outlier set
+ * must still be that of the whole X: an outlier column is one where ANY row reaches the
+ * threshold (blog section LLM.int8() 温和总结: outliers are found per feature column of the
+ * whole hidden state), so a rank's own rows do not decide it.  Each rank computes its
+ * rows' bitmap, the ranks exchange the bitmaps (an all-gather of ceil(K/32) words each), and
+ * every rank runs the layer on its rows with the OR of all of them.  The rows it gets are
+ * the same bytes llmint8_linear gives for those rows of the whole X.
+ *
+ * llmint8_outlier_bitmap: bit (j % 32) of bitmap[j / 32] is set iff some row of X [M, K]
+ *   has |X[i, j]| >= threshold (threshold rules as in
+ *   llmint8_quantize_rows_and_find_outliers).  bitmap: uint32 [ceil(K/32)], device, 4-byte
+ *   aligned, fully overwritten.  ws: llmint8_quantize_workspace_size(M, K) bytes; its device
+ *   status is LLMINT8_OK after the call (every column is listed internally, so no capacity
+ *   applies).
+ */
+LLMINT8_API llmint8_status llmint8_outlier_bitmap(const uint16_t *X, int64_t M, int64_t K,
+                                      float threshold, uint32_t *bitmap, void *ws,
+                                      size_t ws_bytes, void *stream);
+
+/*
+ * llmint8_linear_with_bitmaps: llmint8_linear with the outlier set given instead of found:
+ *   O = the columns set in ANY of the n_bitmaps bitmaps [n_bitmaps][ceil(K/32)] (uint32,
+ *   device, 4-byte aligned; 1 <= n_bitmaps <= 65536).  Bits at columns >= K are ignored.
+ *   Every other argument, the workspace (llmint8_linear_workspace_size(M, N, K,
+ *   max_outliers)) and the output are as for llmint8_linear, without a threshold.  The
+ *   call always runs the outlier compaction, the row quantization and the tcgen05 GEMM
+ *   (the decode kernels find the outliers themselves).  More outlier columns than
+ *   max_outliers sets LLMINT8_ERR_OUTLIER_CAPACITY in the device status.
+ */
+LLMINT8_API llmint8_status llmint8_linear_with_bitmaps(const uint16_t *X, int64_t M, int64_t K,
+                                           const int8_t *CB, const float *SCB, int64_t N,
+                                           const uint16_t *bias, const uint16_t *W_fp16,
+                                           const uint32_t *bitmaps, int64_t n_bitmaps,
+                                           int64_t max_outliers, uint16_t *Y, void *ws,
+                                           size_t ws_bytes, void *stream, int32_t *C_debug);
+
+/*
  * llmint8_linear on HOST activations and outputs (a calling convenience with no counterpart
  * on the pages: the layer itself is llmint8_linear).  On `stream`, in order: copy X_host
  * [M, K] fp16 into the device buffer X_dev, run llmint8_linear(X_dev -> Y_dev), copy Y_dev

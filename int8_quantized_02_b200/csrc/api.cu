@@ -68,9 +68,11 @@ LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t cap) {
 
 struct QuantLayout {
     ScanPlan plan;
-    size_t partial = 0, bitmap = 0, total = 0;
+    size_t partial = 0, bitmap = 0, idx = 0, total = 0;
 };
 
+// Workspace of llmint8_quantize_rows_and_find_outliers and llmint8_outlier_bitmap (the
+// latter also lists every outlier column, so the capacity never runs out there).
 QuantLayout quant_layout(int64_t M, int64_t K) {
     QuantLayout L;
     L.plan = scan_plan(M, K);
@@ -79,6 +81,8 @@ QuantLayout quant_layout(int64_t M, int64_t K) {
     off = (size_t)align_up((int64_t)(off + (size_t)(L.plan.splits * L.plan.nwords) * 4), 256);
     L.bitmap = off;
     off = (size_t)align_up((int64_t)(off + (size_t)L.plan.nwords * 4), 256);
+    L.idx = off;
+    off = (size_t)align_up((int64_t)(off + (size_t)K * 4), 256);
     L.total = off;
     return L;
 }
@@ -219,6 +223,34 @@ llmint8_status check_linear(const uint16_t *X, int64_t M, int64_t K, const int8_
     return LLMINT8_OK;
 }
 
+// Arguments of the GEMM launch of a layer call whose workspace `ws` has layout L.
+GemmLaunch gemm_launch(const LinearLayout &L, void *ws, const int8_t *CB, const float *SCB,
+                       const uint16_t *bias, uint16_t *Y, int32_t *C_debug, StatusRef status,
+                       int64_t M, int64_t N, int64_t K, int64_t max_outliers) {
+    GemmLaunch g;
+    g.Xq = at<int8_t>(ws, L.xq);
+    g.CB = CB;
+    g.Xo = at<__half>(ws, L.xo);
+    g.Wo = at<__half>(ws, L.wo);
+    g.pitch = L.pitch;
+    g.count = &at<WsHeader>(ws, 0)->n_outliers;
+    g.cap = max_outliers;
+    g.SCA = at<float>(ws, L.sca);
+    g.SCB = SCB;
+    g.bias = reinterpret_cast<const __half *>(bias);
+    g.Y = reinterpret_cast<__half *>(Y);
+    g.C_debug = C_debug;
+    g.status = status;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.timeout_ns = g_timeout_ns.load();
+    return g;
+}
+
+// Upper bound of the bitmaps one llmint8_linear_with_bitmaps call merges (ranks).
+constexpr int64_t kMaxBitmaps = 65536;
+
 }  // namespace
 
 extern "C" {
@@ -281,29 +313,63 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
                              reinterpret_cast<const __half *>(W_fp16), N,
                              max_outliers > 0 ? Wo : nullptr, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-    GemmLaunch g;
-    g.Xq = Xq;
-    g.CB = CB;
-    g.Xo = Xo;
-    g.Wo = Wo;
-    g.pitch = L.pitch;
-    g.count = &h->n_outliers;
-    g.cap = max_outliers;
-    g.SCA = SCA;
-    g.SCB = SCB;
-    g.bias = reinterpret_cast<const __half *>(bias);
-    g.Y = reinterpret_cast<__half *>(Y);
-    g.C_debug = C_debug;
-    g.status = status;
-    g.M = M;
-    g.N = N;
-    g.K = K;
-    g.timeout_ns = g_timeout_ns.load();
+    const GemmLaunch g = gemm_launch(L, ws, CB, SCB, bias, Y, C_debug, status, M, N, K,
+                                     max_outliers);
     if (ev0 && record_profile_event(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
     e = launch_gemm(g, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     if (ev1 && record_profile_event(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
     return LLMINT8_OK;
+}
+
+llmint8_status llmint8_outlier_bitmap(const uint16_t *X, int64_t M, int64_t K, float threshold,
+                                     uint32_t *bitmap, void *ws, size_t ws_bytes, void *stream) {
+    if (!X || !bitmap || !ws) return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned4(bitmap) || !aligned16(ws)) return LLMINT8_ERR_INVALID_ARG;
+    if (isnan(threshold)) return LLMINT8_ERR_INVALID_ARG;
+    if (!shape_ok_mk(M, K)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    const QuantLayout L = quant_layout(M, K);
+    if (ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE_TOO_SMALL;
+    WsHeader *h = at<WsHeader>(ws, 0);
+    return from_cuda(launch_outlier_detect(reinterpret_cast<const __half *>(X), M, K, threshold,
+                                           L.plan, at<uint32_t>(ws, L.partial), bitmap,
+                                           at<int32_t>(ws, L.idx), K, &h->n_outliers,
+                                           next_status(h), static_cast<cudaStream_t>(stream)));
+}
+
+llmint8_status llmint8_linear_with_bitmaps(const uint16_t *X, int64_t M, int64_t K,
+                                           const int8_t *CB, const float *SCB, int64_t N,
+                                           const uint16_t *bias, const uint16_t *W_fp16,
+                                           const uint32_t *bitmaps, int64_t n_bitmaps,
+                                           int64_t max_outliers, uint16_t *Y, void *ws,
+                                           size_t ws_bytes, void *stream, int32_t *C_debug) {
+    if (!bitmaps || !aligned4(bitmaps)) return LLMINT8_ERR_INVALID_ARG;
+    if (n_bitmaps < 1 || n_bitmaps > kMaxBitmaps) return LLMINT8_ERR_INVALID_ARG;
+    // the threshold plays no part: 6 only satisfies the shared checks
+    const llmint8_status chk = check_linear(X, M, K, CB, SCB, N, bias, W_fp16, 6.0f,
+                                            max_outliers, Y, ws, ws_bytes, C_debug);
+    if (chk != LLMINT8_OK) return chk;
+    const LinearLayout L = linear_layout(M, N, K, max_outliers);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    WsHeader *h = at<WsHeader>(ws, 0);
+    const __half *Xh = reinterpret_cast<const __half *>(X);
+    uint32_t *bitmap = at<uint32_t>(ws, L.bitmap);
+    int32_t *idx = at<int32_t>(ws, L.idx);
+    __half *Xo = at<__half>(ws, L.xo);
+    __half *Wo = at<__half>(ws, L.wo);
+    const StatusRef status = next_status(h);
+    cudaError_t e = launch_outlier_merge(bitmaps, n_bitmaps, K, bitmap, idx, max_outliers,
+                                         &h->n_outliers, status, s);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    e = launch_quantize_rows(Xh, M, K, bitmap, idx, &h->n_outliers, max_outliers, L.pitch,
+                             at<int8_t>(ws, L.xq), at<float>(ws, L.sca),
+                             max_outliers > 0 ? Xo : nullptr, CB, SCB,
+                             reinterpret_cast<const __half *>(W_fp16), N,
+                             max_outliers > 0 ? Wo : nullptr, s);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    return from_cuda(launch_gemm(gemm_launch(L, ws, CB, SCB, bias, Y, C_debug, status, M, N, K,
+                                             max_outliers),
+                                 s));
 }
 
 llmint8_status llmint8_linear_host(const uint16_t *X_host, int64_t M, int64_t K,

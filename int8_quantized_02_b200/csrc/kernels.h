@@ -26,6 +26,11 @@ cudaError_t launch_outlier_detect(const __half *X, int64_t M, int64_t K, float t
                                   const ScanPlan &plan, uint32_t *partial, uint32_t *bitmap,
                                   int32_t *idx, int64_t cap, int32_t *count, StatusRef status,
                                   cudaStream_t s);
+// The outlier set as the OR of n_bitmaps caller-supplied column bitmaps [n][ceil(K/32)]
+// (bits at columns >= K ignored): merged bitmap, ascending list (first cap), count, status.
+cudaError_t launch_outlier_merge(const uint32_t *bitmaps, int64_t n_bitmaps, int64_t K,
+                                 uint32_t *bitmap, int32_t *idx, int64_t cap, int32_t *count,
+                                 StatusRef status, cudaStream_t s);
 // Row quantization of X (and, with Wo non-null, the gather of the outlier weights Wo
 // [N, xo_pitch] from CB/SCB or W16, in the same launch).  The scan, compaction and this
 // kernel are programmatic dependents of whatever precedes them in the stream.

@@ -118,14 +118,17 @@ outlier_scan_kernel(const __half *__restrict__ X, int64_t M, int64_t K, float th
 // One CTA of 1024 threads: OR over the row splits, popcount, exclusive scan, ascending
 // index list.  Also writes the workspace status word (resetting it for this call).  The OR
 // over the splits is spread over every thread: thread t takes word t % nwords' share of
-// the splits when nwords < 1024, and the shares meet in shared memory.
+// the splits when nwords < 1024, and the shares meet in shared memory.  The "splits" may
+// also be caller-supplied bitmaps (one per row block of a token-parallel layer): bits at
+// columns >= K are dropped, so no index past the last column comes out.
 constexpr int kCompactThreads = 1024;
 constexpr int kMaxWordsPerThread = 4;   // nwords <= 4096 (K <= 131072)
 
 __global__ void __launch_bounds__(kCompactThreads)
 outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t nwords,
-                       int32_t *__restrict__ idx, int64_t cap, int32_t *__restrict__ count_out,
-                       uint32_t *__restrict__ bitmap_out, StatusRef status) {
+                       int64_t K, int32_t *__restrict__ idx, int64_t cap,
+                       int32_t *__restrict__ count_out, uint32_t *__restrict__ bitmap_out,
+                       StatusRef status) {
     pdl_wait_then_release();
     __shared__ int warp_tot[32];
     __shared__ uint32_t merged[kCompactThreads];
@@ -172,6 +175,7 @@ outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t
             } else {
                 for (int sp = 0; sp < splits; ++sp) v |= partial[(int64_t)sp * nwords + wi];
             }
+            if (wi == nwords - 1 && (K & 31) != 0) v &= (1u << (K & 31)) - 1u;
             w[i] = v;
             bitmap_out[wi] = v;
             cnt += __popc(v);
@@ -442,8 +446,18 @@ cudaError_t launch_outlier_detect(const __half *X, int64_t M, int64_t K, float t
     note_launches(1);
     if (e != cudaSuccess) return e;
     e = launch_pdl(outlier_compact_kernel, dim3(1), dim3(kCompactThreads), s,
-                   (const uint32_t *)partial, (int)plan.splits, plan.nwords, idx, cap, count,
+                   (const uint32_t *)partial, (int)plan.splits, plan.nwords, K, idx, cap, count,
                    bitmap, status);
+    note_launches(1);
+    return e;
+}
+
+cudaError_t launch_outlier_merge(const uint32_t *bitmaps, int64_t n_bitmaps, int64_t K,
+                                 uint32_t *bitmap, int32_t *idx, int64_t cap, int32_t *count,
+                                 StatusRef status, cudaStream_t s) {
+    const cudaError_t e = launch_pdl(outlier_compact_kernel, dim3(1), dim3(kCompactThreads), s,
+                                     bitmaps, (int)n_bitmaps, ceil_div(K, 32), K, idx, cap,
+                                     count, bitmap, status);
     note_launches(1);
     return e;
 }

@@ -47,6 +47,9 @@ PROTOTYPES = {
                                               _P, _P, ctypes.POINTER(ctypes.c_void_p)]),
     "llmint8_linear_host": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _F32, _I64, _P,
                                            _P, _P, _P, _SZ, _P]),
+    "llmint8_outlier_bitmap": (ctypes.c_int, [_P, _I64, _I64, _F32, _P, _P, _SZ, _P]),
+    "llmint8_linear_with_bitmaps": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _P, _I64,
+                                                   _I64, _P, _P, _SZ, _P, _P]),
 }
 
 
@@ -254,6 +257,62 @@ class LinearPlan:
         if code != OK:
             raise LLMInt8Error(code, "llmint8_linear")
         return self.Y
+
+
+def bitmap_words(K: int) -> int:
+    """uint32 words of an outlier-column bitmap over K columns."""
+    return (K + 31) // 32
+
+
+def llmint8_outlier_bitmap(X: torch.Tensor, threshold: float = 6.0, bitmap=None,
+                           workspace=None, stream=None) -> torch.Tensor:
+    """X fp16 [M, K] -> int32 [ceil(K/32)] bitmap of its outlier columns (bit j % 32 of word
+    j // 32; the words are uint32 bit patterns held in an int32 tensor)."""
+    M, K = X.shape
+    _want(X, torch.float16, (M, K), "X")
+    W = bitmap_words(K)
+    bitmap = torch.empty((W,), dtype=torch.int32, device=X.device) if bitmap is None else bitmap
+    _want(bitmap, torch.int32, (W,), "bitmap")
+    need = llmint8_quantize_workspace_size(M, K)
+    ws = torch.empty((need,), dtype=torch.uint8, device=X.device) if workspace is None \
+        else workspace
+    _check(load().llmint8_outlier_bitmap(_ptr(X), M, K, ctypes.c_float(threshold), _ptr(bitmap),
+                                         _ptr(ws), ws.numel(), _stream(stream)),
+           "llmint8_outlier_bitmap")
+    return bitmap
+
+
+def llmint8_linear_with_bitmaps(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
+                                bitmaps: torch.Tensor, bias=None, W_fp16=None,
+                                max_outliers: int | None = None, Y=None, workspace=None,
+                                C_debug=None, stream=None) -> torch.Tensor:
+    """The layer with the outlier set given as the OR of `bitmaps` int32 [n, ceil(K/32)]
+    (one row per rank of a token-parallel layer)."""
+    M, K = X.shape
+    N = CB.shape[0]
+    _want(X, torch.float16, (M, K), "X")
+    _want(CB, torch.int8, (N, K), "CB")
+    _want(SCB, torch.float32, (N,), "SCB")
+    if bitmaps.dim() == 1:
+        bitmaps = bitmaps.view(1, -1)
+    _want(bitmaps, torch.int32, (bitmaps.shape[0], bitmap_words(K)), "bitmaps")
+    if bias is not None:
+        _want(bias, torch.float16, (N,), "bias")
+    if W_fp16 is not None:
+        _want(W_fp16, torch.float16, (N, K), "W_fp16")
+    if C_debug is not None:
+        _want(C_debug, torch.int32, (M, N), "C_debug")
+    cap = min(K, 512) if max_outliers is None else int(max_outliers)
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    _want(Y, torch.float16, (M, N), "Y")
+    if workspace is None:
+        workspace = torch.empty((llmint8_linear_workspace_size(M, N, K, cap),), dtype=torch.uint8,
+                                device=X.device)
+    _check(load().llmint8_linear_with_bitmaps(
+        _ptr(X), M, K, _ptr(CB), _ptr(SCB), N, _ptr(bias), _ptr(W_fp16), _ptr(bitmaps),
+        bitmaps.shape[0], cap, _ptr(Y), _ptr(workspace), workspace.numel(), _stream(stream),
+        _ptr(C_debug)), "llmint8_linear_with_bitmaps")
+    return Y
 
 
 class LinearHostPlan:

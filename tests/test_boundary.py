@@ -135,3 +135,32 @@ def test_host_entry_checks_run_before_any_copy(lib):
     assert lib.llmint8_linear_host(fake, 16, 1024, fake, fake, 1024, None, None,
                                    ctypes.c_float(float("nan")), 0, fake, fake, fake, fake,
                                    1 << 30, None) == llmint8.ERR_INVALID_ARG
+
+
+def test_token_parallel_entries_check_arguments_before_any_launch(lib):
+    fake = ctypes.c_void_p(1 << 20)      # aligned, never dereferenced
+    f6 = ctypes.c_float(6.0)
+    ob = lib.llmint8_outlier_bitmap
+    assert ob(None, 16, 1024, f6, fake, fake, 1 << 30, None) == llmint8.ERR_INVALID_ARG
+    assert ob(fake, 16, 1024, f6, None, fake, 1 << 30, None) == llmint8.ERR_INVALID_ARG
+    assert ob(fake, 16, 1024, ctypes.c_float(float("nan")), fake, fake, 1 << 30, None) == \
+        llmint8.ERR_INVALID_ARG
+    assert ob(fake, 16, 1000, f6, fake, fake, 1 << 30, None) == llmint8.ERR_UNSUPPORTED_SHAPE
+    assert ob(fake, 0, 1024, f6, fake, fake, 1 << 30, None) == llmint8.ERR_UNSUPPORTED_SHAPE
+    assert ob(fake, 16, 1024, f6, fake, fake, 64, None) == llmint8.ERR_WORKSPACE_TOO_SMALL
+    # the bitmap call's workspace also lists every column: at least 4 K bytes
+    assert llmint8.llmint8_quantize_workspace_size(16, 1024) >= 4 * 1024
+
+    wb = lib.llmint8_linear_with_bitmaps
+
+    def call(bitmaps=fake, n=1, K=1024, N=1024, ws_bytes=1 << 30, cap=0):
+        return wb(fake, 16, K, fake, fake, N, None, None, bitmaps, n, cap, fake, fake,
+                  ws_bytes, None, None)
+    assert call(bitmaps=None) == llmint8.ERR_INVALID_ARG
+    assert call(bitmaps=ctypes.c_void_p((1 << 20) + 2)) == llmint8.ERR_INVALID_ARG
+    assert call(n=0) == llmint8.ERR_INVALID_ARG
+    assert call(n=65537) == llmint8.ERR_INVALID_ARG
+    assert call(K=1000) == llmint8.ERR_UNSUPPORTED_SHAPE
+    assert call(N=1000) == llmint8.ERR_UNSUPPORTED_SHAPE
+    assert call(cap=2048) == llmint8.ERR_INVALID_ARG
+    assert call(ws_bytes=256) == llmint8.ERR_WORKSPACE_TOO_SMALL
