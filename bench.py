@@ -23,12 +23,9 @@ import json
 import os
 import re
 import statistics
-import subprocess
 import sys
 import threading
 import time
-
-import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
