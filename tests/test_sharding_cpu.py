@@ -124,3 +124,73 @@ def test_token_and_column_exchanges_on_two_gloo_ranks():
         assert set(own) <= set(whole)
         assert y_equal and y_shape == (12, 48)  # gathered columns = the unsplit layer
     assert own0 == [15, 39] and own1 == [39, 49, 79] and results[0][3] == [15, 39, 49, 79]
+
+
+def _token_worker(rank, world, port, q):
+    """token_parallel_linear end to end on CPU ranks.  The two library calls are replaced, in
+    this process only, by stand-ins built on the oracle: the bitmap of the rank's own rows,
+    and the unsplit layer's rows once the gathered bitmaps are checked to OR to the whole
+    X's outlier set."""
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from int8_quantized_02_b200 import sharding as S
+    from int8_quantized_02_b200 import synth
+    from oracle import oracle
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        M, K, N = 2, 48, 32                      # three ranks, two rows: rank 2 has none
+        X, _ = synth.activations(M, K, 0, seed=21)
+        X[0, 40] = np.float16(8.0)
+        X[1, 3] = np.float16(-6.0)
+        W = synth.weight(N, K, 0.02, seed=22)
+        CB, SCB = oracle.quantize_weight_colwise(W)
+        _, _, whole = oracle.quantize_rows_and_find_outliers(X, 6.0)
+        m0, m1 = S.row_range(M, world, rank)
+        seen = {}
+
+        def bitmap_of(X_local, threshold):
+            _, _, own = oracle.quantize_rows_and_find_outliers(X_local.numpy(), threshold)
+            seen["bitmap_calls"] = seen.get("bitmap_calls", 0) + 1
+            return torch.from_numpy(_bitmap(own, K).copy())
+
+        def layer_with(X_local, CB_t, SCB_t, bitmaps, bias=None, W_fp16=None,
+                       max_outliers=None):
+            union = np.bitwise_or.reduce(bitmaps.numpy().view(np.uint32), axis=0)
+            seen["union"] = _set_of(union)
+            seen["n_bitmaps"] = bitmaps.shape[0]
+            return torch.from_numpy(oracle.linear(X, CB, SCB)[m0:m1].copy())
+
+        S.L.llmint8_outlier_bitmap = bitmap_of
+        S.L.llmint8_linear_with_bitmaps = layer_with
+        Y = S.token_parallel_linear(torch.from_numpy(X[m0:m1].copy()), torch.from_numpy(CB),
+                                    torch.from_numpy(SCB))
+        q.put((rank, tuple(Y.shape), seen.get("bitmap_calls", 0), seen.get("union"),
+               seen.get("n_bitmaps"), list(map(int, whole))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_token_parallel_linear_on_three_gloo_ranks_with_an_empty_rank():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_token_worker, args=(r, 3, port, q)) for r in range(3)]
+    for p in procs:
+        p.start()
+    try:
+        results = sorted(q.get(timeout=120) for _ in range(3))
+    finally:
+        for p in procs:
+            p.join(60)
+    assert [p.exitcode for p in procs] == [0, 0, 0]
+    whole = results[0][5]
+    assert whole == [3, 40]
+    for rank, shape, bitmap_calls, union, n_bitmaps, _ in results[:2]:
+        assert shape == (1, 32) and bitmap_calls == 1
+        assert union == whole and n_bitmaps == 3
+    rank, shape, bitmap_calls, union, n_bitmaps, _ = results[2]
+    assert shape == (0, 32) and bitmap_calls == 0 and union is None   # joined the exchange only
