@@ -56,8 +56,9 @@ typedef enum {
 } llmint8_status;
 
 /*
- * Weight quantization, once per layer ("weights are quantized by column" of the logical
- * K x N weight = per output channel; blog section MatMul 内部; CB / SCB of section 用法).
+ * Weight quantization, once per layer.  The blog quantizes the weight per column of the
+ * logical K x N weight, i.e. per output channel (section MatMul 内部); CB and SCB are the
+ * names of section 用法.
  *   W   fp16 [N, K]  input, nn.Linear layout (row n = output channel n).
  *   CB  int8 [N, K]  output: CB[n,k] = round_half_even(fl32(W[n,k] * fl32(127 / SCB[n]))).
  *   SCB fp32 [N]     output: SCB[n] = max_k |W[n,k]| (0 gives an all-zero row).

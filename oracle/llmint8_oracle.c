@@ -120,7 +120,8 @@ static int8_t absmax_quantize(float x, float s)
 
 /* W fp16 [N, K] row-major (row n = output channel n, K contiguous).
    SCB[n] = max_k |W[n, k]|;  CB[n, k] = q(W[n, k], fl32(127 / SCB[n])).
-   ("weights are quantized by column" of the logical K x N weight = per output channel.) */
+   (The blog quantizes the weight per column of the logical K x N weight, which is per
+   output channel: per row of CB.) */
 int oracle_quantize_weight_colwise(const uint16_t *W, int64_t N, int64_t K,
                                    int8_t *CB, float *SCB)
 {
