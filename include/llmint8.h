@@ -202,6 +202,27 @@ LLMINT8_API llmint8_status llmint8_device_status(const void *ws, void *stream);
 /* Also returns the device outlier count of a llmint8_linear workspace (synchronizes). */
 LLMINT8_API llmint8_status llmint8_workspace_outlier_count(const void *ws, void *stream, int32_t *count);
 
+/*
+ * Read-back of the fp16 outlier-weight rows W_o that the last llmint8_linear or
+ * llmint8_linear_with_bitmaps call on `ws` multiplied X's outlier columns with (blog section
+ * 用法: the fp16 weights are recovered as (CB * SCB) / 127; with W_fp16 given, the original
+ * fp16 weights): W_o[n, j] = fp16(fl32(fl32(CB[n, O_j] * SCB[n]) / 127)), or W_fp16[n, O_j],
+ * for the outlier columns O_0 < O_1 < ... of that call.  It lets a test compare this step of
+ * the layer bit for bit.
+ *   ws            the workspace of that call.
+ *   M, N, K, max_outliers  that call's arguments (they fix where W_o lies in the workspace).
+ *   Wo            DEVICE fp16 [N, n_cols], row-major, 16-byte aligned, owned by the caller.
+ *   n_cols        0 <= n_cols <= max_outliers; columns past that call's outlier count hold 0.
+ * The GEMM path keeps W_o in the workspace on every call.  The decode path forms it in
+ * registers and stores it into the workspace only when the call was given C_debug; after a
+ * decode-path call without C_debug the result is undefined.  Asynchronous on `stream` (one
+ * device-to-device copy); LLMINT8_ERR_INVALID_ARG for a bad pointer or n_cols,
+ * LLMINT8_ERR_UNSUPPORTED_SHAPE for shapes llmint8_linear rejects.
+ */
+LLMINT8_API llmint8_status llmint8_workspace_outlier_weights(const void *ws, int64_t M, int64_t N,
+                                                 int64_t K, int64_t max_outliers,
+                                                 uint16_t *Wo, int64_t n_cols, void *stream);
+
 /* Static English text for a status code. */
 LLMINT8_API const char *llmint8_status_string(llmint8_status status);
 

@@ -282,6 +282,8 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
         d.Y = reinterpret_cast<__half *>(Y);
         d.C_debug = C_debug;
         d.count = &h->n_outliers;
+        d.Wo = C_debug ? at<__half>(ws, L.wo) : nullptr;
+        d.wo_pitch = L.pitch;
         d.image = at<uint8_t>(ws, L.dimage);
         d.tables = at<DecodeTables>(ws, L.dtables);
         d.status = status;
@@ -414,6 +416,22 @@ llmint8_status llmint8_workspace_outlier_count(const void *ws, void *stream, int
     return LLMINT8_OK;
 }
 
+llmint8_status llmint8_workspace_outlier_weights(const void *ws, int64_t M, int64_t N, int64_t K,
+                                                 int64_t max_outliers, uint16_t *Wo,
+                                                 int64_t n_cols, void *stream) {
+    if (!ws || !Wo || !aligned16(ws) || !aligned16(Wo)) return LLMINT8_ERR_INVALID_ARG;
+    if (!shape_ok_mk(M, K) || !shape_ok_n(N)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    if (max_outliers < 0 || max_outliers > K || n_cols < 0 || n_cols > max_outliers)
+        return LLMINT8_ERR_INVALID_ARG;
+    if (n_cols == 0) return LLMINT8_OK;
+    const LinearLayout L = linear_layout(M, N, K, max_outliers);
+    return from_cuda(cudaMemcpy2DAsync(Wo, (size_t)n_cols * 2,
+                                       static_cast<const uint8_t *>(ws) + L.wo,
+                                       (size_t)L.pitch * 2, (size_t)n_cols * 2, (size_t)N,
+                                       cudaMemcpyDeviceToDevice,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
 
 // ------------------------------------------------------------------ no-allocation call ----
@@ -505,6 +523,8 @@ llmint8_status llmint8_linear_noalloc(const uint16_t *X, int64_t M, int64_t K, c
     d.bias = reinterpret_cast<const __half *>(bias);
     d.Y = reinterpret_cast<__half *>(Y);
     d.C_debug = nullptr;
+    d.Wo = nullptr;
+    d.wo_pitch = 0;
     d.count = &h->n_outliers;
     d.image = at<uint8_t>(base, image);
     d.tables = at<DecodeTables>(base, tables);

@@ -307,6 +307,8 @@ struct DArgs {
     const __half *bias;
     __half *Y;
     int32_t *C_debug;
+    __half *Wo;                          // [N, wo_pitch] or null
+    int64_t wo_pitch;
     const uint8_t *image;
     const DecodeTables *tables;
     StatusRef status;
@@ -496,9 +498,11 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 const int8_t *cbrow = a.CB + (int64_t)n * a.K;
                 for (int j = 0; j < n_out; ++j) {
                     const int col = tail->tab.idx[j];
-                    const float w = a.W16 ? __half2float(a.W16[(int64_t)n * a.K + col])
-                                          : __half2float(__float2half_rn(__fdiv_rn(
-                                                __fmul_rn((float)cbrow[col], sb), 127.0f)));
+                    const __half wh = a.W16 ? a.W16[(int64_t)n * a.K + col]
+                                            : __float2half_rn(__fdiv_rn(
+                                                  __fmul_rn((float)cbrow[col], sb), 127.0f));
+                    if (a.Wo) a.Wo[(int64_t)n * a.wo_pitch + j] = wh;
+                    const float w = __half2float(wh);
                     const uint4 *xv = reinterpret_cast<const uint4 *>(tail->xo + j * DM);
                     float f0[8], f1[8];
                     unpack8(xv[0], f0);
@@ -634,6 +638,8 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     a.bias = d.bias;
     a.Y = d.Y;
     a.C_debug = d.C_debug;
+    a.Wo = d.Wo;
+    a.wo_pitch = d.wo_pitch;
     a.image = d.image;
     a.tables = d.tables;
     a.status = d.status;

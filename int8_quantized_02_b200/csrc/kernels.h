@@ -100,6 +100,8 @@ struct DecodeLaunch {
     const __half *bias;      // [N] or null
     __half *Y;               // [M, N]
     int32_t *C_debug;        // [M, N] or null
+    __half *Wo;              // [N, wo_pitch] or null: receives the outlier weights used
+    int64_t wo_pitch;
     int32_t *count;          // device outlier count (workspace header)
     uint8_t *image;          // workspace: decode_image_bytes(K), 1024-byte aligned
     DecodeTables *tables;    // workspace

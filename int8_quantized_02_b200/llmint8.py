@@ -48,6 +48,8 @@ PROTOTYPES = {
     "llmint8_linear_host": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _F32, _I64, _P,
                                            _P, _P, _P, _SZ, _P]),
     "llmint8_outlier_bitmap": (ctypes.c_int, [_P, _I64, _I64, _F32, _P, _P, _SZ, _P]),
+    "llmint8_workspace_outlier_weights": (ctypes.c_int, [_P, _I64, _I64, _I64, _I64, _P, _I64,
+                                                         _P]),
     "llmint8_linear_with_bitmaps": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _P, _I64,
                                                    _I64, _P, _P, _SZ, _P, _P]),
 }
@@ -402,6 +404,18 @@ def llmint8_workspace_outlier_count(workspace: torch.Tensor, stream=None) -> int
                                                   ctypes.byref(n)),
            "llmint8_workspace_outlier_count")
     return int(n.value)
+
+
+def llmint8_workspace_outlier_weights(workspace: torch.Tensor, M: int, N: int, K: int,
+                                      max_outliers: int, n_cols: int, stream=None):
+    """fp16 [N, n_cols]: the outlier-weight rows the last llmint8_linear call on `workspace`
+    (with these M, N, K, max_outliers) used; on the decode path only after a call with
+    C_debug."""
+    Wo = torch.empty((N, max(int(n_cols), 1)), dtype=torch.float16, device=workspace.device)
+    _check(load().llmint8_workspace_outlier_weights(_ptr(workspace), M, N, K, max_outliers,
+                                                    _ptr(Wo), int(n_cols), _stream(stream)),
+           "llmint8_workspace_outlier_weights")
+    return Wo[:, :int(n_cols)]
 
 
 def llmint8_set_wait_timeout_ns(ns: int) -> None:

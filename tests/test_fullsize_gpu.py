@@ -39,6 +39,11 @@ def _weights(wl):
 
 
 def _positions(M, N, n=480, seed=0):
+    """Sampled output positions: `n` random ones, the corners of the first and last tiles, and
+    two in every output tile of the GEMM (256 x 256 for M > 128, else 128 x 256).  Across
+    the tiles the samples rotate through every 32-column epilogue chunk, every 32-row
+    epilogue warp and, for 256-row tiles, both CTAs of the pair, so a fault confined to
+    some tiles, one chunk or one warp cannot pass unseen."""
     rng = np.random.default_rng(seed)
     rows = list(rng.integers(0, M, n))
     cols = list(rng.integers(0, N, n))
@@ -48,6 +53,20 @@ def _positions(M, N, n=480, seed=0):
         for c in edge_c:
             rows.append(r)
             cols.append(c)
+    tile_m, tile_n = (256 if M > 128 else 128), 256
+    t = 0
+    for tm in range(-(-M // tile_m)):
+        for tn in range(-(-N // tile_n)):
+            for half in range(2):
+                chunk = (t + 4 * half) % 8
+                warp = (t // 8 + half) % 4
+                r = tm * tile_m + (half * 128 if tile_m == 256 else 0) + warp * 32 + \
+                    int(rng.integers(0, 32))
+                c = tn * tile_n + chunk * 32 + int(rng.integers(0, 32))
+                if r < M and c < N:
+                    rows.append(r)
+                    cols.append(c)
+            t += 1
     return np.asarray(rows, np.int64), np.asarray(cols, np.int64)
 
 
@@ -79,6 +98,11 @@ def _check(wl, threshold, cap):
     assert np.array_equal(host(Y2), Y_b), f"{wl.name}: output differs with C_debug"
     C_h = host(C)
     del C
+    # step a3 bit for bit: the fp16 weight rows used for the outlier columns
+    n_w = min(n_o, cap)
+    Wo = host(L.llmint8_workspace_outlier_weights(ws, M, N, K, cap, n_w))
+    want = oracle.dequant(np.ascontiguousarray(CB_o[:, idx_o[:n_w]]), SCB_o)
+    assert np.array_equal(Wo.view(np.uint16), want.view(np.uint16)), f"{wl.name}: W_o"
 
     if M <= 16:
         Y_o, C_o = oracle.linear(X, CB_o, SCB_o, threshold=threshold, want_C=True)

@@ -290,6 +290,40 @@ def check_half_codec(lib):
     assert np.array_equal(got, want)
 
 
+def check_int8_accumulate(lib):
+    """The stand-alone int8 product against facts outside it: exact Python-integer sums of
+    the brute force on tiny shapes, numpy int64 products on larger ones (every int8 code,
+    -128 included), and the int32 overflow flag exactly at the first K where all-127
+    operands leave the int32 range (INT32_MAX // 127^2 = 133144)."""
+    rng = np.random.default_rng(17)
+    for M, K, N in ((1, 16, 1), (3, 16, 5), (4, 32, 8)):
+        X = (rng.standard_normal((M, K)) * 2).astype(np.float16)
+        W = (rng.standard_normal((N, K)) * 0.05).astype(np.float16)
+        ref = brute.layer(X, W, 6.0)
+        C = oracle.int8_accumulate(ref["Xq"], ref["CB"], lib=lib)
+        assert C.dtype == np.int32 and C.shape == (M, N)
+        assert np.array_equal(C.astype(np.int64), ref["C"])
+    A = rng.integers(-128, 128, (7, 200), dtype=np.int64).astype(np.int8)
+    B = rng.integers(-128, 128, (9, 200), dtype=np.int64).astype(np.int8)
+    C = oracle.int8_accumulate(A, B, lib=lib)
+    assert np.array_equal(C.astype(np.int64), A.astype(np.int64) @ B.astype(np.int64).T)
+    # a row against itself and against its negation: the largest and smallest sums
+    k_ok = (2**31 - 1) // (127 * 127)
+    for K, sign, overflow in ((k_ok, 1, False), (k_ok + 1, 1, True), (k_ok, -1, False),
+                              (k_ok + 1, -1, True)):
+        a = np.full((1, K), 127, np.int8)
+        b = np.full((2, K), 127, np.int8)
+        b[1] = 1
+        b[0] *= sign
+        if overflow:
+            with pytest.raises(oracle.OracleError) as e:
+                oracle.int8_accumulate(a, b, lib=lib)
+            assert e.value.code == oracle.ERR_INT32_OVERFLOW
+        else:
+            C = oracle.int8_accumulate(a, b, lib=lib)
+            assert C[0, 0] == sign * 127 * 127 * K and C[0, 1] == 127 * K
+
+
 def check_capacity(lib):
     X = np.full((2, 32), 7.0, np.float16)
     with pytest.raises(oracle.OracleError) as e:
@@ -301,7 +335,7 @@ ALL_CHECKS = [check_absmax_worked_example, check_scaling_worked_example,
               check_printed_rows_are_per_output_channel, check_threshold_inclusive,
               check_round_half_even, check_closed_form, check_no_outliers_is_pure_int8,
               check_all_outliers_is_fp16_gemm, check_brute_force, check_invariants,
-              check_half_codec, check_capacity]
+              check_half_codec, check_int8_accumulate, check_capacity]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda c: c.__name__[6:])
@@ -334,6 +368,14 @@ MUTANTS = [
     ("half_exponent_bias", r"ldexp\(\(double\)\(m \+ 1024\), e - 25\)",
      "ldexp((double)(m + 1024), e - 24)"),
     ("stores_multiplier_not_absmax", r"SCB\[n\] = amax;", "SCB[n] = 127.0f / amax;"),
+    ("accumulate_reversed_k_index",
+     r"CB\[n \* K \+ k\];\n            if \(acc > INT32_MAX",
+     "CB[n * K + (K - 1 - k)];\n            if (acc > INT32_MAX"),
+    ("accumulate_overflow_unflagged",
+     r"if \(acc > INT32_MAX \|\| acc < INT32_MIN\) overflow = 1;\n            C\[i \* N \+ n\]",
+     "C[i * N + n]"),
+    ("accumulate_output_transposed", r"C\[i \* N \+ n\] = \(int32_t\)acc;",
+     "C[n * M + i] = (int32_t)acc;"),
     ("sampled_rows_and_cols_swapped", r"Xq, SCA, rows\[s\], cols\[s\],",
      "Xq, SCA, cols[s] % M, rows[s] % N,"),
 ]
@@ -362,6 +404,6 @@ def test_pins_catch_planted_mistake(name, pattern, repl, mutant_dir):
     for check in ALL_CHECKS:
         try:
             check(lib)
-        except (AssertionError, oracle.OracleError, Exception):  # noqa: BLE001
+        except (Exception, pytest.fail.Exception):  # noqa: BLE001 - a failed pytest.raises too
             caught.append(check.__name__)
     assert caught, f"no pin catches the planted mistake {name}"

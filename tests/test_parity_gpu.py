@@ -126,7 +126,22 @@ def _check_linear(X, W, t, bias=None, keep_fp16=False, cap=None):
                              threshold=t, want_C=True)
     assert np.array_equal(host(C), C_o)
     assert_y_close(host(Y), Y_o)
+    _check_outlier_weights(ws, X, W, CB_o, SCB_o, t, keep_fp16, cap)
     return host(Y), Y_o
+
+
+def _check_outlier_weights(ws, X, W, CB_o, SCB_o, t, keep_fp16, cap):
+    """Step a3 bit for bit: the fp16 weight rows the call used for the outlier columns are
+    the oracle's dequantized int8 weights (CB * SCB) / 127 at those columns, or the given fp16
+    weights (blog section 用法)."""
+    M, K = X.shape
+    N = W.shape[0]
+    _, _, O = oracle.quantize_rows_and_find_outliers(X, t)
+    n = min(O.size, cap)
+    Wo = host(L.llmint8_workspace_outlier_weights(ws, M, N, K, cap, n))
+    want = (W if keep_fp16 else oracle.dequant(CB_o, SCB_o))[:, O[:n]]
+    assert np.array_equal(Wo.view(np.uint16), np.ascontiguousarray(want).view(np.uint16)), \
+        "outlier weight rows W_o"
 
 
 LINEAR_CASES = {
