@@ -2,26 +2,30 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-Prints ONE JSON line (rank 0).  Workloads (seeded synthetic inputs, int8_quantized_02_b200.synth):
-  decode     (default) X [b, 4096] for b in (1, 8, 16), six outlier columns |x| in [6, 60] on
-             every row; CB [16384, 4096] quantized once beforehand.  One step = the three
-             llmint8_linear calls.  Metric: weight-streaming GB/s =
-             sum_b (N*K + 4N + 2bK + 2bN) / time.
+Prints ONE JSON line (rank 0).  By default every workload runs: decode is the headline (the
+line's value, roofline, e2e, ...), and the prefill workloads follow under "workloads", each
+with the same keys.  Workloads (seeded synthetic inputs, int8_quantized_02_b200.synth):
+  decode     X [b, 4096] for b in (1, 8, 16), six outlier columns |x| in [6, 60] on every row;
+             CB [16384, 4096] quantized once beforehand.  One step = the three llmint8_linear
+             calls.  Metric: weight-streaming GB/s = sum_b (N*K + 4N + 2bK + 2bN) / time.
   ffn6.7b    X [2048, 4096] . W1^T (16384 outputs), then X2 [2048, 16384] . W2^T (4096 outputs);
              six outlier columns of U(6, 20) on 75 % of rows.  Metric: TOPS = 2MNK / time.
   proj175b   X [4096, 12288] . W^T (49152 outputs), W ~ N(0, 0.01).  TOPS.
   sweep      X [4096, 8192] . W^T (8192 outputs); one step = K' in {0, 6, 64, 512} at
              threshold 6, plus threshold=inf and threshold=0.  TOPS.
+Timing: each workload's region of K whole steps (inputs resident in HBM, larger than L2 or
+rotated through more than 3 x L2) is bracketed by a barrier and a synchronize on both sides and
+timed with CUDA events on the launching stream (the slowest rank's time); the region is
+repeated until the repeats add up to about a second (half a second per prefill workload) and
+the value is the median over the repeats, reported with its spread.
 Multi-GPU (torchrun): replicas only - every rank runs the same workload on its own GPU with no
 data-path collective; value = units of all ranks / max-over-ranks time ("scaling": "weak").
 """
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import os
-import re
 import statistics
 import sys
 import threading
@@ -123,30 +127,6 @@ class ClockSampler:
         sm = [s for s, _ in self.samples]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(active), "samples": len(sm)}
-
-
-def kernel_source_hash() -> str:
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "int8_quantized_02_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
-    return h.hexdigest()[:16]
-
-
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the product kernel from the committed ncu summary of this
-    workload, when it was taken on the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.md")
-    if not os.path.exists(path):
-        return None
-    text = open(path).read()
-    m_hash = re.search(r"kernel_source_hash:\s*(\w+)", text)
-    m_val = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_val or m_hash.group(1) != kernel_source_hash():
-        return None
-    return float(m_val.group(1))
 
 
 # -------------------------------------------------------------------------- workloads ----
@@ -264,18 +244,41 @@ def whole_job_value(units_per_step: float, steps: int, world: int, seconds: floa
     return unit_value(units_per_step * steps * world, seconds, unit)
 
 
+def repeat_count(region_s: float, target_s: float, lo: int = 3, hi: int = 200) -> int:
+    """How many times to repeat a timed region of `region_s` seconds so that the repeats
+    together last about `target_s` (at least `lo`, at most `hi`)."""
+    if region_s <= 0:
+        return hi
+    return int(max(lo, min(hi, -(-target_s // region_s))))
+
+
+def spread(values):
+    """Median and spread of the per-repeat values of a metric."""
+    v = sorted(values)
+    q = lambda f: v[min(len(v) - 1, int(round(f * (len(v) - 1))))]  # noqa: E731
+    return {"n": len(v), "median": statistics.median(v), "min": v[0], "max": v[-1],
+            "p10": q(0.1), "p90": q(0.9)}
+
+
 # ------------------------------------------------------------------------ our arm ----
 
-def run_ours(args, rank, world, local_rank):
+# Seconds of timed work the repeats of each workload's region add up to.
+TARGET_S = {"decode": 1.0, "ffn6.7b": 0.5, "proj175b": 0.5, "sweep": 0.5}
+ALL_WORKLOADS = ("decode", "ffn6.7b", "proj175b", "sweep")
+
+
+def run_workload(name, args, rank, world, local_rank):
+    """Every figure of one workload: the repeated timed region (value), the dominant kernel's
+    roofline, the per-call figures, end to end through the host-buffer call, clocks, and
+    (rank 0, one GPU) the oracle on the host cores."""
     import torch
     import torch.distributed as dist
 
     from int8_quantized_02_b200 import llmint8 as L
 
-    torch.cuda.set_device(local_rank)
-    L.load()
-    calls, unit, bound = build_workload(args.workload, L, torch)
+    calls, unit, bound = build_workload(name, L, torch)
     step_units = sum(c.units for c in calls)
+    stream = torch.cuda.current_stream()
 
     def step():
         for c in calls:
@@ -286,174 +289,187 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    for c in calls:
-        st = L.llmint8_device_status(c.ws)
-        if st != L.OK:
-            raise SystemExit(f"{c.name}: device status {L.status_string(st)}")
+    def check_status(what):
+        for c in calls:
+            st = L.llmint8_device_status(c.ws)
+            if st != L.OK:
+                raise SystemExit(f"{c.name}{what}: device status {L.status_string(st)}")
 
-    # ---- timed region: whole steps, inputs resident, CUDA events on the launching stream.
-    # Prefill calls run for a tenth of a millisecond or more, so a pair of profile events
-    # around each GEMM launch costs little (the GEMM then starts after its quantize kernel
-    # instead of overlapping its tail) and gives the dominant kernel's own duration.  A decode call
-    # lasts about 20 us and an event pair adds about 5 us, so decode records no per-call
-    # events: its weight-streaming kernel spans the whole call (the quantize kernel runs under
-    # it as a programmatic dependent), and the call's duration is region time / calls.
-    stream = torch.cuda.current_stream()
-    per_call_events = bound != "hbm"
-    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in calls] for _ in range(args.steps if per_call_events else 0)]
-    # torch creates an event's CUDA handle on its first record(): record each once here so
-    # the library can re-record the same handles around the product kernel
-    for row in kev:
-        for ev_a, ev_b in row:
-            ev_a.record(stream)
-            ev_b.record(stream)
-    torch.cuda.synchronize()
-    launches0 = L.llmint8_kernel_launch_count()
-    barrier()
-    with ClockSampler(local_rank) as clk:
+    def region(n_steps, run=step):
+        """One timed region of n_steps whole steps: barrier + synchronize on both sides,
+        CUDA events on the launching stream, the slowest rank's time."""
+        barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for s in range(args.steps):
-            for j, c in enumerate(calls):
-                if per_call_events:
-                    L.llmint8_set_profile_events(*kev[s][j])
-                c.run()
+        for _ in range(n_steps):
+            run()
         e1.record(stream)
-        if per_call_events:
-            L.llmint8_set_profile_events(None, None)
         torch.cuda.synchronize()
-    barrier()
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1) / 1e3, world, device="cuda")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    check_status("")
+
+    # ---- the timed region, K whole steps with inputs resident, repeated; an untimed region
+    # of the same length first sets the repeat count (the same on every rank)
+    reps = repeat_count(region(args.steps), TARGET_S.get(name, 0.5),
+                        hi=1000 if bound == "hbm" else 200)
+    launches0 = L.llmint8_kernel_launch_count()
+    with ClockSampler(local_rank) as clk:
+        times = [region(args.steps) for _ in range(reps)]
     launches = L.llmint8_kernel_launch_count() - launches0
-    elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, device="cuda")
-    if per_call_events:
-        call_s = [sum(kev[s][j][0].elapsed_time(kev[s][j][1]) for s in range(args.steps))
-                  / 1e3 / args.steps for j in range(len(calls))]
-    else:
-        # no per-call split inside the region: each call gets its share of the step by units
-        call_s = [elapsed / args.steps * c.units / step_units for c in calls]
-    kern_s = sum(call_s) * args.steps
-    for c in calls:
-        st = L.llmint8_device_status(c.ws)
-        if st != L.OK:
-            raise SystemExit(f"{c.name}: device status {L.status_string(st)}")
+    check_status("")
+    vals = [whole_job_value(step_units, args.steps, world, t, unit) for t in times]
+    rep = spread(vals)
+    t_med = statistics.median(times)
 
-    # ---- per-call figures, after the timed region: each decode call alone, back to back on
-    # rotating weights, between one pair of events (the headline above does not use these)
-    alone_s = None
-    if not per_call_events:
-        alone_s = []
+    # ---- the dominant kernel.  Decode: one kernel per call, so its duration is the region's
+    # time per call (per-call events would add several microseconds to a ~15 us call).
+    # Prefill: CUDA events around each GEMM launch in one extra region of K steps (the events
+    # keep the GEMM from overlapping the tail of its row-quantization kernel, which costs
+    # little at these sizes).
+    peaks = measured_peaks()
+    per_call = {}
+    if bound == "hbm":
+        achieved = step_units * args.steps / t_med / 1e9
+        peak, roof_unit = peaks["hbm_gbs"], "GB/s"
+        kernel_name = "llmint8_decode_kernel"
+        timing = "median region time / calls (one kernel per call, no per-call events)"
+        # each call alone, steps calls back to back (not used by the headline)
         for c in calls:
-            b0 = torch.cuda.Event(enable_timing=True)
-            b1 = torch.cuda.Event(enable_timing=True)
-            b0.record(stream)
-            for _ in range(args.steps):
+            t = region(args.steps, c.run)
+            per_call[c.name] = {"call_us": t / args.steps * 1e6,
+                                "GB/s": c.units / (t / args.steps) / 1e9,
+                                "timing": "this call alone, steps back-to-back calls"}
+        whole = None
+    else:
+        kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in calls] for _ in range(args.steps)]
+        # torch creates an event's CUDA handle on its first record(): record each once here
+        # so the library can re-record the same handles around the product kernel
+        for row in kev:
+            for ev_a, ev_b in row:
+                ev_a.record(stream)
+                ev_b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        for s_ in range(args.steps):
+            for j, c in enumerate(calls):
+                L.llmint8_set_profile_events(*kev[s_][j])
                 c.run()
-            b1.record(stream)
-            torch.cuda.synchronize()
-            alone_s.append(max_over_ranks(b0.elapsed_time(b1) / 1e3 / args.steps, world,
-                                          device="cuda"))
+        L.llmint8_set_profile_events(None, None)
+        torch.cuda.synchronize()
+        barrier()
+        call_s = [max_over_ranks(sum(kev[s_][j][0].elapsed_time(kev[s_][j][1])
+                                     for s_ in range(args.steps)) / 1e3 / args.steps,
+                                 world, device="cuda") for j in range(len(calls))]
+        achieved = step_units / sum(call_s) / 1e12
+        peak, roof_unit = 2.0 * peaks["bf16_tflops"], "TOPS"   # int8 = 2 x bf16 (nominal)
+        kernel_name = ("llmint8_gemm_pair_kernel" if all(c.M > 128 for c in calls)
+                       else "llmint8_gemm_kernel")
+        timing = "CUDA events around each GEMM launch, one region of K steps"
+        for j, c in enumerate(calls):
+            per_call[c.name] = {"kernel_us": call_s[j] * 1e6,
+                                "TOPS": c.units / call_s[j] / 1e12}
+        w = rep["median"] / world
+        whole = {"achieved": w, "frac": w / peak,
+                 "timing": "whole llmint8_linear calls (every kernel of the layer): median "
+                           "region time"}
 
-    # ---- end to end through the C ABI's host-buffer call: every call copies its X from pinned
-    # host memory, runs the layer and copies Y back into pinned host memory.  The calls of a
-    # step share no buffer (own X, Y and workspace), so each runs on a stream of its own and
-    # one call's copies overlap the others' kernels; a call's steps stay in order.
+    # ---- end to end through the C ABI's host-buffer call, on the same single stream as the
+    # timed region: every call copies its X in from pinned host memory, runs the layer and
+    # copies Y out into pinned host memory
     hosts = [(c.X.cpu().pin_memory(),
               torch.empty((c.M, c.N), dtype=torch.float16).pin_memory()) for c in calls]
     xd = [torch.empty_like(c.X) for c in calls]
-    e2e_streams = [torch.cuda.Stream() for _ in calls]
-    e2e_plans = [c.host_plan(hosts[j][0], hosts[j][1], xd[j], e2e_streams[j])
+    e2e_plans = [c.host_plan(hosts[j][0], hosts[j][1], xd[j], stream)
                  for j, c in enumerate(calls)]
-    e2e_steps = max(1, min(args.steps, 50))
 
-    def e2e_run(n):
-        start = torch.cuda.Event()
-        start.record(stream)
-        for st in e2e_streams:
-            st.wait_event(start)
-        for _ in range(n):
-            for j, c in enumerate(calls):
-                c.run(e2e_plans[j])
-        for st in e2e_streams:
-            done = torch.cuda.Event()
-            done.record(st)
-            stream.wait_event(done)
+    def e2e_step():
+        for j, c in enumerate(calls):
+            c.run(e2e_plans[j])
 
-    e2e_run(2)
-    barrier()
-    a0 = torch.cuda.Event(enable_timing=True)
-    a1 = torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    e2e_run(e2e_steps)
-    a1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_s = max_over_ranks(a0.elapsed_time(a1) / 1e3, world, device="cuda")
+    for _ in range(2):
+        e2e_step()
+    e2e_reps = repeat_count(region(args.steps, e2e_step), TARGET_S.get(name, 0.5) / 2, lo=3,
+                            hi=50)
+    e2e_times = [region(args.steps, e2e_step) for _ in range(e2e_reps)]
+    e2e_vals = [whole_job_value(step_units, args.steps, world, t, unit) for t in e2e_times]
+    check_status(" (end to end)")
     for j, c in enumerate(calls):
-        st = L.llmint8_device_status(c.ws)
-        if st != L.OK:
-            raise SystemExit(f"{c.name} (end to end): device status {L.status_string(st)}")
         if not torch.equal(hosts[j][1], c.Y.cpu()):
             raise SystemExit(f"{c.name} (end to end): host Y differs from the device Y")
 
-    peaks = measured_peaks()
-    traffic = profiled_traffic(args.workload)
-    if bound == "hbm":
-        # algorithmic bytes of a call: N*K + 4N + 2MK + 2MN (weights, scales, X in, Y out)
-        achieved = step_units * args.steps / kern_s / 1e9
-        peak = peaks["hbm_gbs"]
-        roof_unit = "GB/s"
-        kernel_name = "llmint8_decode_kernel (+ llmint8_decode_quantize_kernel under it)"
-        timing = "device time of the timed region / calls (no per-call events)"
-    else:
-        achieved = step_units * args.steps / kern_s / 1e12
-        peak = 2.0 * peaks["bf16_tflops"]           # int8 dense = 2 x bf16 dense (nominal ratio)
-        roof_unit = "TOPS"
-        kernel_name = ("llmint8_gemm_pair_kernel" if all(c.M > 128 for c in calls)
-                       else "llmint8_gemm_kernel")
-        timing = "CUDA events around each GEMM launch, averaged over the timed region"
+    out = {
+        "value": rep["median"],
+        "unit": unit,
+        "ms_per_step": t_med / args.steps * 1e3,
+        "repeats": {**rep, "steps_per_repeat": args.steps,
+                    "note": "value = median over repeats of the K-step timed region"},
+        "config": workload_config(name, calls),
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": roof_unit,
+                     "frac": achieved / peak,
+                     "peak_source": f"{peaks['source']} "
+                                    + ("hbm_gbs" if bound == "hbm" else "2 x bf16_tflops (burst)"),
+                     "kernel": kernel_name, "timing": timing,
+                     "traffic": None,
+                     "traffic_note": "DRAM bytes are not measurable inside this run (no "
+                                     "profiler); the per-launch ncu counters are in profiles/"},
+        "e2e": {"value": statistics.median(e2e_vals), "unit": unit,
+                "h2d_bytes_per_step": sum(c.h2d_bytes for c in calls),
+                "d2h_bytes_per_step": sum(c.d2h_bytes for c in calls),
+                "repeats": len(e2e_vals), "min": min(e2e_vals), "max": max(e2e_vals),
+                "arrangement": "llmint8_linear_host per call, one stream (as the timed region)"},
+        "gpu_launches": int(launches),
+        "gpu_launches_note": f"library kernels launched in the {reps} timed repeats",
+        "clocks": clk.summary(),
+        "per_call": per_call,
+    }
+    if whole is not None:
+        out["roofline"]["whole_call"] = whole
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(name, budget_s=15.0 if name == "decode" else 8.0)
+    del calls, hosts, xd, e2e_plans
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    from int8_quantized_02_b200 import llmint8 as L
+
+    torch.cuda.set_device(local_rank)
+    L.load()
+    names = ALL_WORKLOADS if args.workload == "all" else (args.workload,)
+    results = {n: run_workload(n, args, rank, world, local_rank) for n in names}
+    head_name = names[0]
+    head = results[head_name]
     result = {
         "metric": "LLM.int8 linear TOPS (prefill) / weight GB/s (decode); fraction of roofline",
-        "value": whole_job_value(step_units, args.steps, world, elapsed, unit),
-        "unit": unit,
+        "value": head["value"],
+        "unit": head["unit"],
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": elapsed / args.steps * 1e3,
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "i8",
         "dtype_note": "int8 x int8 -> int32 product; fp16 in/out; fp16 x fp16 -> fp32 outlier part",
         "data": "synthetic (seeded, int8_quantized_02_b200.synth)",
-        "config": workload_config(args.workload, calls),
-        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": roof_unit,
-                     "frac": achieved / peak,
-                     "peak_source": f"{peaks['source']} "
-                                    + ("hbm_gbs" if bound == "hbm" else "2 x bf16_tflops (burst)"),
-                     "kernel": kernel_name, "timing": timing,
-                     "traffic": traffic},
-        "e2e": {"value": whole_job_value(step_units, e2e_steps, world, e2e_s, unit), "unit": unit,
-                "h2d_bytes_per_step": sum(c.h2d_bytes for c in calls),
-                "d2h_bytes_per_step": sum(c.d2h_bytes for c in calls)},
-        "gpu_launches": int(launches),
-        "clocks": clk.summary(),
-        "per_call": {c.name: None for c in calls},
     }
-    # per-call figure: the GEMM's own events (prefill) or the call run alone (decode)
-    for j, c in enumerate(calls):
-        sec = call_s[j] if alone_s is None else alone_s[j]
-        v = c.units / sec / (1e9 if bound == "hbm" else 1e12)
-        result["per_call"][c.name] = {("call_us" if bound == "hbm" else "kernel_us"):
-                                      sec * 1e6, unit: v}
-        if alone_s is not None:
-            result["per_call"][c.name]["timing"] = "this call alone, steps back-to-back calls"
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(args.workload)
+    for k in ("config", "repeats", "roofline", "e2e", "gpu_launches", "gpu_launches_note",
+              "clocks", "per_call", "cpu_baseline"):
+        if k in head:
+            result[k] = head[k]
+    if len(names) > 1:
+        result["workloads"] = {n: results[n] for n in names[1:]}
     return result
 
 
@@ -558,23 +574,25 @@ def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default: 1000 for decode, 20 otherwise; 20 for the "
-                         "reference arm)")
+                    help="steps per timed region (default 20); the region is repeated until "
+                         "the repeats add up to about a second, and the value is their median")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="decode",
-                    choices=("decode", "ffn6.7b", "proj175b", "sweep"))
+    ap.add_argument("--workload", default="all", choices=("all",) + ALL_WORKLOADS,
+                    help="all (default): decode is the headline, the prefill workloads are "
+                         "reported under 'workloads' in the same line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.steps is None:
-        # a decode step lasts about 65 us: 1000 of them keep the clock sampler in the region
-        args.steps = 1000 if args.workload == "decode" and args.impl == "ours" else 20
+        args.steps = 20
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
+        if args.workload == "all":
+            args.workload = "decode"      # the headline's workload
         out = run_reference(args, rank, world)
         if out is not None:
             print(json.dumps(out), flush=True)

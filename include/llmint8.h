@@ -109,11 +109,13 @@ LLMINT8_API size_t llmint8_quantize_workspace_size(int64_t M, int64_t K);
  *           evaluated in fp32 with int32 C.
  *   ws      device workspace of llmint8_linear_workspace_size(M, N, K, max_outliers) bytes.
  *   C_debug int32 [M, N] or NULL: when given, also receives the exact int8 accumulators C.
- * Kernels (the results do not depend on the choice): M <= 16, K <= 8192, threshold > 0 and
- * max_outliers <= 256 run two kernels, a row quantizer and a weight-streaming tcgen05 kernel
- * launched as its programmatic dependent.  Other shapes run outlier detection, row
- * quantization (with the gather of the outlier weight rows) and a persistent tcgen05 GEMM,
- * on CTA pairs when M > 128.
+ * Kernels (int8 codes, outlier columns and C do not depend on the choice; Y may differ in
+ * the last fp32 rounding): M <= 16, K <= 16384, threshold > 0 and max_outliers <= 256 run one
+ * weight-streaming tcgen05 kernel whose CTAs each quantize X themselves.  Other shapes run
+ * outlier detection, row quantization (with the gather of the outlier weight rows) and a
+ * persistent tcgen05 GEMM, on CTA pairs when M > 128.  Kernels of a call are launched as
+ * programmatic dependents: each may start while the work before it on the stream finishes,
+ * and waits for that work before it reads or writes global memory.
  */
 LLMINT8_API llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
                               const float *SCB, int64_t N, const uint16_t *bias,
@@ -130,7 +132,9 @@ LLMINT8_API size_t llmint8_linear_workspace_size(int64_t M, int64_t N, int64_t K
  * whole hidden state), so a rank's own rows do not decide it.  Each rank computes its
  * rows' bitmap, the ranks exchange the bitmaps (an all-gather of ceil(K/32) words each), and
  * every rank runs the layer on its rows with the OR of all of them.  The rows it gets are
- * the same bytes llmint8_linear gives for those rows of the whole X.
+ * llmint8_linear's int8 codes and int32 C for those rows of the whole X, and Y within the
+ * layer's tolerance (the same bytes when the same kernel serves both: the decode kernel for
+ * at most 16 rows, the GEMM otherwise; the two may round the last fp32 step differently).
  *
  * llmint8_outlier_bitmap: bit (j % 32) of bitmap[j / 32] is set iff some row of X [M, K]
  *   has |X[i, j]| >= threshold (threshold rules as in
@@ -148,10 +152,11 @@ LLMINT8_API llmint8_status llmint8_outlier_bitmap(const uint16_t *X, int64_t M, 
  *   O = the columns set in ANY of the n_bitmaps bitmaps [n_bitmaps][ceil(K/32)] (uint32,
  *   device, 4-byte aligned; 1 <= n_bitmaps <= 65536).  Bits at columns >= K are ignored.
  *   Every other argument, the workspace (llmint8_linear_workspace_size(M, N, K,
- *   max_outliers)) and the output are as for llmint8_linear, without a threshold.  The
- *   call always runs the outlier compaction, the row quantization and the tcgen05 GEMM
- *   (the decode kernels find the outliers themselves).  More outlier columns than
- *   max_outliers sets LLMINT8_ERR_OUTLIER_CAPACITY in the device status.
+ *   max_outliers)) and the output are as for llmint8_linear, without a threshold.  Shapes of
+ *   the decode path (M <= 16, K <= 16384, max_outliers <= 256) run the decode kernel with the
+ *   merged bitmaps as its outlier set; others run the outlier compaction, the row
+ *   quantization and the tcgen05 GEMM.  More outlier columns than max_outliers sets
+ *   LLMINT8_ERR_OUTLIER_CAPACITY in the device status.
  */
 LLMINT8_API llmint8_status llmint8_linear_with_bitmaps(const uint16_t *X, int64_t M, int64_t K,
                                            const int8_t *CB, const float *SCB, int64_t N,
@@ -253,26 +258,32 @@ LLMINT8_API uint64_t llmint8_kernel_launch_count(void);
  * calling convenience.  It is for callers that cannot allocate device memory where they
  * call the layer: a token-by-token decode loop that must not call cudaMalloc/cudaFree
  * between steps (cudaFree waits for the whole device), or a plain C host without a device
- * allocator of its own.  The call allocates nothing.  Its scratch is a fixed 160 KiB
- * device array inside this library, one per device.
+ * allocator of its own.  The call allocates nothing.  Its scratch - the 256-byte header that
+ * receives the call's status words and outlier count - is a fixed device array inside this
+ * library, one per device.
  *   Arguments X, M, K, CB, SCB, N, bias, W_fp16, threshold, max_outliers, Y, stream: as
- *     for llmint8_linear (same layouts, same output).  There is no C_debug output.
- *   Covered shapes are those of the decode path: M <= 16, K <= 8192 (K, N multiples of
+ *     for llmint8_linear (same layouts, same output, the same bytes).  There is no C_debug
+ *     output.  Profile events set with llmint8_set_profile_events are recorded around its
+ *     kernel as for llmint8_linear.
+ *   Covered shapes are those of the decode path: M <= 16, K <= 16384 (K, N multiples of
  *     16), threshold > 0 and max_outliers <= 256.  Anything larger returns
  *     LLMINT8_ERR_UNSUPPORTED_SHAPE before any CUDA call; use llmint8_linear there.
- *   scratch_out  NULL, or receives the device address of the calling device's scratch.
- *     The scratch begins with the same 256-byte header as an llmint8_linear workspace.
- *     So llmint8_device_status(*scratch_out, stream) and
+ *   scratch_out  NULL, or receives the device address of the calling device's scratch, the
+ *     same 256-byte header as at the start of an llmint8_linear workspace.  So
+ *     llmint8_device_status(*scratch_out, stream) and
  *     llmint8_workspace_outlier_count(*scratch_out, ...) report the device status and the
  *     outlier count of the last call on that device.
  *   Set-up: the first call on each device looks up the scratch's address
  *     (cudaGetSymbolAddress, with the device current), which may load this library's
- *     device code.  Make that first call before any stream capture.
- *   The scratch starts zero-filled when the module loads.  Nothing in it needs clearing
- *     between calls.
- *   Calls on one stream, in order, are safe.  Calls that overlap on one device share its
- *     scratch and race, with undefined outputs.  Overlap means two streams, or host
- *     threads without stream order between them.
+ *     device code.  Make that first call before any stream capture.  The address is kept for
+ *     the life of the process: a device reset (cudaDeviceReset) between calls is not
+ *     supported.
+ *   Nothing in the scratch needs clearing between calls: each call tags its status words
+ *     with a fresh call number and stores the outlier count.
+ *   Calls on one stream, in order, are safe.  Calls that overlap on one device (two
+ *     streams, or host threads without stream order between them) share its scratch and
+ *     race on it: their outputs are unaffected, but the status and count read back may
+ *     belong to either call.
  * Returns LLMINT8_ERR_INVALID_ARG for NULL or misaligned pointers (16 bytes) or a NaN
  * threshold, and LLMINT8_ERR_CUDA if the set-up or a launch fails.
  */

@@ -36,7 +36,7 @@ struct LinearLayout {
     ScanPlan plan;
     int64_t cap = 0, pitch = 0;
     size_t partial = 0, bitmap = 0, idx = 0, sca = 0, xq = 0, xo = 0, wo = 0, total = 0;
-    size_t dimage = 0, dtables = 0;   // decode path (shapes with M <= 16, K <= 8192 only)
+    size_t dtable = 0, dimage = 0;    // decode path (shapes with M <= 16, K <= 16384 only)
 };
 
 LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t cap) {
@@ -58,9 +58,9 @@ LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t cap) {
     L.xo = take((size_t)(M * L.pitch) * 2);
     L.wo = take((size_t)(N * L.pitch) * 2);
     if (M <= kDecodeMaxM && K <= kDecodeMaxK) {
+        L.dtable = take(sizeof(DecodeTable));
         off = (size_t)align_up((int64_t)off, 1024);
-        L.dimage = take((size_t)decode_image_bytes(K));
-        L.dtables = take(sizeof(DecodeTables));
+        L.dimage = take((size_t)decode_image_bytes(M, K));
     }
     L.total = off;
     return L;
@@ -110,6 +110,46 @@ llmint8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK :
 bool use_decode_path(int64_t M, int64_t K, float threshold, int64_t cap) {
     return M <= kDecodeMaxM && K <= kDecodeMaxK && threshold > 0.0f &&
            cap <= kDecodeMaxOutliers;
+}
+
+// Arguments of a decode-path launch whose status words live in the header `h`.
+DecodeLaunch decode_launch(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
+                           const float *SCB, int64_t N, const uint16_t *bias,
+                           const uint16_t *W_fp16, float threshold, int64_t cap, uint16_t *Y,
+                           int32_t *C_debug, WsHeader *h, DecodeTable *table,
+                           uint8_t *image, StatusRef status) {
+    DecodeLaunch d;
+    d.X = reinterpret_cast<const __half *>(X);
+    d.CB = CB;
+    d.SCB = SCB;
+    d.W16 = reinterpret_cast<const __half *>(W_fp16);
+    d.bias = reinterpret_cast<const __half *>(bias);
+    d.Y = reinterpret_cast<__half *>(Y);
+    d.C_debug = C_debug;
+    d.Wo = nullptr;
+    d.wo_pitch = 0;
+    d.bitmaps = nullptr;
+    d.n_bitmaps = 0;
+    d.count = &h->n_outliers;
+    d.table = table;
+    d.image = image;
+    d.status = status;
+    d.M = M;
+    d.N = N;
+    d.K = K;
+    d.cap = cap;
+    d.threshold = threshold;
+    d.timeout_ns = g_timeout_ns.load();
+    return d;
+}
+
+// launch_decode between the process-wide profile events (when set).
+llmint8_status run_decode(const DecodeLaunch &d, cudaStream_t s) {
+    cudaEvent_t ev0 = g_prof_start.load(), ev1 = g_prof_stop.load();
+    if (ev0 && record_profile_event(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (launch_decode(d, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (ev1 && record_profile_event(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    return LLMINT8_OK;
 }
 
 }  // namespace
@@ -272,32 +312,16 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     cudaError_t e;
 
     if (use_decode_path(M, K, threshold, max_outliers)) {
-        // quantize X once, then the weight-streaming tcgen05 kernel (programmatic dependent)
-        DecodeLaunch d;
-        d.X = Xh;
-        d.CB = CB;
-        d.SCB = SCB;
-        d.W16 = reinterpret_cast<const __half *>(W_fp16);
-        d.bias = reinterpret_cast<const __half *>(bias);
-        d.Y = reinterpret_cast<__half *>(Y);
-        d.C_debug = C_debug;
-        d.count = &h->n_outliers;
-        d.Wo = C_debug ? at<__half>(ws, L.wo) : nullptr;
-        d.wo_pitch = L.pitch;
-        d.image = at<uint8_t>(ws, L.dimage);
-        d.tables = at<DecodeTables>(ws, L.dtables);
-        d.status = status;
-        d.M = M;
-        d.N = N;
-        d.K = K;
-        d.cap = max_outliers;
-        d.threshold = threshold;
-        d.timeout_ns = g_timeout_ns.load();
-        if (ev0 && record_profile_event(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
-        e = launch_decode(d, s);
-        if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-        if (ev1 && record_profile_event(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
-        return LLMINT8_OK;
+        // one weight-streaming tcgen05 kernel; every CTA quantizes X itself
+        DecodeLaunch d = decode_launch(X, M, K, CB, SCB, N, bias, W_fp16, threshold,
+                                       max_outliers, Y, C_debug, h,
+                                       at<DecodeTable>(ws, L.dtable), at<uint8_t>(ws, L.dimage),
+                                       status);
+        if (C_debug) {
+            d.Wo = at<__half>(ws, L.wo);
+            d.wo_pitch = L.pitch;
+        }
+        return run_decode(d, s);
     }
 
     uint32_t *bitmap = at<uint32_t>(ws, L.bitmap);
@@ -355,11 +379,24 @@ llmint8_status llmint8_linear_with_bitmaps(const uint16_t *X, int64_t M, int64_t
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsHeader *h = at<WsHeader>(ws, 0);
     const __half *Xh = reinterpret_cast<const __half *>(X);
+    const StatusRef status = next_status(h);
+    if (use_decode_path(M, K, 6.0f, max_outliers)) {
+        // few rows: the decode kernel, its outlier columns taken from the merged bitmaps
+        DecodeLaunch d = decode_launch(X, M, K, CB, SCB, N, bias, W_fp16, 6.0f, max_outliers,
+                                       Y, C_debug, h, at<DecodeTable>(ws, L.dtable),
+                                       at<uint8_t>(ws, L.dimage), status);
+        d.bitmaps = bitmaps;
+        d.n_bitmaps = n_bitmaps;
+        if (C_debug) {
+            d.Wo = at<__half>(ws, L.wo);
+            d.wo_pitch = L.pitch;
+        }
+        return run_decode(d, s);
+    }
     uint32_t *bitmap = at<uint32_t>(ws, L.bitmap);
     int32_t *idx = at<int32_t>(ws, L.idx);
     __half *Xo = at<__half>(ws, L.xo);
     __half *Wo = at<__half>(ws, L.wo);
-    const StatusRef status = next_status(h);
     cudaError_t e = launch_outlier_merge(bitmaps, n_bitmaps, K, bitmap, idx, max_outliers,
                                          &h->n_outliers, status, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
@@ -436,42 +473,41 @@ llmint8_status llmint8_workspace_outlier_weights(const void *ws, int64_t M, int6
 
 // ------------------------------------------------------------------ no-allocation call ----
 //
-// llmint8_linear_noalloc runs the decode path (the X-quantize kernel and the weight-streaming
-// kernel) on scratch that lives in this file-scope device array instead of a caller
-// workspace.  It is meant for callers that cannot allocate device memory at the call site: a
-// token-by-token decode loop that must not call cudaMalloc or cudaFree between steps (cudaFree
-// waits for the whole device), and plain C hosts that hold no device allocator of their own.
-// Nothing here allocates: no cudaMalloc, cudaFree or allocating library routine.
+// llmint8_linear_noalloc runs the decode kernel with its scratch - the 256-byte header that
+// receives the call's status words and outlier count, and the table of outlier columns and row
+// scales and the int8 image of X that the kernel's first CTA hands to the others - in this
+// file-scope device array (about 260 KiB) instead of a caller workspace.  It is meant for callers that cannot allocate device memory
+// at the call site: a token-by-token decode loop that must not call cudaMalloc or cudaFree
+// between steps (cudaFree waits for the whole device), and plain C hosts that hold no device
+// allocator of their own.  Nothing here allocates: no cudaMalloc, cudaFree or allocating
+// library routine.
 //
-// Layout of the scratch (one copy per device; the module zero-fills it when it loads):
-//   [0, 256)                         WsHeader: status words and outlier count of the last call
-//   [first 1024-aligned address ...) quantized-X operand image, decode_image_bytes(K) bytes
-//   [next 256-aligned address ...)   DecodeTables
-// Nothing in it must be zeroed between calls: every call tags the words it hands from one
-// kernel to the other, and its status words, with a fresh call epoch (the counter only grows
-// and starts above zero).  Calls in stream order are safe: the X-quantize kernel of a call
-// waits for the previous grid on its stream to finish before it writes the scratch.  Calls
+// Nothing in it needs clearing between calls: every call tags its status words and its table
+// with a fresh call epoch (the counter only grows and starts above zero), and the outlier
+// count is plain-stored by each call.  Calls in stream order are safe: the decode kernel of a
+// call writes the scratch only after the previous grid on its stream has finished.  Calls
 // that overlap - on two streams, or from two host threads without stream order between them -
-// share the one scratch of their device and race; their outputs are undefined.
+// share the one scratch of their device and race on its table; their outputs are undefined.
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 160 * 1024;
+// the header, the table (256-byte aligned), then the operand image (1024-byte aligned) of the
+// largest decode shape: 16 rows x 16384 columns
+constexpr size_t kNoAllocTableOffset = sizeof(WsHeader);
+constexpr size_t kNoAllocImageOffset =
+    (size_t)align_up((int64_t)(kNoAllocTableOffset + sizeof(DecodeTable)), 1024);
+constexpr size_t kNoAllocScratchBytes =
+    kNoAllocImageOffset + (size_t)decode_image_bytes(kDecodeMaxM, kDecodeMaxK);
 
-constexpr size_t noalloc_image_offset_bound() { return 1024; }   // header + worst alignment pad
-constexpr size_t noalloc_need_bound() {
-    return noalloc_image_offset_bound() + (size_t)decode_image_bytes(kDecodeMaxK) + 256 +
-           sizeof(DecodeTables);
-}
-static_assert(noalloc_need_bound() <= kNoAllocScratchBytes,
-              "the no-allocation scratch holds the decode path's largest shape");
-
-__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+__device__ __align__(1024) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
 
-// Set-up, once per device, with that device current: the scratch's device address.
+// Set-up, once per device, with that device current: the scratch's device address (the
+// array's name in host code is only a host-side stand-in).  The address is cached for the
+// life of the process; a device reset (cudaDeviceReset) invalidates it and is not supported
+// between calls of this entry point.
 cudaError_t noalloc_scratch(void **ptr) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
@@ -504,39 +540,18 @@ llmint8_status llmint8_linear_noalloc(const uint16_t *X, int64_t M, int64_t K, c
     if (isnan(threshold)) return LLMINT8_ERR_INVALID_ARG;
     if (!shape_ok_mk(M, K) || !shape_ok_n(N)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
     if (max_outliers < 0 || max_outliers > K) return LLMINT8_ERR_INVALID_ARG;
-    // only what the decode path covers fits the fixed scratch
+    // only what the decode path covers runs without a workspace
     if (!use_decode_path(M, K, threshold, max_outliers)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
 
     void *base = nullptr;
     if (noalloc_scratch(&base) != cudaSuccess) return LLMINT8_ERR_CUDA;
-    const uintptr_t b = reinterpret_cast<uintptr_t>(base);
-    const size_t image = (size_t)(align_up((int64_t)(b + sizeof(WsHeader)), 1024) - (int64_t)b);
-    const size_t tables = (size_t)align_up((int64_t)(image + decode_image_bytes(K)), 256);
-    if (tables + sizeof(DecodeTables) > kNoAllocScratchBytes) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
-
     WsHeader *h = at<WsHeader>(base, 0);
-    DecodeLaunch d;
-    d.X = reinterpret_cast<const __half *>(X);
-    d.CB = CB;
-    d.SCB = SCB;
-    d.W16 = reinterpret_cast<const __half *>(W_fp16);
-    d.bias = reinterpret_cast<const __half *>(bias);
-    d.Y = reinterpret_cast<__half *>(Y);
-    d.C_debug = nullptr;
-    d.Wo = nullptr;
-    d.wo_pitch = 0;
-    d.count = &h->n_outliers;
-    d.image = at<uint8_t>(base, image);
-    d.tables = at<DecodeTables>(base, tables);
-    d.status = next_status(h);
-    d.M = M;
-    d.N = N;
-    d.K = K;
-    d.cap = max_outliers;
-    d.threshold = threshold;
-    d.timeout_ns = g_timeout_ns.load();
+    const DecodeLaunch d = decode_launch(X, M, K, CB, SCB, N, bias, W_fp16, threshold,
+                                         max_outliers, Y, nullptr, h,
+                                         at<DecodeTable>(base, kNoAllocTableOffset),
+                                         at<uint8_t>(base, kNoAllocImageOffset), next_status(h));
     if (scratch_out) *scratch_out = base;
-    return from_cuda(launch_decode(d, static_cast<cudaStream_t>(stream)));
+    return run_decode(d, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -1,37 +1,32 @@
 // Decode path of the LLM.int8() layer (few activation rows, M <= 16).
 //
-// At decode sizes the layer is bound by streaming the int8 weight CB from HBM once, and
-// everything else must hide under that stream.  Two kernels:
+// At decode sizes the layer is bound by streaming the int8 weight CB from HBM once; the rest
+// must hide under that stream.  One kernel per call, one CTA per SM:
 //
-// llmint8_decode_quantize_kernel (one cluster of 8 CTAs x 1024 threads) quantizes X once:
-//   one thread per (row, 8-column chunk), each warp holding all 16 rows of two chunks, CTA r
-//   of the cluster 1/8 of the columns.  The outlier bits of a chunk (|x| >= threshold in any
-//   row) are an OR across 16 lanes; the row maxima over the regular columns reduce in
-//   registers, across warps, and across the cluster through distributed shared memory
-//   (one hardware cluster barrier); the int8 codes go into the workspace as a byte-exact
-//   image of the tensor-core operand (16 rows, 128-byte swizzled K-major blocks, outlier
-//   columns and padding 0), next to a table of SCA and the ascending outlier columns.  It
-//   lets its dependent launch as soon as the work before it in the stream is complete.
-//
-// llmint8_decode_kernel (one CTA per 128-row weight tile, programmatic dependent launch):
-//   warp 0        TMA producer: streams 128-row x 128-byte tiles of CB (16 KB) through a ring
-//                 of shared-memory stages from its first cycle - it needs nothing from X - and
-//                 asks L2 for the rest of its first tile as well, so that HBM keeps streaming
-//                 while the MMA waits for the quantized X (every weight byte is still read
-//                 from HBM once per call; the later stage loads find it in L2);
-//   warp 1        waits until the quantize kernel publishes (an acquire on the call epoch it
-//                 stores last), bulk-copies the operand image and the table into shared
-//                 memory, then issues tcgen05.mma kind::i8
-//                 with the weight tile as the 128-row operand and the quantized X as the
-//                 16-column operand: D[n, m] = sum_k CB[n, k] Xq[m, k] into a 128 x 16 int32
-//                 TMEM accumulator (double-buffered over tiles);
-//   warps 4..7    epilogue: while the weights stream, each thread (one output row n) builds
-//                 sum_{j in O} X[m, O_j] * W_o[n, O_j] + bias_n (the fp16 outlier part of the
-//                 decomposition, weights from the bytes of the outlier columns) and its scale;
-//                 after the tile's last MMA: D -> registers, y = D * SCA_m * SCB_n / 127^2 +
-//                 that part -> fp16.
-// Same method and rounding as the GEMM path (LLM.int8() summary, sections الابتكار الثاني
-// and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded.
+//   CTA 0, the quantizer: waits for the previous grid on the stream (X may be its output),
+//       reads X once and finds the outlier columns (|x| >= threshold in any row, an OR over
+//       the lanes holding a column's rows) and the row maxima over the regular columns,
+//       lists the outlier columns in ascending order and publishes that table (row absmax,
+//       per-chunk outlier bits, the list) in the workspace with a release store of the call
+//       number; then it exits, so the next call's quantizer can take its SM early.
+//   CTAs 1.., the streamers, each own a band of Rt consecutive weight rows (output channels);
+//       Rt = ceil(N / streamers) rounded up to 8 rows (at most 128), so the bands spread
+//       evenly over every SM and no streamer waits on another:
+//     warp 0      TMA producer: 128-byte k-blocks of the band through a shared-memory ring;
+//     warps 2, 3  wait for the table, then write the int8 codes of X (absmax quantization with
+//                 the published row scales, outlier columns 0) one k-block at a time into a
+//                 small ring of operand images (K-major, 128-byte swizzle), in the order the
+//                 MMAs consume them, re-reading that block of X from L2;
+//     warp 1      one thread issues tcgen05.mma kind::i8 with the weight rows as the 128-row
+//                 operand and the image block as the 16-column operand, D[n, m] = sum_k
+//                 CB[n, k] Xq[m, k], into int32 TMEM sub-accumulators;
+//     warps 4..7  epilogue: while the weights stream, each thread (one output channel n)
+//                 forms the fp16 outlier part sum_{j in O} X[m, O_j] * W_o[n, O_j] + bias_n and
+//                 its scale; after the last MMA: y = D * SCA_m * SCB_n / 127^2 + that part.
+// Every loop is rolled (the SM fetches little code while the weight stream keeps the memory
+// system busy), and the operand image is never held whole, so K is not bound by shared
+// memory.  Same method and rounding as the GEMM path (LLM.int8() summary, sections
+// الابتكار الثاني and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include <cstddef>
@@ -45,25 +40,24 @@ namespace llmint8 {
 namespace {
 
 constexpr int DM = kDecodeMaxM;         // activation rows held (MMA N)
-constexpr int DBM = 128;                // weight rows per tile (MMA M)
-constexpr int DBK = 128;                // bytes of K per stage
-constexpr int DSTAGE = DBM * DBK;       // 16 KB
+constexpr int DMMA_M = 128;             // MMA rows; rows of the MMA past the band are discarded
+constexpr int DBK = 128;                // bytes of K per k-block
 constexpr int DTHREADS = 256;
-constexpr int DMAX_STAGES = 12;
+constexpr int DWARPS = DTHREADS / 32;
+constexpr int DKS = 2;                  // k-blocks per weight stage (one wait, one commit)
+constexpr int DMAX_STAGES = 32;
+constexpr int DIMG_MAX = 32;            // operand-image stages at most ...
+constexpr int DIMG_BYTES = 65536;       // ... and the shared memory they take at most
+constexpr int QKB = 8;                  // k-blocks per quantizer CTA (aim)
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
-constexpr int QTHREADS = 1024;          // quantize kernel: one cluster of QCL CTAs
-constexpr int QWARPS = QTHREADS / 32;
-constexpr int QCL = 8;
-// chunk pairs (16 columns) per warp: K <= kDecodeMaxK keeps every item in registers
-constexpr int QKEEP = (kDecodeMaxK / 16 / QCL + QWARPS - 1) / QWARPS;
-// k-blocks of a CTA's first tile requested into L2 ahead of the stage ring, so that HBM keeps
-// streaming while the first MMA waits for the quantized X
-constexpr int kPrefetchBlocks = 64;
-// Independent int32 accumulators per tile: k-block it accumulates into sub-accumulator
-// it % DSUB, so consecutive MMAs do not wait on each other's result (a 128 x 16 MMA is too
-// short to hide the accumulate dependency); the epilogue adds them (exact in int32).
-constexpr int DSUB = 4;
-constexpr uint32_t DTMEM_COLS = 2 * DSUB * kDecodeMaxM;   // double-buffered over tiles
+// Two MMA issuers per CTA (warps 1 and 3): issuer i takes the weight stages j with
+// j % 2 == i of every tile, into its own int32 accumulator of 16 columns; the epilogue adds the
+// two (exact).  Measured on B200: one thread issues a 128 x 16 x 32 MMA about every 60 cycles,
+// two threads together one every 40 (the tensor pipe's floor for this shape), and a
+// tcgen05.commit costs about 150 cycles; with one issuer the k-loop, not HBM, bounded a call.
+// Each issuer issues 8 MMAs per wait and per commit.  Accumulators are double-buffered over
+// tiles: column (acc * 2 + issuer) * 16.
+constexpr uint32_t DTMEM_COLS = 64;
 
 __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&v);
@@ -75,26 +69,20 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     }
 }
 
-// Byte offset of Xq[m, k0 ..] (k0 a multiple of 8) in the 128-byte-swizzled K-major layout:
-// per 128-column block, `rows` (16, or 8 when M <= 8) rows of 128 bytes in 8-row atoms of
-// 1024 bytes; the 16-byte chunk index within a row is XORed with (row mod 8).  With 8 rows
-// the MMA's second 8-row group is one shared all-zero atom after the last block (see
-// image_desc), so the image takes half the shared memory and the weight ring two more stages.
-__device__ __forceinline__ uint32_t xq_offset(int m, int k0, int rows) {
-    const int kb = k0 >> 7, c = k0 & 127;
-    return (uint32_t)(kb * (rows * 128) + (m >> 3) * 1024 + (m & 7) * 128 +
-                      ((((c >> 4) ^ (m & 7)) << 4) | (c & 15)));
+// Byte offset of Xq[m, c0 ..] (c0 a multiple of 8, < 128) in one k-block of the
+// 128-byte-swizzled K-major image: `rows` (16, or 8 when M <= 8) rows of 128 bytes in 8-row
+// atoms of 1024 bytes; the 16-byte chunk index within a row is XORed with (row mod 8).  With
+// 8 rows the MMA's second 8-row group is one shared all-zero atom after the image ring (see
+// image_desc), which halves the ring's shared memory.
+__device__ __forceinline__ uint32_t xq_offset(int m, int c0) {
+    return (uint32_t)((m >> 3) * 1024 + (m & 7) * 128 + ((((c0 >> 4) ^ (m & 7)) << 4) | (c0 & 15)));
 }
 
 __host__ __device__ constexpr int image_rows(int M) { return M <= 8 ? 8 : kDecodeMaxM; }
-// Bytes of the image: the blocks, plus the shared zero atom when it has 8 rows.
-__host__ __device__ constexpr int image_bytes(int kblocks, int rows) {
-    return kblocks * rows * 128 + (rows == 8 ? 1024 : 0);
-}
 
-// Descriptor of the image's block at `saddr` (+ k offset) for the 16-column MMA operand: the
-// two 8-row groups are `sbo` bytes apart (1024 in the 16-row image; in the 8-row image the
-// distance to the zero atom, so that rows 8..15 read as zeros).
+// Descriptor of an image block at `saddr` (+ k offset) for the 16-column MMA operand: the two
+// 8-row groups are `sbo` bytes apart (1024 in a 16-row block; for an 8-row block the distance
+// to the zero atom, so that rows 8..15 read as zeros).
 __device__ __forceinline__ uint64_t image_desc(uint32_t saddr, uint32_t sbo) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);      // start address / 16
@@ -105,201 +93,84 @@ __device__ __forceinline__ uint64_t image_desc(uint32_t saddr, uint32_t sbo) {
     return d;
 }
 
-__device__ __forceinline__ uint32_t outlier_bits(const float *f, float threshold) {
-    uint32_t b = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) b |= (fabsf(f[e]) >= threshold ? 1u : 0u) << e;
-    return b;
+// int8 code of x with multiplier s: round_half_even(fl32(x * s)) as the low byte of a float.
+// fl32(y + 1.5 * 2^23) for |y| < 2^22 is 1.5 * 2^23 + (y rounded to an integer, ties to
+// even), whose low significand bits are that integer in two's complement.  |y| <= 127 here
+// (|x| <= absmax of its row and s = fl32(127 / absmax)), so no clamp is ever active.
+__device__ __forceinline__ uint32_t code_byte(float x, float s) {
+    return __float_as_uint(__fadd_rn(__fmul_rn(x, s), 12582912.0f)) & 0xffu;
 }
 
-__device__ __forceinline__ float masked_max(const float *f, uint32_t skip, float r) {
+// Eight codes packed little-endian; a set bit in `skip` gives 0.
+__device__ __forceinline__ uint2 quant8(const float *f, float s, uint32_t skip) {
+    uint32_t b[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-        if (!((skip >> e) & 1u)) r = fmaxf(r, fabsf(f[e]));
-    return r;
-}
-
-// Eight absmax-quantized int8 codes, packed little-endian; a set bit in `skip` gives 0.
-__device__ __forceinline__ uint2 quant8(const float *f, float mul, uint32_t skip) {
-    uint32_t lo = 0, hi = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        int q = 0;
-        if (!((skip >> e) & 1u)) q = max(-127, min(127, __float2int_rn(__fmul_rn(f[e], mul))));
-        const uint32_t b = (uint32_t)(q & 0xff);
-        if (e < 4) lo |= b << (8 * e);
-        else hi |= b << (8 * (e - 4));
-    }
+    for (int e = 0; e < 8; ++e) b[e] = code_byte(((skip >> e) & 1u) ? 0.0f : f[e], s);
+    const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040),
+                                    0x5410);
+    const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040),
+                                    0x5410);
     return make_uint2(lo, hi);
 }
 
-struct QArgs {
-    const __half *X;
-    int M, K, cap;
-    float threshold;
-    uint8_t *image;
-    DecodeTables *tables;
-    int32_t *count;
-    StatusRef status;
-    unsigned long long epoch;
-    int rows;                                // image rows: 16, or 8 when M <= 8
-};
-
-// One cluster of QCL CTAs.  CTA r owns the chunk pairs [r*PP, (r+1)*PP); one thread per
-// (row, chunk) item, its values kept in registers between the two passes.
-__global__ void __launch_bounds__(QTHREADS, 1) llmint8_decode_quantize_kernel(const QArgs a) {
-    // launched as a programmatic dependent of whatever precedes it in the stream: wait for it
-    // before touching X or the workspace, then let the weight-streaming kernel launch
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    __shared__ float part[QCL][DM];          // row maxima of every CTA of the cluster
-    __shared__ uint32_t pmax[DM];            // this CTA's (float bits, >= 0: int order)
-    __shared__ float mult[DM];
-    __shared__ uint8_t flags_all[kDecodeMaxK / 8];   // CTA 0: outlier bits of every chunk
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int m = lane & 15;                 // the row this thread handles
-    const int half = lane >> 4;              // which chunk of the warp's pair
-    const uint32_t r = cluster_ctarank();
-    const int nchunks = a.K / 8;
-    const int npairs = nchunks / 2;          // K is a multiple of 16
-    const int pp = (npairs + QCL - 1) / QCL;
-    const int p0 = (int)r * pp, p1 = min(npairs, p0 + pp);
-    const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
-
-    uint4 v[QKEEP];
-#pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        const int p = p0 + warp + i * QWARPS;
-        v[i] = (p < p1 && m < a.M) ? __ldg(X4 + (int64_t)m * nchunks + 2 * p + half)
-                                   : make_uint4(0, 0, 0, 0);
-    }
-    if (t < DM) pmax[t] = 0u;
-    __syncthreads();
-
-    // pass 1: outlier bits of each chunk (OR over its 16 lanes = rows), published to CTA 0;
-    // row maxima over the regular columns
-    uint32_t fl[QKEEP];
-    float rm = 0.0f;
-    const uint32_t flags0 = map_to_rank(smem_addr(flags_all), 0);
-#pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        fl[i] = 0;
-        const int p = p0 + warp + i * QWARPS;
-        if (p < p1) {                        // uniform over the warp
-            float f[8];
-            unpack8(v[i], f);
-            uint32_t b = outlier_bits(f, a.threshold);
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, o);
-            fl[i] = b;
-            if (m == 0) st_cluster_u8(flags0 + (uint32_t)(2 * p + half), b);
-            rm = masked_max(f, b, rm);
-        }
-    }
-    rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 16));
-    if (half == 0 && m < a.M && rm > 0.0f) atomicMax(&pmax[m], __float_as_uint(rm));
-    __syncthreads();
-    if (t < DM) {
-        const uint32_t dst = smem_addr(&part[r][t]);
-        for (int rr = 0; rr < QCL; ++rr) st_cluster_u32(map_to_rank(dst, (uint32_t)rr), pmax[t]);
-    }
-    // every CTA's flags and partial maxima are in place after this
-    cluster_barrier_all();
-
-    if (t < DM) {
-        float amax = 0.0f;
-        for (int rr = 0; rr < QCL; ++rr) amax = fmaxf(amax, part[rr][t]);
-        mult[t] = (t < a.M && amax > 0.0f) ? __fdiv_rn(127.0f, amax) : 0.0f;
-        if (r == 0) a.tables->sca[t] = amax;
-    }
-    __syncthreads();
-
-    // pass 2: every (row, chunk) of this CTA into the operand image; rows >= M, all-zero rows
-    // and outlier columns are written as 0
-    const float mul = mult[m];
-#pragma unroll
-    for (int i = 0; i < QKEEP; ++i) {
-        const int p = p0 + warp + i * QWARPS;
-        if (p < p1) {
-            const int c = 2 * p + half;
-            uint2 q = make_uint2(0, 0);
-            if (mul > 0.0f) {
-                float f[8];
-                unpack8(v[i], f);
-                q = quant8(f, mul, fl[i]);
-            }
-            if (m < a.rows) *reinterpret_cast<uint2 *>(a.image + xq_offset(m, c * 8, a.rows)) = q;
-        }
-    }
-    // every CTA's part of the image is written before CTA 0 publishes it
-    __threadfence();
-    __syncwarp();
-    cluster_barrier_all();
-    if (r != 0) return;   // nothing of this CTA is read by its peers any more
-
-    // CTA 0: padding columns of the image (and its zero atom), ascending outlier list, count,
-    // status
-    const int kpad_chunks = (a.K + 127) / 128 * 16;
-    for (int i = t; i < (kpad_chunks - nchunks) * a.rows; i += QTHREADS) {
-        const int c = nchunks + i / a.rows, mm = i % a.rows;
-        *reinterpret_cast<uint2 *>(a.image + xq_offset(mm, c * 8, a.rows)) = make_uint2(0, 0);
-    }
-    if (a.rows == 8 && t < 128)
-        reinterpret_cast<uint2 *>(a.image + (kpad_chunks / 16) * 1024)[t] = make_uint2(0, 0);
-    if (warp == 0) {
-        const int per = (nchunks + 31) / 32;
-        const int c0 = lane * per, c1 = min(nchunks, c0 + per);
-        int cnt = 0;
-        for (int c = c0; c < c1; ++c) cnt += __popc(flags_all[c]);
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        int pos = incl - cnt;
-        for (int c = c0; c < c1; ++c) {
-            uint32_t b = flags_all[c];
-            while (b) {
-                const int e = __ffs(b) - 1;
-                b &= b - 1;
-                if (pos < a.cap) a.tables->idx[pos] = c * 8 + e;
-                ++pos;
-            }
-        }
-        const int total = __shfl_sync(0xffffffffu, incl, 31);
-        if (lane == 0) {
-            a.tables->n_out = min(total, a.cap);
-            *a.count = total;
-            a.status.set(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
-        }
-    }
-    // publish: the image and table are complete (the dependent kernel bulk-copies them)
-    __threadfence();
-    fence_proxy_async_global();
-    __syncthreads();
-    if (t == 0)
-        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(&a.tables->ready), "l"(a.epoch)
-                     : "memory");
+// L2 eviction policy of the weight stream: it is read once per call (evict first).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void tma_load_2d_policy(uint32_t dst, const CUtensorMap *tm, int x, int y,
+                                                   uint32_t bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar), "l"(pol)
+        : "memory");
 }
 
+// Packed-half helpers on raw bits: |x| (clear the sign bits), |x| >= t per half (0xffff
+// where true), max per half.  fp16 comparisons and maxima are exact.
+__device__ __forceinline__ uint32_t habs2_bits(uint32_t v) { return v & 0x7fff7fffu; }
+__device__ __forceinline__ uint32_t hge2_bits(uint32_t a, uint32_t t) {
+    return __hge2_mask(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&t));
+}
+__device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
+    const __half2 r = __hmax2(*reinterpret_cast<const __half2 *>(&a),
+                              *reinterpret_cast<const __half2 *>(&b));
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+// Shared memory of the quantizer CTA.
+struct QShared {
+    uint64_t xbar;                       // this quantizer's columns of X have landed
+    int ok;                              // every quantizer's partials arrived in time
+    float wmax[DWARPS][DM];              // per-warp partial row maxima
+    float sca[DM];                       // row absmax over all regular columns
+    float mult[DM];                      // fl32(127 / absmax), 0 for an all-zero row
+    int wsum[DWARPS];                    // per-warp outlier counts (list scan)
+    uint8_t flags[kDecodeMaxK / 8];      // outlier bits of each 8-column chunk
+};
+// A quantizer's shared memory: QShared, then M rows x its columns of X, then their int8 image.
+constexpr int QX_OFF = 4096;
+static_assert(sizeof(QShared) <= QX_OFF, "quantizer tables fit before the staged X");
+
+// Shared memory tail of a streamer CTA.
 struct DTail {
     uint64_t full[DMAX_STAGES];
     uint64_t empty[DMAX_STAGES];
-    uint64_t acc_full[2];
+    uint64_t ifull[DIMG_MAX];            // an image stage has landed
+    uint64_t iempty[DIMG_MAX];           // ... and been consumed by the MMAs
+    uint64_t acc_full[2];                // both issuers (one when a tile has one stage) are done
     uint64_t acc_empty[2];
-    uint64_t mma_done;
-    uint64_t xbar;                       // operand image and table have landed
+    uint64_t mma_done[2];
+    uint64_t tbar;                       // the quantizer's table is published (one poller)
     uint32_t tmem_base;
     int abort_flag;
-    alignas(16) DecodeTables tab;
-    alignas(16) __half xo[kDecodeMaxOutliers * DM];   // X at the outlier columns, [j][m]
+    int32_t idx[kDecodeMaxOutliers];     // outlier columns, ascending (epilogue copy)
 };
-static_assert(offsetof(DTail, tab) % 16 == 0, "the table is a bulk-copy destination");
-static_assert(offsetof(DTail, xbar) % 8 == 0, "mbarriers are 8-byte aligned");
+static_assert(offsetof(DTail, acc_full) % 8 == 0, "mbarriers are 8-byte aligned");
 
 struct DArgs {
-    unsigned long long epoch;
     const __half *X;
     const int8_t *CB;
     const float *SCB;
@@ -309,73 +180,330 @@ struct DArgs {
     int32_t *C_debug;
     __half *Wo;                          // [N, wo_pitch] or null
     int64_t wo_pitch;
-    const uint8_t *image;
-    const DecodeTables *tables;
+    const uint32_t *bitmaps;             // [n_bitmaps][ceil(K/32)] given outlier set, or null
+    int n_bitmaps;
+    int32_t *count;
+    DecodeTable *table;                  // workspace: what the quantizer publishes
+    uint8_t *image;                      // workspace: the int8 operand image, block by block
     StatusRef status;
-    int M, N, K;
-    int stages;
-    int kblocks;
-    int tiles;
-    uint32_t xq_off;                     // byte offsets in shared memory
-    uint32_t tail_off;
-    uint64_t timeout_ns;
+    unsigned long long epoch;
+    int M, N, K, cap;
+    float threshold;
+    uint32_t thr2;                       // the threshold rounded up to fp16, in both halves:
+                                         // for an fp16 x, |x| >= threshold iff |x| >= that
     int rows;                            // image rows: 16, or 8 when M <= 8
+    int Rt;                              // weight rows per tile (band)
+    int tiles, kblocks, stages;
+    int nq, bpq;                         // quantizer CTAs, k-blocks per quantizer
+    int nst;                             // weight stages per tile: ceil(kblocks / DKS)
+    int nistage;                         // operand-image stages (DKS blocks each) of a streamer
+    int resident;                        // the image stages hold every k-block: filled once
+    uint32_t tail_off, xo_off, ring_off; // byte offsets in shared memory (image ring at 0)
+    uint64_t timeout_ns;
 };
+
+// ------------------------------------------------------------------ the quantizers ----------
+// Quantizer q (CTA q < nq) owns k-blocks [q * bpq, (q + 1) * bpq) of X.  Its columns come into
+// shared memory by bulk copies, one per row.  Pass 1: thread t takes the 8-column chunks t,
+// t + 256, ... of every row, ORs the rows' |x| >= threshold into the chunk's outlier bits and
+// keeps per-row maxima of |x| over the regular columns (packed fp16 compares and maxima,
+// exact); the quantizer publishes its bits and row maxima.  Every quantizer then takes the
+// row maxima of all of them (the row absmax over all regular columns), and pass 2 writes the
+// int8 codes of its columns into a shared-memory image, k-block by k-block in the layout the
+// streamers copy into their own shared memory; one bulk store puts it in the workspace.
+// Quantizer 0 also lists the outlier columns in ascending order.
+__device__ __forceinline__ void bulk_store_1d(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(src), "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_store_wait() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void release_word(unsigned long long *w, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(w), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long acquire_word(const unsigned long long *w) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
+    return v;
+}
+// Bounded, backed-off poll (one thread) until every word w[0..n) holds v; false on timeout.
+__device__ bool poll_words(const unsigned long long *w, int n, unsigned long long v,
+                           StatusRef status, uint64_t timeout_ns, volatile int *abort_flag) {
+    const uint64_t t0 = global_timer_ns();
+    int i = 0;
+    for (uint32_t it = 0;; ++it) {
+        while (i < n && acquire_word(w + i) == v) ++i;
+        if (i == n) return true;
+        __nanosleep(200);
+        if ((it & 15u) == 15u) {
+            if (abort_flag && *abort_flag) return false;
+            if (global_timer_ns() - t0 > timeout_ns) {
+                if (abort_flag) *abort_flag = 1;
+                status.timed_out();
+                return false;
+            }
+        }
+    }
+}
+
+__device__ void quantize_x(const DArgs &a, uint8_t *smem) {
+    QShared *q = reinterpret_cast<QShared *>(smem);
+    const int qi = blockIdx.x;
+    const int kb0 = qi * a.bpq, kb1 = min(a.kblocks, kb0 + a.bpq);
+    const int c0 = kb0 * DBK;                             // first column of this quantizer
+    const int w = min(a.K, kb1 * DBK) - c0;               // its columns (a multiple of 16)
+    uint8_t *xs = smem + QX_OFF;                          // [M][w] fp16
+    uint8_t *is = xs + (size_t)a.M * a.bpq * DBK * 2;     // image of its k-blocks
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nchunks = a.K / 8;
+    const int nwords = (a.K + 31) / 32;
+    const uint32_t xbar = smem_addr(&q->xbar);
+    if (threadIdx.x == 0) {
+        mbar_init(xbar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(xbar, (uint32_t)(a.M * w * 2));
+        for (int m = 0; m < a.M; ++m)
+            bulk_load_1d(smem_addr(xs + (size_t)m * w * 2), a.X + (int64_t)m * a.K + c0,
+                         (uint32_t)(w * 2), xbar);
+    }
+    __syncthreads();
+    // bounded like every wait; a slice that never lands leaves nothing published
+    if (!drain_wait(xbar, 0, a.status)) return;
+
+    // pass 1
+    uint32_t rmax[DM];                        // per row, max |x| over this thread's columns
+#pragma unroll
+    for (int m = 0; m < DM; ++m) rmax[m] = 0u;
+    for (int c = threadIdx.x; c < w / 8; c += DTHREADS) {
+        const int cg = c0 / 8 + c;                    // chunk index in the whole row
+        uint4 v[DM];
+#pragma unroll
+        for (int m = 0; m < DM; ++m)
+            v[m] = m < a.M ? *reinterpret_cast<const uint4 *>(xs + (size_t)m * w * 2 + c * 16)
+                           : make_uint4(0, 0, 0, 0);
+        uint32_t col[4];                              // 0xffff per outlier half
+        if (a.bitmaps) {
+            uint32_t wd = 0;
+            for (int r = 0; r < a.n_bitmaps; ++r)
+                wd |= __ldg(a.bitmaps + (int64_t)r * nwords + (cg >> 2));
+            const uint32_t b = (wd >> ((cg & 3) * 8)) & 0xffu;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                col[e] = (((b >> (2 * e)) & 1u) ? 0x0000ffffu : 0u) |
+                         (((b >> (2 * e + 1)) & 1u) ? 0xffff0000u : 0u);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) col[e] = 0u;
+#pragma unroll
+            for (int m = 0; m < DM; ++m) {
+                const uint32_t *wv = reinterpret_cast<const uint32_t *>(&v[m]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) col[e] |= hge2_bits(habs2_bits(wv[e]), a.thr2);
+            }
+        }
+        uint32_t b = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            b |= ((col[e] & 1u) << (2 * e)) | ((col[e] >> 16 & 1u) << (2 * e + 1));
+        q->flags[c] = (uint8_t)b;
+        a.table->flags[cg] = (uint8_t)b;
+#pragma unroll
+        for (int m = 0; m < DM; ++m) {
+            const uint32_t *wv = reinterpret_cast<const uint32_t *>(&v[m]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                rmax[m] = hmax2_bits(rmax[m], habs2_bits(wv[e]) & ~col[e]);
+        }
+    }
+    // this quantizer's row maxima: over the two halves, the warp's lanes, then the warps
+#pragma unroll
+    for (int m = 0; m < DM; ++m) {
+        uint32_t r = rmax[m];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) r = hmax2_bits(r, __shfl_xor_sync(0xffffffffu, r, o));
+        const __half2 h = *reinterpret_cast<const __half2 *>(&r);
+        if (lane == 0) q->wmax[warp][m] = fmaxf(__low2float(h), __high2float(h));
+    }
+    __syncthreads();
+    if (threadIdx.x < DM) {
+        float amax = 0.0f;
+        for (int wi = 0; wi < DWARPS; ++wi) amax = fmaxf(amax, q->wmax[wi][threadIdx.x]);
+        a.table->part[qi][threadIdx.x] = amax;
+    }
+    // publish the bits and row maxima, then take every quantizer's
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        release_word(&a.table->pready[qi], a.epoch);
+        q->ok = poll_words(a.table->pready, a.nq, a.epoch, a.status, a.timeout_ns, nullptr) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!q->ok) return;
+    if (threadIdx.x < DM) {
+        float amax = 0.0f;
+        for (int r = 0; r < a.nq; ++r) amax = fmaxf(amax, __ldcg(&a.table->part[r][threadIdx.x]));
+        if ((int)threadIdx.x >= a.M) amax = 0.0f;
+        q->sca[threadIdx.x] = amax;
+        q->mult[threadIdx.x] = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    }
+    __syncthreads();
+
+    // pass 2: item (block, 16-column group, row) -> 16 codes, one 16-byte store
+    const uint32_t blk_bytes = (uint32_t)a.rows * DBK;
+    const int nblk = kb1 - kb0;
+    for (int i = threadIdx.x; i < nblk * 8 * a.rows; i += DTHREADS) {
+        const int grp = i & 7, m = (i >> 3) % a.rows, blk = (i >> 3) / a.rows;
+        uint4 code = make_uint4(0, 0, 0, 0);
+        if (m < a.M) {
+            const int cl = blk * 16 + grp * 2;             // chunk within this slice
+            const uint32_t b0 = cl * 8 < w ? q->flags[cl] : 0xffu;
+            const uint32_t b1 = cl * 8 + 8 < w ? q->flags[cl + 1] : 0xffu;
+            const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)m * w * 2 + cl * 16);
+            const uint4 v0 = cl * 8 < w ? src[0] : make_uint4(0, 0, 0, 0);
+            const uint4 v1 = cl * 8 + 8 < w ? src[1] : make_uint4(0, 0, 0, 0);
+            float f[8];
+            unpack8(v0, f);
+            const uint2 lo = quant8(f, q->mult[m], b0);
+            unpack8(v1, f);
+            const uint2 hi = quant8(f, q->mult[m], b1);
+            code = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
+        *reinterpret_cast<uint4 *>(is + blk * blk_bytes + xq_offset(m, grp * 16)) = code;
+    }
+    // the image is read by the bulk store (async proxy)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        bulk_store_1d(a.image + (size_t)kb0 * blk_bytes, smem_addr(is), (uint32_t)nblk * blk_bytes);
+        bulk_store_wait();
+        fence_proxy_async_global();
+        release_word(&a.table->iready[qi], a.epoch);
+    }
+    if (qi != 0) return;
+
+    // quantizer 0: the row scales and the ascending list of outlier columns (every
+    // quantizer's bits are published: pready above)
+    if (threadIdx.x < DM) a.table->sca[threadIdx.x] = q->sca[threadIdx.x];
+    const int cpt = (nchunks + DTHREADS - 1) / DTHREADS;
+    const int l0 = min(nchunks, (int)threadIdx.x * cpt), l1 = min(nchunks, l0 + cpt);
+    int cnt = 0;
+    for (int c = l0; c < l1; ++c) cnt += __popc((uint32_t)__ldcg(&a.table->flags[c]));
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) q->wsum[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int wi = 0; wi < DWARPS; ++wi) {
+        const int sm = q->wsum[wi];
+        before += wi < warp ? sm : 0;
+        total += sm;
+    }
+    int pos = before + incl - cnt;
+    for (int c = l0; c < l1; ++c) {
+        uint32_t b = __ldcg(&a.table->flags[c]);
+        while (b) {
+            const int e = __ffs(b) - 1;
+            b &= b - 1;
+            if (pos < a.cap) a.table->idx[pos] = c * 8 + e;
+            ++pos;
+        }
+    }
+    if (threadIdx.x == 0) {
+        a.table->total = total;
+        a.table->n_out = min(total, a.cap);
+        *a.count = total;
+        a.status.set(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) release_word(&a.table->ready, a.epoch);
+}
 
 __global__ void __launch_bounds__(DTHREADS, 1)
 llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    DTail *tail = reinterpret_cast<DTail *>(smem + a.tail_off);
-    uint8_t *xq = smem + a.xq_off;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if ((int)blockIdx.x < a.nq) {
+        // the next call's kernel may launch now; this one waits for the previous grid
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        quantize_x(a, smem);
+        return;
+    }
+
+    uint8_t *img = smem;                          // nistage x DKS blocks (+ zero atom)
+    DTail *tail = reinterpret_cast<DTail *>(smem + a.tail_off);
+    __half *xo = reinterpret_cast<__half *>(smem + a.xo_off);     // [j][m]
+    uint8_t *ring = smem + a.ring_off;
     const int S = a.stages;
+    const uint32_t stage_bytes = (uint32_t)DKS * a.Rt * DBK;
+    const uint32_t img_bytes = (uint32_t)a.rows * DBK;            // one k-block of the image
+    const int band0 = blockIdx.x - a.nq, bands = gridDim.x - a.nq;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(smem_addr(&tail->full[s]), 1);
             mbar_init(smem_addr(&tail->empty[s]), 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_addr(&tail->acc_full[s]), 1);
-            mbar_init(smem_addr(&tail->acc_empty[s]), 4);
+        for (int s = 0; s < a.nistage; ++s) {
+            mbar_init(smem_addr(&tail->ifull[s]), 1);
+            mbar_init(smem_addr(&tail->iempty[s]), 1);
         }
-        mbar_init(smem_addr(&tail->mma_done), 1);
-        mbar_init(smem_addr(&tail->xbar), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_addr(&tail->acc_full[s]), a.nst >= 2 ? 2 : 1);
+            mbar_init(smem_addr(&tail->acc_empty[s]), 4);
+            mbar_init(smem_addr(&tail->mma_done[s]), 1);
+        }
+        mbar_init(smem_addr(&tail->tbar), 1);
         tail->abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmCB);
     }
     if (warp == 1) tmem_alloc(smem_addr(&tail->tmem_base), DTMEM_COLS);
-    // the next call's first kernel may launch now (it waits for this grid before it reads)
+    // the next call's kernel may launch now (it waits for this grid before it reads or
+    // writes anything); this one waits for the previous grid before it touches memory
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tail->tmem_base;
     const BoundedWait wait{&tail->abort_flag, a.status, a.timeout_ns};
 
+    // stage j of a tile covers k-blocks DKS * sj .. (sj = j rotated by a tile-dependent
+    // offset, so that the CTAs streaming at the same moment read different column ranges of
+    // the 2^n-strided weight rows); the last one may hold a single k-block
+    const uint32_t kbox = (uint32_t)a.Rt * DBK;                  // one k-block of the band
+    auto rot_of = [&](int tile) { return (int)(((unsigned)tile * 7u) % (unsigned)a.nst); };
+
     if (warp == 0) {
         // --------------------------------------------------- weight stream (TMA) ----
         if (lane == 0) {
+            const uint64_t once = policy_evict_first();
             int stage = 0;
             uint32_t phase = 0, used = 0, last_parity = 0;
-            for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
-                const int n0 = tile * DBM;
-                for (int it = 0; it < a.kblocks; ++it) {
-                    const int kb = rotated_kblock(it, tile, a.kblocks);
-                    if (tile == (int)blockIdx.x && it == S) {
-                        // the ring is full: request the rest of this first tile into L2
-                        const int last = min(a.kblocks, S + kPrefetchBlocks);
-                        for (int pf = S; pf < last; ++pf)
-                            tma_prefetch_l2_2d(&tmCB, rotated_kblock(pf, tile, a.kblocks) * DBK,
-                                               n0);
-                    }
+            for (int tile = band0; tile < a.tiles; tile += bands) {
+                const int rot = rot_of(tile);
+                for (int j = 0; j < a.nst; ++j) {
+                    int sj = j + rot;
+                    if (sj >= a.nst) sj -= a.nst;
+                    const int kb0 = sj * DKS, nkb = min(DKS, a.kblocks - kb0);
                     if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
                     const uint32_t full = smem_addr(&tail->full[stage]);
-                    mbar_arrive_expect_tx(full, DSTAGE);
-                    tma_load_2d(smem_addr(smem + stage * DSTAGE), &tmCB, kb * DBK, n0, full);
+                    mbar_arrive_expect_tx(full, (uint32_t)nkb * kbox);
+                    for (int h = 0; h < nkb; ++h)
+                        tma_load_2d_policy(smem_addr(ring + stage * stage_bytes + h * kbox), &tmCB,
+                                           (kb0 + h) * DBK, tile * a.Rt, full, once);
                     used |= 1u << stage;
                     last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
                     if (++stage == S) {
@@ -389,132 +517,183 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 if (used & (1u << s))
                     drain_wait(smem_addr(&tail->full[s]), (last_parity >> s) & 1u, a.status);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 3) {
         // ------------------------------------------------------------- MMA issue ----
-        if (lane == 0) {
-            // the quantize kernel (already running: this grid is its programmatic dependent)
-            // publishes the image with a release store of the call's epoch
-            bool published = false;
-            {
-                const uint64_t t0 = global_timer_ns();
-                for (uint32_t it = 0;; ++it) {
-                    unsigned long long v;
-                    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];"
-                                 : "=l"(v)
-                                 : "l"(&a.tables->ready)
-                                 : "memory");
-                    if (v == a.epoch) {
-                        published = true;
-                        break;
-                    }
-                    if ((it & 63u) == 0u && (tail->abort_flag ||
-                                             global_timer_ns() - t0 > a.timeout_ns)) {
-                        tail->abort_flag = 1;
-                        a.status.timed_out();
-                        break;
-                    }
-                }
-            }
-            fence_proxy_async_global();
-            const uint32_t xbar = smem_addr(&tail->xbar);
-            const uint32_t img_bytes = (uint32_t)image_bytes(a.kblocks, a.rows);
-            mbar_arrive_expect_tx(xbar, img_bytes + (uint32_t)sizeof(DecodeTables));
-            bulk_load_1d(smem_addr(xq), a.image, img_bytes, xbar);
-            bulk_load_1d(smem_addr(&tail->tab), a.tables, (uint32_t)sizeof(DecodeTables), xbar);
-            const bool have_x = published && wait(xbar, 0);
-            const uint32_t idesc = idesc_i8(DBM, DM);
-            const uint32_t xq_base = smem_addr(xq);
-            int stage = 0, acc = 0;
-            uint32_t phase = 0, acc_phase = 0;
-            for (int tile = blockIdx.x; have_x && tile < a.tiles; tile += gridDim.x) {
+        const int issuer = warp == 1 ? 0 : 1;
+        if (lane == 0 && (issuer == 0 || a.nst >= 2)) {
+            const uint32_t idesc = idesc_i8(DMMA_M, DM);
+            const uint32_t img_base = smem_addr(img);
+            const uint32_t ring_base = smem_addr(ring);
+            const uint32_t zero_atom = img_base + (uint32_t)a.nistage * DKS * img_bytes;
+            int acc = 0, tl_ = 0;                          // tl_: this CTA's tile count so far
+            uint32_t acc_phase = 0;
+            bool good = true;
+            for (int tile = band0; good && tile < a.tiles; tile += bands, ++tl_) {
                 if (!wait(smem_addr(&tail->acc_empty[acc]), acc_phase ^ 1)) break;
                 tc_fence_after();
-                const uint32_t d = tmem + (uint32_t)(acc * DSUB * DM);
-                bool good = true;
-                for (int it = 0; it < a.kblocks; ++it) {
-                    const int kb = rotated_kblock(it, tile, a.kblocks);
-                    if (!wait(smem_addr(&tail->full[stage]), phase)) {
+                const uint32_t d = tmem + (uint32_t)((acc * 2 + issuer) * DM);
+                const int rot = rot_of(tile);
+                bool first = true;
+                for (int j = issuer; j < a.nst; j += 2) {
+                    const int g = tl_ * a.nst + j;               // stage in the producer's order
+                    const int stage = g % S;
+                    const uint32_t phase = (uint32_t)(g / S) & 1u;
+                    int sj = j + rot;
+                    if (sj >= a.nst) sj -= a.nst;
+                    const int nkb = min(DKS, a.kblocks - sj * DKS);
+                    // the image stage of these k-blocks: fixed when resident, else a ring
+                    const int ist = a.resident ? sj : g % a.nistage;
+                    const uint32_t ipar = a.resident ? 0u : (uint32_t)(g / a.nistage) & 1u;
+                    if (!wait(smem_addr(&tail->ifull[ist]), ipar) ||
+                        !wait(smem_addr(&tail->full[stage]), phase)) {
                         good = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_addr(smem + stage * DSTAGE);
-                    const uint32_t sb = xq_base + (uint32_t)(kb * a.rows * 128);
-                    const uint32_t sbo =
-                        a.rows == 8 ? (uint32_t)((a.kblocks - kb) * 1024) : 1024u;
-                    const uint32_t dsub = d + (uint32_t)((it % DSUB) * DM);
+                    for (int h = 0; h < nkb; ++h) {
+                        const uint32_t sa = ring_base + (uint32_t)stage * stage_bytes + h * kbox;
+                        const uint32_t sb = img_base + (uint32_t)(ist * DKS + h) * img_bytes;
+                        const uint64_t adesc = sw128_desc(sa);
+                        const uint64_t bdesc = image_desc(sb, a.rows == 8 ? zero_atom - sb : 1024u);
 #pragma unroll
-                    for (int k = 0; k < DBK / 32; ++k)
-                        mma_i8(dsub, sw128_desc(sa + 32 * k), image_desc(sb + 32 * k, sbo), idesc,
-                               (it >= DSUB) || k != 0);
-                    tc_commit(smem_addr(&tail->empty[stage]));
-                    if (++stage == S) {
-                        stage = 0;
-                        phase ^= 1;
+                        for (int k = 0; k < DBK / 32; ++k) {
+                            mma_i8(d, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
+                                   first ? 0u : 1u);
+                            first = false;
+                        }
                     }
+                    tc_commit(smem_addr(&tail->empty[stage]));
+                    if (!a.resident) tc_commit(smem_addr(&tail->iempty[ist]));
                 }
                 if (!good) break;
                 tc_commit(smem_addr(&tail->acc_full[acc]));
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
             }
-            if (!have_x) drain_wait(xbar, 0, a.status);   // the copies land before exit
-            tc_commit(smem_addr(&tail->mma_done));
-            drain_wait(smem_addr(&tail->mma_done), 0, a.status);
+            tc_commit(smem_addr(&tail->mma_done[issuer]));
+            drain_wait(smem_addr(&tail->mma_done[issuer]), 0, a.status);
         }
-    } else if (warp >= 4) {
+    } else if (warp == 2) {
+        // ------------------------------------------------- operand image of X, by k-block ----
+        // Once the quantizer has published, one thread copies the image blocks (rows x 128
+        // bytes each) from the workspace: when every k-block fits (resident), each once, into
+        // the image stage of its weight stage; otherwise through a ring of image stages, in
+        // the order the MMAs consume them.
+        if (a.rows == 8) {
+            // the zero atom read as rows 8..15 of an 8-row image block
+            for (int i = lane; i < 64; i += 32)
+                reinterpret_cast<uint4 *>(img + a.nistage * DKS * img_bytes)[i] =
+                    make_uint4(0, 0, 0, 0);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        __syncwarp();
+        if (lane == 0 && poll_words(a.table->iready, a.nq, a.epoch, a.status, a.timeout_ns,
+                                    &tail->abort_flag)) {
+            fence_proxy_async_global();           // the image is read by the async proxy
+            const int ntiles = (a.tiles - band0 + bands - 1) / bands;   // tiles of this CTA
+            const int nstg = a.resident ? a.nst : ntiles * a.nst;
+            uint32_t used = 0, last_parity = 0;
+            for (int g = 0; g < nstg; ++g) {
+                const int tile = band0 + (g / a.nst) * bands;
+                int sj = g % a.nst + rot_of(tile);
+                if (sj >= a.nst) sj -= a.nst;
+                const int kb0 = sj * DKS, nkb = min(DKS, a.kblocks - kb0);
+                const int ist = a.resident ? sj : g % a.nistage;
+                const uint32_t ipar = a.resident ? 0u : (uint32_t)(g / a.nistage) & 1u;
+                if (!a.resident && !wait(smem_addr(&tail->iempty[ist]), ipar ^ 1)) break;
+                const uint32_t full = smem_addr(&tail->ifull[ist]);
+                mbar_arrive_expect_tx(full, (uint32_t)nkb * img_bytes);
+                for (int h = 0; h < nkb; ++h)
+                    bulk_load_1d(smem_addr(img + (ist * DKS + h) * img_bytes),
+                                 a.image + (size_t)(kb0 + h) * img_bytes, img_bytes, full);
+                used |= 1u << ist;
+                last_parity = (last_parity & ~(1u << ist)) | (ipar << ist);
+            }
+            // every copy lands before the CTA may exit
+            for (int sl = 0; sl < 32; ++sl)
+                if (used & (1u << sl))
+                    drain_wait(smem_addr(&tail->ifull[sl]), (last_parity >> sl) & 1u, a.status);
+        }
+    } else {
         // ------------------------------------------------------------------ epilogue ----
-        // Everything of an output row except the int8 product - its scale, bias and fp16
+        // Everything of an output channel except the int8 product - its scale, bias and fp16
         // outlier part - is computed while the MMAs still stream the weights; after the last
         // MMA of a tile only the accumulator read, one FMA per value and the stores remain.
         const int qd = warp & 3;
         const int et = threadIdx.x - 128;                 // 0..127 over the epilogue warps
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
         const float inv = 1.0f / 16129.0f;
-        int okx = 0;
-        if (lane == 0) okx = wait(smem_addr(&tail->xbar), 0) ? 1 : 0;   // the table is in
-        okx = __shfl_sync(0xffffffffu, okx, 0);
-        const int n_out = okx ? tail->tab.n_out : 0;
-        // X at the outlier columns (an input of the call, complete before this grid launched)
+        // warp 4 polls quantizer 0's table; the other epilogue warps wait on it in shared memory
+        int ok = 0;
+        if (warp == 4 && lane == 0) {
+            ok = poll_words(&a.table->ready, 1, a.epoch, a.status, a.timeout_ns, &tail->abort_flag)
+                     ? 1 : 0;
+            if (ok) mbar_arrive(smem_addr(&tail->tbar));
+        } else if (lane == 0) {
+            ok = wait(smem_addr(&tail->tbar), 0) ? 1 : 0;
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        // every lane acquires the published table itself (it is there: one load each)
+        if (ok && acquire_word(&a.table->ready) != a.epoch) ok = 0;
+        const int n_out = ok ? a.table->n_out : 0;
+        float sca[DM];
+#pragma unroll
+        for (int mm = 0; mm < DM; ++mm) sca[mm] = ok ? a.table->sca[mm] : 0.0f;
+        // the outlier columns and X at them (a 16-row [j][m] table; rows >= M hold 0)
+        for (int i = et; i < n_out; i += 128) tail->idx[i] = a.table->idx[i];
         for (int i = et; i < n_out * DM; i += 128) {
             const int j = i / DM, mm = i % DM;
-            tail->xo[i] = mm < a.M ? a.X[(int64_t)mm * a.K + tail->tab.idx[j]]
-                                   : __float2half_rn(0.0f);
+            xo[i] = mm < a.M ? a.X[(int64_t)mm * a.K + a.table->idx[j]] : __float2half_rn(0.0f);
         }
         named_barrier(1, 128);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; okx && tile < a.tiles; tile += gridDim.x) {
-            const int n = tile * DBM + qd * 32 + lane;
-            const bool live = n < a.N;
+        for (int tile = band0; ok && tile < a.tiles; tile += bands) {
+            const int r = qd * 32 + lane;                 // TMEM lane = row of the band
+            const int n = tile * a.Rt + r;
+            const bool live = r < a.Rt && n < a.N;
             float o[DM];
             float scale = 0.0f;
 #pragma unroll
-            for (int m = 0; m < DM; ++m) o[m] = 0.0f;
+            for (int mm = 0; mm < DM; ++mm) o[mm] = 0.0f;
             if (live) {
                 const float sb = a.SCB[n];
                 const float b = a.bias ? __half2float(a.bias[n]) : 0.0f;
                 scale = sb * inv;
                 const int8_t *cbrow = a.CB + (int64_t)n * a.K;
-                for (int j = 0; j < n_out; ++j) {
-                    const int col = tail->tab.idx[j];
-                    const __half wh = a.W16 ? a.W16[(int64_t)n * a.K + col]
-                                            : __float2half_rn(__fdiv_rn(
-                                                  __fmul_rn((float)cbrow[col], sb), 127.0f));
-                    if (a.Wo) a.Wo[(int64_t)n * a.wo_pitch + j] = wh;
-                    const float w = __half2float(wh);
-                    const uint4 *xv = reinterpret_cast<const uint4 *>(tail->xo + j * DM);
-                    float f0[8], f1[8];
-                    unpack8(xv[0], f0);
-                    unpack8(xv[1], f1);
+                const __half *wrow = a.W16 ? a.W16 + (int64_t)n * a.K : nullptr;
+                for (int j0 = 0; j0 < n_out; j0 += 8) {
+                    // eight independent loads of the outlier weights before any use
+                    int8_t cb8[8];
+                    __half w8[8];
 #pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        o[m] = fmaf(f0[m], w, o[m]);
-                        o[m + 8] = fmaf(f1[m], w, o[m + 8]);
+                    for (int u = 0; u < 8; ++u) {
+                        const int col = tail->idx[min(j0 + u, n_out - 1)];
+                        if (wrow) w8[u] = wrow[col];
+                        else cb8[u] = cbrow[col];
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = j0 + u;
+                        if (j >= n_out) break;
+                        const __half wh = wrow ? w8[u]
+                                               : __float2half_rn(__fdiv_rn(
+                                                     __fmul_rn((float)cb8[u], sb), 127.0f));
+                        if (a.Wo) a.Wo[(int64_t)n * a.wo_pitch + j] = wh;
+                        const float w = __half2float(wh);
+                        const uint4 *xv = reinterpret_cast<const uint4 *>(xo + j * DM);
+                        float f0[8], f1[8];
+                        unpack8(xv[0], f0);
+                        unpack8(xv[1], f1);
+#pragma unroll
+                        for (int mm = 0; mm < 8; ++mm) {
+                            o[mm] = fmaf(f0[mm], w, o[mm]);
+                            o[mm + 8] = fmaf(f1[mm], w, o[mm + 8]);
+                        }
                     }
                 }
 #pragma unroll
-                for (int m = 0; m < DM; ++m) o[m] += b;
+                for (int mm = 0; mm < DM; ++mm) o[mm] += b;
             }
             int okw = 0;
             if (lane == 0) okw = wait(smem_addr(&tail->acc_full[acc]), acc_phase) ? 1 : 0;
@@ -522,14 +701,13 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             if (!okw) break;
             tc_fence_after();
             uint32_t d[DM];
-            tmem_ld_32x16(tl + (uint32_t)(acc * DSUB * DM), d);
-            for (int u = 1; u < DSUB; ++u) {
-                if (u >= a.kblocks) break;               // sub-accumulators never written
+            tmem_ld_32x16(tl + (uint32_t)(acc * 2 * DM), d);
+            if (a.nst >= 2) {
                 uint32_t e[DM];
-                tmem_ld_32x16(tl + (uint32_t)((acc * DSUB + u) * DM), e);
+                tmem_ld_32x16(tl + (uint32_t)((acc * 2 + 1) * DM), e);
                 tmem_wait_ld();
 #pragma unroll
-                for (int m = 0; m < DM; ++m) d[m] += e[m];
+                for (int mm = 0; mm < DM; ++mm) d[mm] += e[mm];
             }
             tmem_wait_ld();
             tc_fence_before();
@@ -539,11 +717,11 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             if (acc == 0) acc_phase ^= 1;
             if (live) {
 #pragma unroll
-                for (int m = 0; m < DM; ++m) {
-                    if (m < a.M) {
-                        const float y = fmaf((float)(int32_t)d[m], tail->tab.sca[m] * scale, o[m]);
-                        a.Y[(int64_t)m * a.N + n] = __float2half_rn(y);
-                        if (a.C_debug) a.C_debug[(int64_t)m * a.N + n] = (int32_t)d[m];
+                for (int mm = 0; mm < DM; ++mm) {
+                    if (mm < a.M) {
+                        const float y = fmaf((float)(int32_t)d[mm], sca[mm] * scale, o[mm]);
+                        a.Y[(int64_t)mm * a.N + n] = __float2half_rn(y);
+                        if (a.C_debug) a.C_debug[(int64_t)mm * a.N + n] = (int32_t)d[mm];
                     }
                 }
             }
@@ -573,6 +751,39 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 }  // namespace
 
+DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int64_t cap, int sms) {
+    DecodePlan p;
+    const int64_t kblocks = ceil_div(K, DBK);
+    p.nq = (int)std::max<int64_t>(1, std::min<int64_t>(kDecodeMaxQuantizers, kblocks / QKB));
+    p.bpq = (int)ceil_div(kblocks, p.nq);
+    p.nq = (int)ceil_div(kblocks, p.bpq);                 // every quantizer owns k-blocks
+    const int64_t streamers = std::max(1, sms - p.nq);
+    const int64_t per_cta = ceil_div(N, streamers * DMMA_M);               // bands per CTA
+    p.Rt = (int)std::min<int64_t>(DMMA_M, align_up(ceil_div(N, streamers * per_cta), 8));
+    p.tiles = (int)ceil_div(N, p.Rt);
+    p.grid = p.nq + (int)std::min<int64_t>(p.tiles, streamers);
+    p.kblocks = (int)ceil_div(K, DBK);
+    p.rows = image_rows((int)M);
+    // shared memory of a streamer: [image ring (+ zero atom)][tail][xo][weight ring][slack for
+    // the MMA's 128 rows]; the quantizer uses the first sizeof(QShared) bytes
+    p.nst = (int)ceil_div(p.kblocks, DKS);
+    const int64_t istage = (int64_t)DKS * p.rows * DBK;
+    p.resident = p.nst <= DIMG_MAX && p.nst * istage <= DIMG_BYTES;
+    p.nistage = p.resident ? p.nst : (int)std::min<int64_t>(DIMG_MAX, DIMG_BYTES / istage);
+    const int64_t img = align_up((int64_t)p.nistage * istage + (p.rows == 8 ? 1024 : 0), 1024);
+    p.tail_off = (uint32_t)img;
+    p.xo_off = (uint32_t)align_up(p.tail_off + (int64_t)sizeof(DTail), 16);
+    p.ring_off = (uint32_t)align_up(p.xo_off + std::max<int64_t>(cap, 1) * DM * 2, 1024);
+    const int64_t stage = (int64_t)DKS * p.Rt * DBK;
+    const int64_t slack = (int64_t)(DMMA_M - p.Rt) * DBK;
+    const int64_t room = SMEM_LIMIT - 1024 - (int64_t)p.ring_off - slack;
+    p.stages = (int)std::max<int64_t>(0, std::min<int64_t>(DMAX_STAGES, room / stage));
+    // a quantizer: tables, M x (its columns) of X, their image
+    const int64_t qsmem = QX_OFF + M * p.bpq * DBK * 2 + (int64_t)p.bpq * p.rows * DBK + 1024;
+    p.smem = (int)std::max<int64_t>(p.ring_off + p.stages * stage + slack + 1024, qsmem);
+    return p;
+}
+
 cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     static std::mutex mu;
     static int sms_cache[64] = {0};
@@ -594,43 +805,10 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
         }
         sms = sms_cache[dev];
     }
+    const DecodePlan p = decode_plan(d.M, d.N, d.K, d.cap, sms);
+    if (p.stages < 2 || p.smem > SMEM_LIMIT) return cudaErrorInvalidValue;
 
-    // 1. quantize X once (one CTA)
-    QArgs q;
-    q.X = d.X;
-    q.M = (int)d.M;
-    q.K = (int)d.K;
-    q.cap = (int)d.cap;
-    q.threshold = d.threshold;
-    q.image = d.image;
-    q.tables = d.tables;
-    q.count = d.count;
-    q.status = d.status;
-    q.epoch = d.status.tag >> 4;
-    q.rows = image_rows((int)d.M);
-    {
-        cudaLaunchConfig_t qc = {};
-        cudaLaunchAttribute qa[2];
-        qa[0].id = cudaLaunchAttributeClusterDimension;
-        qa[0].val.clusterDim.x = QCL;
-        qa[0].val.clusterDim.y = 1;
-        qa[0].val.clusterDim.z = 1;
-        qa[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        qa[1].val.programmaticStreamSerializationAllowed = 1;
-        qc.gridDim = dim3(QCL);
-        qc.blockDim = dim3(QTHREADS);
-        qc.dynamicSmemBytes = 0;
-        qc.stream = s;
-        qc.attrs = qa;
-        qc.numAttrs = 2;
-        err = cudaLaunchKernelEx(&qc, llmint8_decode_quantize_kernel, q);
-        note_launches(1);
-        if (err != cudaSuccess) return err;
-    }
-
-    // 2. the weight-streaming product, allowed to start before step 1 finishes
     DArgs a;
-    a.epoch = d.status.tag >> 4;
     a.X = d.X;
     a.CB = d.CB;
     a.SCB = d.SCB;
@@ -640,33 +818,45 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     a.C_debug = d.C_debug;
     a.Wo = d.Wo;
     a.wo_pitch = d.wo_pitch;
+    a.bitmaps = d.bitmaps;
+    a.n_bitmaps = (int)d.n_bitmaps;
+    a.count = d.count;
+    a.table = d.table;
     a.image = d.image;
-    a.tables = d.tables;
     a.status = d.status;
+    a.epoch = d.status.tag >> 4;
     a.M = (int)d.M;
     a.N = (int)d.N;
     a.K = (int)d.K;
-    a.kblocks = (int)ceil_div(d.K, DBK);
-    a.tiles = (int)ceil_div(d.N, DBM);
+    a.cap = (int)d.cap;
+    a.threshold = d.threshold;
+    {
+        // smallest fp16 >= threshold (threshold > 0 here), in both halves
+        const __half t16 = __float2half_ru(d.threshold);
+        const uint32_t tb = (uint32_t)*reinterpret_cast<const uint16_t *>(&t16);
+        a.thr2 = tb | (tb << 16);
+    }
+    a.rows = p.rows;
+    a.Rt = p.Rt;
+    a.tiles = p.tiles;
+    a.kblocks = p.kblocks;
+    a.stages = p.stages;
+    a.nq = p.nq;
+    a.bpq = p.bpq;
+    a.nst = p.nst;
+    a.nistage = p.nistage;
+    a.resident = p.resident ? 1 : 0;
+    a.tail_off = p.tail_off;
+    a.xo_off = p.xo_off;
+    a.ring_off = p.ring_off;
     a.timeout_ns = d.timeout_ns;
-    // shared memory: [stages][quantized X][tail], 1024-byte aligned pieces
-    a.rows = image_rows((int)d.M);
-    const int xq_bytes = (int)align_up(image_bytes(a.kblocks, a.rows), 1024);
-    const int tail_bytes = (int)align_up(sizeof(DTail), 1024);
-    const int room = SMEM_LIMIT - 1024 - xq_bytes - tail_bytes;
-    a.stages = std::min(DMAX_STAGES, room / DSTAGE);
-    if (a.stages < 2) return cudaErrorInvalidValue;
-    a.xq_off = (uint32_t)(a.stages * DSTAGE);
-    a.tail_off = a.xq_off + (uint32_t)xq_bytes;
-    const int smem = (int)(a.tail_off + sizeof(DTail) + 1024);
-    if (smem > SMEM_LIMIT) return cudaErrorInvalidValue;
 
     auto enc = encoder();
     if (!enc) return cudaErrorInvalidValue;
     CUtensorMap tm;
     cuuint64_t dims[2] = {(cuuint64_t)d.K, (cuuint64_t)d.N};
     cuuint64_t strides[1] = {(cuuint64_t)d.K};
-    cuuint32_t box[2] = {DBK, DBM};
+    cuuint32_t box[2] = {DBK, (cuuint32_t)p.Rt};
     cuuint32_t estr[2] = {1, 1};
     if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(d.CB), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -677,10 +867,9 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    // QCL SMs stay with the quantize kernel while this grid starts
-    cfg.gridDim = dim3((unsigned)std::min(a.tiles, std::max(1, sms - QCL)));
+    cfg.gridDim = dim3((unsigned)p.grid);
     cfg.blockDim = dim3(DTHREADS);
-    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.dynamicSmemBytes = (size_t)p.smem;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;

@@ -68,29 +68,53 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s);
 
 namespace llmint8 {
 
-// Decode path (M <= kDecodeMaxM, K <= kDecodeMaxK): a cluster of CTAs quantizes X into a
-// ready-to-copy image of the tensor-core operand plus small tables in the workspace; the
-// weight-streaming tcgen05 kernel, launched as its programmatic dependent, starts streaming
-// CB at once and waits for that image only before its first MMA.
+// Decode path (M <= kDecodeMaxM, K <= kDecodeMaxK, at most kDecodeMaxOutliers outlier
+// columns): one weight-streaming tcgen05 kernel per call.  Its first CTAs quantize X (each a
+// slice of the columns) and publish the outlier columns, row scales and the int8 operand image
+// through a DecodeTable and the image in the workspace; every other CTA streams a band of
+// weight rows.
 constexpr int kDecodeMaxM = 16;
-constexpr int kDecodeMaxK = 8192;
+constexpr int kDecodeMaxK = 16384;
 constexpr int kDecodeMaxOutliers = 256;
 
-// Written by the decode quantize kernel, copied whole into every decode CTA.
-struct DecodeTables {
-    unsigned long long ready;                 // call epoch, stored last (release)
-    int32_t n_out;                            // outlier columns used (<= capacity)
-    int32_t pad;
+// What the quantizer CTAs publish (workspace, 256-byte aligned).  Every word tagged with the
+// call number is stored with release semantics after the data it covers:
+//   pready[q]  quantizer q's outlier bits (flags of its chunks) and row maxima (part[q]);
+//   iready[q]  quantizer q's k-blocks of the operand image;
+//   ready      quantizer 0's row scales, outlier list and counts.
+constexpr int kDecodeMaxQuantizers = 8;
+struct DecodeTable {
+    unsigned long long ready;
+    unsigned long long pready[kDecodeMaxQuantizers];
+    unsigned long long iready[kDecodeMaxQuantizers];
+    int32_t total;                            // outlier columns found
+    int32_t n_out;                            // ... of them listed (<= capacity)
     float sca[kDecodeMaxM];                   // row absmax over the regular columns
+    float part[kDecodeMaxQuantizers][kDecodeMaxM];   // per-quantizer row maxima
     int32_t idx[kDecodeMaxOutliers];          // outlier columns, ascending
+    uint8_t flags[kDecodeMaxK / 8];           // outlier bits of each 8-column chunk
 };
-static_assert(sizeof(DecodeTables) % 16 == 0, "copied with a bulk copy");
 
-// Bytes of the quantized-X operand image: 16 rows x K rounded up to 128, in 128-column
-// blocks of two 1024-byte swizzled 8-row atoms.
-__host__ __device__ constexpr int64_t decode_image_bytes(int64_t K) {
-    return kDecodeMaxM * ((K + 127) / 128 * 128);
+// Bytes of the int8 operand image the quantizer writes: one block of 16 rows (8 when M <= 8)
+// x 128 bytes per 128-column k-block.
+__host__ __device__ constexpr int64_t decode_image_bytes(int64_t M, int64_t K) {
+    return (K + 127) / 128 * (M <= 8 ? 8 : kDecodeMaxM) * 128;
 }
+
+// Launch geometry of the decode kernel for one shape.
+struct DecodePlan {
+    int Rt = 0;              // weight rows (output channels) per tile
+    int tiles = 0, grid = 0, kblocks = 0;
+    int rows = 0;            // rows of an operand-image block (8 or 16)
+    int stages = 0, smem = 0;
+    int nq = 0;              // quantizer CTAs (the first nq of the grid)
+    int bpq = 0;             // k-blocks per quantizer
+    int nst = 0;             // weight stages per tile (2 k-blocks each)
+    int nistage = 0;         // operand-image stages of a streamer
+    bool resident = false;   // ... holding every k-block (filled once)
+    uint32_t tail_off = 0, xo_off = 0, ring_off = 0;
+};
+DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int64_t cap, int sms);
 
 struct DecodeLaunch {
     const __half *X;         // [M, K]
@@ -102,9 +126,11 @@ struct DecodeLaunch {
     int32_t *C_debug;        // [M, N] or null
     __half *Wo;              // [N, wo_pitch] or null: receives the outlier weights used
     int64_t wo_pitch;
+    const uint32_t *bitmaps; // [n_bitmaps][ceil(K/32)]: the outlier set given, or null
+    int64_t n_bitmaps;
     int32_t *count;          // device outlier count (workspace header)
-    uint8_t *image;          // workspace: decode_image_bytes(K), 1024-byte aligned
-    DecodeTables *tables;    // workspace
+    DecodeTable *table;      // workspace
+    uint8_t *image;          // workspace: decode_image_bytes(M, K), 1024-byte aligned
     StatusRef status;
     int64_t M, N, K, cap;
     float threshold;

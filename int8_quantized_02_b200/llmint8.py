@@ -440,7 +440,7 @@ def llmint8_linear_noalloc(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
                            bias=None, W_fp16=None, threshold: float = 6.0,
                            max_outliers: int = 64, stream=None) -> int:
     """llmint8_linear on the library's fixed per-device scratch: no workspace, nothing
-    allocated (the caller passes Y).  Decode shapes only (M <= 16, K <= 8192, threshold > 0,
+    allocated (the caller passes Y).  Decode shapes only (M <= 16, K <= 16384, threshold > 0,
     max_outliers <= 256).  Returns the device address of the scratch, whose header
     llmint8_device_status / llmint8_workspace_outlier_count read through the C ABI."""
     M, K = X.shape

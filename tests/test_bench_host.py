@@ -1,10 +1,8 @@
-"""bench.py's host-side rules, on the CPU: the traffic figure is used only for the kernel
-sources it was measured on, and the peaks fall back to the stated figures without a
-measured-peaks file."""
+"""bench.py's host-side rules, on the CPU: the peaks fall back to the stated figures without a
+measured-peaks file, and the repeat count and spread of the repeated timed region."""
 from __future__ import annotations
 
 import os
-import shutil
 import sys
 
 import pytest
@@ -16,24 +14,8 @@ import bench  # noqa: E402
 
 @pytest.fixture
 def fake_root(tmp_path, monkeypatch):
-    shutil.copytree(os.path.join(ROOT, "int8_quantized_02_b200", "csrc"),
-                    tmp_path / "int8_quantized_02_b200" / "csrc")
-    (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     return tmp_path
-
-
-def test_traffic_is_used_only_for_the_sources_it_was_taken_on(fake_root):
-    h = bench.kernel_source_hash()
-    assert len(h) == 16
-    (fake_root / "profiles" / "traffic_decode.md").write_text(
-        f"# x\n\nkernel_source_hash: {h}\ndram_bytes_per_launch: 67566848\n")
-    assert bench.profiled_traffic("decode") == 67566848.0
-    assert bench.profiled_traffic("proj175b") is None              # no file
-    src = fake_root / "int8_quantized_02_b200" / "csrc" / "decode.cu"
-    src.write_bytes(src.read_bytes() + b"\n// changed\n")
-    assert bench.kernel_source_hash() != h
-    assert bench.profiled_traffic("decode") is None                 # sources changed
 
 
 def test_peaks_fall_back_without_the_measured_file(fake_root):
@@ -44,3 +26,20 @@ def test_peaks_fall_back_without_the_measured_file(fake_root):
     p = bench.measured_peaks()
     assert p["source"] == "measured" and p["hbm_gbs"] == 6464.9
     assert p["bf16_tflops_sustained"] == 1368.0
+
+
+def test_repeat_count():
+    assert bench.repeat_count(0.001, 1.0) == 200           # capped
+    assert bench.repeat_count(0.01, 1.0) == 100
+    assert bench.repeat_count(0.3, 1.0) == 4               # ceil(1 / 0.3)
+    assert bench.repeat_count(2.0, 1.0) == 3               # at least three
+    assert bench.repeat_count(0.0, 1.0) == 200
+    assert bench.repeat_count(0.1, 1.0, lo=3, hi=5) == 5
+
+
+def test_spread():
+    s = bench.spread([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert s["n"] == 5 and s["median"] == 3.0 and s["min"] == 1.0 and s["max"] == 5.0
+    assert s["p10"] == 1.0 and s["p90"] == 5.0
+    s = bench.spread([float(i) for i in range(101)])
+    assert s["p10"] == 10.0 and s["p90"] == 90.0 and s["median"] == 50.0

@@ -67,8 +67,6 @@ def test_workspace_sizes(lib):
     assert base > 16 * 1024          # holds at least Xq
     assert f(16, 1024, 1024, 64) > base
     assert f(32, 1024, 1024, 64) > f(17, 1024, 1024, 64)
-    # shapes the decode path can take (M <= 16, K <= 8192) also hold its quantized-X image
-    assert f(16, 1024, 1024, 64) > f(17, 1024, 1024, 64) - 1024 * 64 * 2
     # shapes outside the rules give 0
     assert f(0, 1024, 1024, 0) == 0
     assert f(16, 1000, 1024, 0) == 0          # N not a multiple of 16

@@ -100,9 +100,10 @@ def _check(wl, threshold, cap):
     del C
     # step a3 bit for bit: the fp16 weight rows used for the outlier columns
     n_w = min(n_o, cap)
-    Wo = host(L.llmint8_workspace_outlier_weights(ws, M, N, K, cap, n_w))
-    want = oracle.dequant(np.ascontiguousarray(CB_o[:, idx_o[:n_w]]), SCB_o)
-    assert np.array_equal(Wo.view(np.uint16), want.view(np.uint16)), f"{wl.name}: W_o"
+    if n_w > 0:
+        Wo = host(L.llmint8_workspace_outlier_weights(ws, M, N, K, cap, n_w))
+        want = oracle.dequant(np.ascontiguousarray(CB_o[:, idx_o[:n_w]]), SCB_o)
+        assert np.array_equal(Wo.view(np.uint16), want.view(np.uint16)), f"{wl.name}: W_o"
 
     if M <= 16:
         Y_o, C_o = oracle.linear(X, CB_o, SCB_o, threshold=threshold, want_C=True)

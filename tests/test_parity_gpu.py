@@ -341,10 +341,11 @@ def test_maximum_K_accumulator_bound():
     assert np.isfinite(Y_gpu).all()
 
 
-def test_decode_path_limits_K8192_cap256():
+@pytest.mark.parametrize("M", [16, 3])
+def test_decode_path_limits_K16384_cap256(M):
     # the decode path's largest K and outlier capacity, with 200 outlier columns
-    X = _x(16, 8192, 200, lo=6.0, hi=60.0, row_frac=1.0, seed=41)
-    W = synth.weight(512, 8192, 0.02, seed=41)
+    X = _x(M, 16384, 200, lo=6.0, hi=60.0, row_frac=1.0, seed=41)
+    W = synth.weight(512, 16384, 0.02, seed=41)
     _check_linear(X, W, 6.0, cap=256)
 
 

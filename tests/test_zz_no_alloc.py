@@ -1,4 +1,6 @@
-"""llmint8_linear_noalloc: the decode path on the library's fixed per-device scratch.
+"""llmint8_linear_noalloc: the decode kernel with its scratch (the status header) in the
+library's fixed per-device array, for callers that cannot allocate device memory where they
+call the layer.
 
 Collected last on purpose (file name), so that it also runs after every other GPU test of
 the session has used the library; it passes alone as well.
@@ -13,6 +15,7 @@ import torch
 
 from int8_quantized_02_b200 import llmint8 as L
 from int8_quantized_02_b200 import synth
+from oracle import oracle
 from tests.gpu_util import assert_y_close, dev, host
 
 _FAKE = ctypes.c_void_p(1 << 20)     # aligned, never dereferenced: rejected before any CUDA call
@@ -25,7 +28,7 @@ def _raw(M, K, N, threshold=6.0, cap=64, X=_FAKE):
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     assert _raw(17, 4096, 4096) == L.ERR_UNSUPPORTED_SHAPE        # M above 16
-    assert _raw(16, 8208, 4096) == L.ERR_UNSUPPORTED_SHAPE        # K above 8192
+    assert _raw(16, 16400, 4096) == L.ERR_UNSUPPORTED_SHAPE       # K above 16384
     assert _raw(16, 4096, 4096, cap=257) == L.ERR_UNSUPPORTED_SHAPE
     assert _raw(16, 4096, 4096, threshold=0.0) == L.ERR_UNSUPPORTED_SHAPE
     assert _raw(16, 4096, 4096, threshold=float("nan")) == L.ERR_INVALID_ARG
@@ -51,11 +54,15 @@ def _count(addr):
 @pytest.mark.gpu
 @pytest.mark.parametrize("M,K,N", [(16, 4096, 4096), (5, 1040, 592), (1, 8192, 1024)])
 def test_noalloc_matches_llmint8_linear_two_calls_in_a_row(M, K, N):
+    """Two calls in a row on different inputs: each output has the same bytes as
+    llmint8_linear's on the same inputs (the same kernel runs both), the first is also within
+    the layer's tolerance of the CPU oracle, and the calls allocate no device memory."""
     cap = 64
     X1 = synth.activations(M, K, 6, lo=6.0, hi=60.0, row_frac=1.0, seed=101 + M)[0]
     X2 = synth.activations(M, K, 3, lo=6.0, hi=20.0, row_frac=0.5, seed=202 + M)[0]
     W = synth.weight(N, K, 0.02, seed=303)
-    bias = dev(synth.bias(N, seed=4))
+    b = synth.bias(N, seed=4)
+    bias = dev(b)
     CB, SCB = L.llmint8_quantize_weight_colwise(dev(W))
     X1d, X2d = dev(X1), dev(X2)
     Y1 = torch.empty((M, N), dtype=torch.float16, device="cuda")
@@ -66,10 +73,14 @@ def test_noalloc_matches_llmint8_linear_two_calls_in_a_row(M, K, N):
     assert addr != 0 and addr % 256 == 0
     torch.cuda.synchronize()
     free0 = torch.cuda.mem_get_info()[0]
+    reserved0 = torch.cuda.memory_reserved()
     a1 = L.llmint8_linear_noalloc(X1d, CB, SCB, Y1, bias=bias, threshold=6.0, max_outliers=cap)
     a2 = L.llmint8_linear_noalloc(X2d, CB, SCB, Y2, bias=bias, threshold=6.0, max_outliers=cap)
     torch.cuda.synchronize()
-    assert torch.cuda.mem_get_info()[0] == free0
+    # torch's allocator saw no request, and the device lost less than the 2 MiB granule any
+    # device allocation takes (tolerating unrelated changes smaller than that)
+    assert torch.cuda.memory_reserved() == reserved0
+    assert torch.cuda.mem_get_info()[0] > free0 - (2 << 20)
     assert a1 == addr and a2 == addr
     assert _status(addr) == L.OK
     n2 = _count(addr)
@@ -85,9 +96,12 @@ def test_noalloc_matches_llmint8_linear_two_calls_in_a_row(M, K, N):
         assert L.llmint8_device_status(ws) == L.OK
         counts.append(L.llmint8_workspace_outlier_count(ws))
     assert n2 == counts[1]
-    assert_y_close(host(Y1), ref[0], "Y (first call)")
-    assert_y_close(host(Y2), ref[1], "Y (second call)")
+    assert np.array_equal(host(Y1).view(np.uint16), ref[0].view(np.uint16)), "Y (first call)"
+    assert np.array_equal(host(Y2).view(np.uint16), ref[1].view(np.uint16)), "Y (second call)"
     assert not np.array_equal(ref[0], ref[1])
+    # and the first output against the CPU oracle, within the layer's tolerance
+    CB_o, SCB_o = oracle.quantize_weight_colwise(W)
+    assert_y_close(host(Y1), oracle.linear(X1, CB_o, SCB_o, bias=b, threshold=6.0), "Y vs oracle")
 
 
 @pytest.mark.gpu
