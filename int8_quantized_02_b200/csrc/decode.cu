@@ -48,7 +48,8 @@ constexpr int DKS = 2;                  // k-blocks per weight stage (one wait, 
 constexpr int DMAX_STAGES = 32;
 constexpr int DIMG_MAX = 32;            // operand-image stages at most ...
 constexpr int DIMG_BYTES = 65536;       // ... and the shared memory they take at most
-constexpr int QKB = 8;                  // k-blocks per quantizer CTA (aim)
+constexpr int QKB = 4;                  // k-blocks per quantizer CTA (aim)
+constexpr int DINFLIGHT = 3;            // weight stages a streamer keeps on their way
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
 // Two MMA issuers per CTA (warps 1 and 3): issuer i takes the weight stages j with
 // j % 2 == i of every tile, into its own int32 accumulator of 16 columns; the epilogue adds the
@@ -141,16 +142,21 @@ __device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
 }
 
 // Shared memory of the quantizer CTA.
+constexpr int QMAX_CHUNKS = 256;         // 8-column chunks of a slice (16 k-blocks)
+constexpr int QWORDS = kDecodeMaxQuantizers * (DM + 1);
+constexpr int QPOLL = (QWORDS + 31) / 32;  // words a polling lane loads per round
 struct QShared {
-    uint64_t xbar;                       // this quantizer's columns of X have landed
-    int ok;                              // every quantizer's partials arrived in time
-    float wmax[DWARPS][DM];              // per-warp partial row maxima
+    uint64_t xbar;                       // the slice of X has landed (bulk copies)
     float sca[DM];                       // row absmax over all regular columns
     float mult[DM];                      // fl32(127 / absmax), 0 for an all-zero row
     int wsum[DWARPS];                    // per-warp outlier counts (list scan)
-    uint8_t flags[kDecodeMaxK / 8];      // outlier bits of each 8-column chunk
+    int ok;                              // every quantizer's partials arrived in time
+    int before, total;                   // outliers of the slices before this one; in all
+    uint32_t fl[QMAX_CHUNKS];            // outlier bits of each 8-column chunk of the slice
+    unsigned long long xp[QWORDS];       // every quantizer's published partials
 };
-// A quantizer's shared memory: QShared, then M rows x its columns of X, then their int8 image.
+// A quantizer's shared memory: QShared, then its M x w slice of X (fp16, row stride w), then
+// the int8 image of its k-blocks.
 constexpr int QX_OFF = 4096;
 static_assert(sizeof(QShared) <= QX_OFF, "quantizer tables fit before the staged X");
 
@@ -194,6 +200,7 @@ struct DArgs {
     int rows;                            // image rows: 16, or 8 when M <= 8
     int Rt;                              // weight rows per tile (band)
     int tiles, kblocks, stages;
+    int inflight;                        // weight stages on their way at most
     int nq, bpq;                         // quantizer CTAs, k-blocks per quantizer
     int nst;                             // weight stages per tile: ceil(kblocks / DKS)
     int nistage;                         // operand-image stages (DKS blocks each) of a streamer
@@ -203,15 +210,15 @@ struct DArgs {
 };
 
 // ------------------------------------------------------------------ the quantizers ----------
-// Quantizer q (CTA q < nq) owns k-blocks [q * bpq, (q + 1) * bpq) of X.  Its columns come into
-// shared memory by bulk copies, one per row.  Pass 1: thread t takes the 8-column chunks t,
-// t + 256, ... of every row, ORs the rows' |x| >= threshold into the chunk's outlier bits and
-// keeps per-row maxima of |x| over the regular columns (packed fp16 compares and maxima,
-// exact); the quantizer publishes its bits and row maxima.  Every quantizer then takes the
-// row maxima of all of them (the row absmax over all regular columns), and pass 2 writes the
-// int8 codes of its columns into a shared-memory image, k-block by k-block in the layout the
-// streamers copy into their own shared memory; one bulk store puts it in the workspace.
-// Quantizer 0 also lists the outlier columns in ascending order.
+// Quantizer q (CTA q < nq) owns the k-blocks [q * bpq, (q + 1) * bpq), a slice of w columns.
+// It copies its slice of X to shared memory (one bulk copy per row) and finds there the outlier
+// bits of every 8-column chunk (an OR over the rows of |x| >= threshold, packed fp16 compares,
+// exact) and, per row, the maximum of |x| over the slice's regular columns.  It publishes those
+// maxima and its outlier count as call-tagged words, reads every quantizer's, and so knows the
+// row scales of the whole layer and where its outlier columns go in the ascending list.  Then
+// it writes the int8 codes of its slice into a shared-memory image, k-block by k-block in the
+// layout the streamers copy into their own shared memory, stores the image to the workspace
+// with one bulk copy, lists its outlier columns, and releases done[q].
 __device__ __forceinline__ void bulk_store_1d(void *dst, uint32_t src, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
                  "r"(src), "r"(bytes)
@@ -224,24 +231,35 @@ __device__ __forceinline__ void bulk_store_wait() {
 __device__ __forceinline__ void release_word(unsigned long long *w, unsigned long long v) {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(w), "l"(v) : "memory");
 }
-__device__ __forceinline__ unsigned long long acquire_word(const unsigned long long *w) {
+__device__ __forceinline__ void relaxed_store(unsigned long long *w, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(w), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long relaxed_load(const unsigned long long *w) {
     unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
     return v;
 }
-// Bounded, backed-off poll (one thread) until every word w[0..n) holds v; false on timeout.
-__device__ bool poll_words(const unsigned long long *w, int n, unsigned long long v,
-                           StatusRef status, uint64_t timeout_ns, volatile int *abort_flag) {
+// Bounded, backed-off poll by one thread until each of the n <= kDecodeMaxQuantizers words
+// holds v.  Each round loads the words together (relaxed); the fence after the round that
+// finds them all makes this thread acquire what their writers released.  False, with the
+// timeout recorded, when they do not all arrive in time or the CTA is winding down.
+__device__ bool poll_all(const unsigned long long *w, int n, unsigned long long v,
+                         StatusRef status, uint64_t timeout_ns, volatile int *abort_flag) {
     const uint64_t t0 = global_timer_ns();
-    int i = 0;
     for (uint32_t it = 0;; ++it) {
-        while (i < n && acquire_word(w + i) == v) ++i;
-        if (i == n) return true;
-        __nanosleep(200);
+        bool ok = true;
+#pragma unroll
+        for (int j = 0; j < kDecodeMaxQuantizers; ++j)
+            if (j < n) ok = (relaxed_load(w + j) == v) && ok;
+        if (ok) {
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            return true;
+        }
+        __nanosleep(32);
         if ((it & 15u) == 15u) {
-            if (abort_flag && *abort_flag) return false;
+            if (*abort_flag) return false;
             if (global_timer_ns() - t0 > timeout_ns) {
-                if (abort_flag) *abort_flag = 1;
+                *abort_flag = 1;
                 status.timed_out();
                 return false;
             }
@@ -249,119 +267,194 @@ __device__ bool poll_words(const unsigned long long *w, int n, unsigned long lon
     }
 }
 
+// Stage j of a tile covers k-blocks DKS * sj ..., sj = j rotated by this offset, so that the
+// CTAs streaming at the same moment read different column ranges of the 2^n-strided rows.
+__device__ __forceinline__ int stage_rot(int tile, int nst) {
+    return (int)(((unsigned)tile * 7u) % (unsigned)nst);
+}
+
+// 0xffff in each half of the four words of a chunk whose outlier bit is set in b
+__device__ __forceinline__ void expand_bits(uint32_t b, uint32_t (&col)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        col[e] = (((b >> (2 * e)) & 1u) ? 0x0000ffffu : 0u) |
+                 (((b >> (2 * e + 1)) & 1u) ? 0xffff0000u : 0u);
+}
+
 __device__ void quantize_x(const DArgs &a, uint8_t *smem) {
     QShared *q = reinterpret_cast<QShared *>(smem);
     const int qi = blockIdx.x;
-    const int kb0 = qi * a.bpq, kb1 = min(a.kblocks, kb0 + a.bpq);
-    const int c0 = kb0 * DBK;                             // first column of this quantizer
-    const int w = min(a.K, kb1 * DBK) - c0;               // its columns (a multiple of 16)
-    uint8_t *xs = smem + QX_OFF;                          // [M][w] fp16
-    uint8_t *is = xs + (size_t)a.M * a.bpq * DBK * 2;     // image of its k-blocks
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nchunks = a.K / 8;
+    const int kb0 = qi * a.bpq, kb1 = min(a.kblocks, kb0 + a.bpq);
+    const int c0 = kb0 * DBK;
+    const int w = min(a.K, kb1 * DBK) - c0;               // columns of the slice (16 | w)
+    const int nch = w / 8;
+    uint8_t *xs = smem + QX_OFF;                          // [M][w] fp16
+    uint8_t *is = xs + (size_t)a.M * a.bpq * DBK * 2;     // image of the slice's k-blocks
+    const unsigned long long tag = (unsigned long long)(uint32_t)a.epoch << 32;
     const int nwords = (a.K + 31) / 32;
-    const uint32_t xbar = smem_addr(&q->xbar);
+
     if (threadIdx.x == 0) {
-        mbar_init(xbar, 1);
-        fence_mbar_init();
+        const uint32_t xbar = smem_addr(&q->xbar);
         mbar_arrive_expect_tx(xbar, (uint32_t)(a.M * w * 2));
         for (int m = 0; m < a.M; ++m)
             bulk_load_1d(smem_addr(xs + (size_t)m * w * 2), a.X + (int64_t)m * a.K + c0,
                          (uint32_t)(w * 2), xbar);
     }
+    for (int c = threadIdx.x; c < nch; c += DTHREADS) q->fl[c] = 0u;
     __syncthreads();
-    // bounded like every wait; a slice that never lands leaves nothing published
-    if (!drain_wait(xbar, 0, a.status)) return;
+    if (!drain_wait(smem_addr(&q->xbar), 0, a.status)) return;
 
-    // pass 1
-    uint32_t rmax[DM];                        // per row, max |x| over this thread's columns
-#pragma unroll
-    for (int m = 0; m < DM; ++m) rmax[m] = 0u;
-    for (int c = threadIdx.x; c < w / 8; c += DTHREADS) {
-        const int cg = c0 / 8 + c;                    // chunk index in the whole row
-        uint4 v[DM];
-#pragma unroll
-        for (int m = 0; m < DM; ++m)
-            v[m] = m < a.M ? *reinterpret_cast<const uint4 *>(xs + (size_t)m * w * 2 + c * 16)
-                           : make_uint4(0, 0, 0, 0);
-        uint32_t col[4];                              // 0xffff per outlier half
-        if (a.bitmaps) {
+    // outlier bits: thread t takes chunk t % nch and the rows congruent to t / nch
+    if (a.bitmaps) {
+        for (int c = threadIdx.x; c < nch; c += DTHREADS) {
+            const int cg = c0 / 8 + c;
             uint32_t wd = 0;
             for (int r = 0; r < a.n_bitmaps; ++r)
                 wd |= __ldg(a.bitmaps + (int64_t)r * nwords + (cg >> 2));
-            const uint32_t b = (wd >> ((cg & 3) * 8)) & 0xffu;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                col[e] = (((b >> (2 * e)) & 1u) ? 0x0000ffffu : 0u) |
-                         (((b >> (2 * e + 1)) & 1u) ? 0xffff0000u : 0u);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) col[e] = 0u;
-#pragma unroll
-            for (int m = 0; m < DM; ++m) {
-                const uint32_t *wv = reinterpret_cast<const uint32_t *>(&v[m]);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) col[e] |= hge2_bits(habs2_bits(wv[e]), a.thr2);
+            q->fl[c] = (wd >> ((cg & 3) * 8)) & 0xffu;
+        }
+    } else {
+        const int rg = max(1, min(a.M, DTHREADS / nch));  // row groups
+        if ((int)threadIdx.x < rg * nch) {
+            const int c = threadIdx.x % nch;
+            uint32_t col[4] = {0u, 0u, 0u, 0u};
+#pragma unroll 4
+            for (int m = threadIdx.x / nch; m < a.M; m += rg) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(xs + ((size_t)m * w + c * 8) * 2);
+                col[0] |= hge2_bits(habs2_bits(v.x), a.thr2);
+                col[1] |= hge2_bits(habs2_bits(v.y), a.thr2);
+                col[2] |= hge2_bits(habs2_bits(v.z), a.thr2);
+                col[3] |= hge2_bits(habs2_bits(v.w), a.thr2);
             }
-        }
-        uint32_t b = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            b |= ((col[e] & 1u) << (2 * e)) | ((col[e] >> 16 & 1u) << (2 * e + 1));
-        q->flags[c] = (uint8_t)b;
-        a.table->flags[cg] = (uint8_t)b;
-#pragma unroll
-        for (int m = 0; m < DM; ++m) {
-            const uint32_t *wv = reinterpret_cast<const uint32_t *>(&v[m]);
+            uint32_t b = 0;
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                rmax[m] = hmax2_bits(rmax[m], habs2_bits(wv[e]) & ~col[e]);
+                b |= ((col[e] & 1u) << (2 * e)) | ((col[e] >> 16 & 1u) << (2 * e + 1));
+            if (b) atomicOr(&q->fl[c], b);
         }
-    }
-    // this quantizer's row maxima: over the two halves, the warp's lanes, then the warps
-#pragma unroll
-    for (int m = 0; m < DM; ++m) {
-        uint32_t r = rmax[m];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) r = hmax2_bits(r, __shfl_xor_sync(0xffffffffu, r, o));
-        const __half2 h = *reinterpret_cast<const __half2 *>(&r);
-        if (lane == 0) q->wmax[warp][m] = fmaxf(__low2float(h), __high2float(h));
-    }
-    __syncthreads();
-    if (threadIdx.x < DM) {
-        float amax = 0.0f;
-        for (int wi = 0; wi < DWARPS; ++wi) amax = fmaxf(amax, q->wmax[wi][threadIdx.x]);
-        a.table->part[qi][threadIdx.x] = amax;
-    }
-    // publish the bits and row maxima, then take every quantizer's
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        release_word(&a.table->pready[qi], a.epoch);
-        q->ok = poll_words(a.table->pready, a.nq, a.epoch, a.status, a.timeout_ns, nullptr) ? 1 : 0;
-    }
-    __syncthreads();
-    if (!q->ok) return;
-    if (threadIdx.x < DM) {
-        float amax = 0.0f;
-        for (int r = 0; r < a.nq; ++r) amax = fmaxf(amax, __ldcg(&a.table->part[r][threadIdx.x]));
-        if ((int)threadIdx.x >= a.M) amax = 0.0f;
-        q->sca[threadIdx.x] = amax;
-        q->mult[threadIdx.x] = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
     }
     __syncthreads();
 
-    // pass 2: item (block, 16-column group, row) -> 16 codes, one 16-byte store
+    // row maxima over the slice's regular columns (warp w: rows w and w + 8); lane 0 publishes
+    // each as a tagged word
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int m = warp + 8 * r;
+        if (m >= a.M) break;                                  // uniform over the warp
+        uint32_t rm = 0u;
+#pragma unroll 4
+        for (int c = lane; c < nch; c += 32) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(xs + ((size_t)m * w + c * 8) * 2);
+            uint32_t col[4];
+            expand_bits(q->fl[c], col);
+            rm = hmax2_bits(rm, habs2_bits(v.x) & ~col[0]);
+            rm = hmax2_bits(rm, habs2_bits(v.y) & ~col[1]);
+            rm = hmax2_bits(rm, habs2_bits(v.z) & ~col[2]);
+            rm = hmax2_bits(rm, habs2_bits(v.w) & ~col[3]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) rm = hmax2_bits(rm, __shfl_xor_sync(0xffffffffu, rm, o));
+        if (lane == 0) {
+            const __half2 h = *reinterpret_cast<const __half2 *>(&rm);
+            const float amax = fmaxf(__low2float(h), __high2float(h));
+            relaxed_store(&a.table->part[qi][m], tag | __float_as_uint(amax));
+        }
+    }
+
+    // this slice's outlier count (published too) and each thread's position within the
+    // slice's list
+    const int cpt = (nch + DTHREADS - 1) / DTHREADS;
+    const int l0 = min(nch, (int)threadIdx.x * cpt), l1 = min(nch, l0 + cpt);
+    int cnt = 0;
+    for (int c = l0; c < l1; ++c) cnt += __popc(q->fl[c]);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) q->wsum[warp] = incl;
+    __syncthreads();
+    int before = 0, mine = 0;
+    for (int wi = 0; wi < DWARPS; ++wi) {
+        const int sm = q->wsum[wi];
+        before += wi < warp ? sm : 0;
+        mine += sm;
+    }
+    before += incl - cnt;
+    if (threadIdx.x == 0) relaxed_store(&a.table->part[qi][DM], tag | (uint32_t)mine);
+
+    // every quantizer's partials: words (j, m < M) and (j, DM).  Warp 0 polls; lane i loads
+    // words i, i + 32, ... together each round.
+    if (warp == 0) {
+        const int per = a.M + 1, n = a.nq * per;
+        const unsigned long long *src[QPOLL];
+        int dst[QPOLL];
+#pragma unroll
+        for (int k = 0; k < QPOLL; ++k) {
+            const int i = min(lane + 32 * k, n - 1);
+            const int j = i / per, mm = i - j * per == a.M ? DM : i - j * per;
+            src[k] = &a.table->part[j][mm];
+            dst[k] = j * (DM + 1) + mm;
+        }
+        const uint64_t t0 = global_timer_ns();
+        bool ok = false;
+        for (uint32_t it = 0;; ++it) {
+            unsigned long long v[QPOLL];
+#pragma unroll
+            for (int k = 0; k < QPOLL; ++k) v[k] = relaxed_load(src[k]);
+            bool all = true;
+#pragma unroll
+            for (int k = 0; k < QPOLL; ++k) all = all && (v[k] & 0xffffffff00000000ull) == tag;
+            if (__all_sync(0xffffffffu, all)) {
+#pragma unroll
+                for (int k = 0; k < QPOLL; ++k) q->xp[dst[k]] = v[k];
+                ok = true;
+                break;
+            }
+            __nanosleep(32);
+            if ((it & 15u) == 15u &&
+                __shfl_sync(0xffffffffu, global_timer_ns() - t0 > a.timeout_ns ? 1 : 0, 0)) {
+                break;
+            }
+        }
+        if (!ok && lane == 0) a.status.timed_out();
+        if (lane == 0) q->ok = ok ? 1 : 0;
+    }
+    __syncthreads();
+    if (!q->ok) return;                                   // timed out (uniform)
+    if (threadIdx.x < DM) {
+        float amax = 0.0f;
+        if ((int)threadIdx.x < a.M)
+            for (int j = 0; j < a.nq; ++j)
+                amax = fmaxf(amax, __uint_as_float((uint32_t)q->xp[j * (DM + 1) + threadIdx.x]));
+        q->sca[threadIdx.x] = amax;
+        q->mult[threadIdx.x] = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    } else if (threadIdx.x == DM) {
+        int bq = 0, tot = 0;
+        for (int j = 0; j < a.nq; ++j) {
+            const int cj = (int)(uint32_t)q->xp[j * (DM + 1) + DM];
+            bq += j < qi ? cj : 0;
+            tot += cj;
+        }
+        q->before = bq;
+        q->total = tot;
+    }
+    __syncthreads();
+
+    // the image of the slice; item (block, 16-column group, row) -> 16 codes, one 16-byte store
     const uint32_t blk_bytes = (uint32_t)a.rows * DBK;
     const int nblk = kb1 - kb0;
+#pragma unroll 2
     for (int i = threadIdx.x; i < nblk * 8 * a.rows; i += DTHREADS) {
         const int grp = i & 7, m = (i >> 3) % a.rows, blk = (i >> 3) / a.rows;
         uint4 code = make_uint4(0, 0, 0, 0);
         if (m < a.M) {
-            const int cl = blk * 16 + grp * 2;             // chunk within this slice
-            const uint32_t b0 = cl * 8 < w ? q->flags[cl] : 0xffu;
-            const uint32_t b1 = cl * 8 + 8 < w ? q->flags[cl + 1] : 0xffu;
-            const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)m * w * 2 + cl * 16);
+            const int cl = blk * 16 + grp * 2;             // chunk within the slice
+            const uint32_t b0 = cl * 8 < w ? q->fl[cl] : 0xffu;
+            const uint32_t b1 = cl * 8 + 8 < w ? q->fl[cl + 1] : 0xffu;
+            const uint4 *src = reinterpret_cast<const uint4 *>(xs + ((size_t)m * w + cl * 8) * 2);
             const uint4 v0 = cl * 8 < w ? src[0] : make_uint4(0, 0, 0, 0);
             const uint4 v1 = cl * 8 + 8 < w ? src[1] : make_uint4(0, 0, 0, 0);
             float f[8];
@@ -376,54 +469,37 @@ __device__ void quantize_x(const DArgs &a, uint8_t *smem) {
     // the image is read by the bulk store (async proxy)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0)
         bulk_store_1d(a.image + (size_t)kb0 * blk_bytes, smem_addr(is), (uint32_t)nblk * blk_bytes);
-        bulk_store_wait();
-        fence_proxy_async_global();
-        release_word(&a.table->iready[qi], a.epoch);
-    }
-    if (qi != 0) return;
 
-    // quantizer 0: the row scales and the ascending list of outlier columns (every
-    // quantizer's bits are published: pready above)
-    if (threadIdx.x < DM) a.table->sca[threadIdx.x] = q->sca[threadIdx.x];
-    const int cpt = (nchunks + DTHREADS - 1) / DTHREADS;
-    const int l0 = min(nchunks, (int)threadIdx.x * cpt), l1 = min(nchunks, l0 + cpt);
-    int cnt = 0;
-    for (int c = l0; c < l1; ++c) cnt += __popc((uint32_t)__ldcg(&a.table->flags[c]));
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) q->wsum[warp] = incl;
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int wi = 0; wi < DWARPS; ++wi) {
-        const int sm = q->wsum[wi];
-        before += wi < warp ? sm : 0;
-        total += sm;
-    }
-    int pos = before + incl - cnt;
+    // this slice's entries of the ascending outlier list; quantizer 0 also the row scales and
+    // the counts
+    int pos = q->before + before;
     for (int c = l0; c < l1; ++c) {
-        uint32_t b = __ldcg(&a.table->flags[c]);
+        uint32_t b = q->fl[c];
         while (b) {
             const int e = __ffs(b) - 1;
             b &= b - 1;
-            if (pos < a.cap) a.table->idx[pos] = c * 8 + e;
+            if (pos < a.cap) a.table->idx[pos] = c0 + c * 8 + e;
             ++pos;
         }
     }
-    if (threadIdx.x == 0) {
-        a.table->total = total;
-        a.table->n_out = min(total, a.cap);
-        *a.count = total;
-        a.status.set(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
+    if (qi == 0) {
+        if (threadIdx.x < DM) a.table->sca[threadIdx.x] = q->sca[threadIdx.x];
+        if (threadIdx.x == DM) {
+            const int total = q->total;
+            a.table->total = total;
+            a.table->n_out = min(total, a.cap);
+            *a.count = total;
+            a.status.set(total > a.cap ? LLMINT8_ERR_OUTLIER_CAPACITY : LLMINT8_OK);
+        }
     }
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) release_word(&a.table->ready, a.epoch);
+    if (threadIdx.x == 0) {
+        bulk_store_wait();
+        fence_proxy_async_global();
+        release_word(&a.table->done[qi], a.epoch);
+    }
 }
 
 __global__ void __launch_bounds__(DTHREADS, 1)
@@ -434,8 +510,13 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if ((int)blockIdx.x < a.nq) {
-        // the next call's kernel may launch now; this one waits for the previous grid
+        // the next call's kernel may launch now; this one waits for the previous grid before it
+        // reads X or writes the workspace
         asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        if (threadIdx.x == 0) {
+            mbar_init(smem_addr(&reinterpret_cast<QShared *>(smem)->xbar), 1);
+            fence_mbar_init();
+        }
         asm volatile("griddepcontrol.wait;" ::: "memory");
         quantize_x(a, smem);
         return;
@@ -480,17 +561,16 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
     const uint32_t tmem = tail->tmem_base;
     const BoundedWait wait{&tail->abort_flag, a.status, a.timeout_ns};
 
-    // stage j of a tile covers k-blocks DKS * sj .. (sj = j rotated by a tile-dependent
-    // offset, so that the CTAs streaming at the same moment read different column ranges of
-    // the 2^n-strided weight rows); the last one may hold a single k-block
+    // stage j of a tile: k-blocks DKS * sj .. (sj rotated by stage_rot; the last stage may hold
+    // a single k-block)
     const uint32_t kbox = (uint32_t)a.Rt * DBK;                  // one k-block of the band
-    auto rot_of = [&](int tile) { return (int)(((unsigned)tile * 7u) % (unsigned)a.nst); };
+    auto rot_of = [&](int tile) { return stage_rot(tile, a.nst); };
 
     if (warp == 0) {
         // --------------------------------------------------- weight stream (TMA) ----
         if (lane == 0) {
             const uint64_t once = policy_evict_first();
-            int stage = 0;
+            int stage = 0, issued = 0;
             uint32_t phase = 0, used = 0, last_parity = 0;
             for (int tile = band0; tile < a.tiles; tile += bands) {
                 const int rot = rot_of(tile);
@@ -498,6 +578,14 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                     int sj = j + rot;
                     if (sj >= a.nst) sj -= a.nst;
                     const int kb0 = sj * DKS, nkb = min(DKS, a.kblocks - kb0);
+                    // at most `inflight` stages on their way: a short memory queue keeps the
+                    // latency of everything else on the GPU (X, the tables, the image) low
+                    if (issued >= a.inflight) {
+                        const int prev = issued - a.inflight;
+                        if (!wait(smem_addr(&tail->full[prev % S]), (uint32_t)(prev / S) & 1u))
+                            goto drain;
+                    }
+                    ++issued;
                     if (!wait(smem_addr(&tail->empty[stage]), phase ^ 1)) goto drain;
                     const uint32_t full = smem_addr(&tail->full[stage]);
                     mbar_arrive_expect_tx(full, (uint32_t)nkb * kbox);
@@ -587,8 +675,8 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
         __syncwarp();
-        if (lane == 0 && poll_words(a.table->iready, a.nq, a.epoch, a.status, a.timeout_ns,
-                                    &tail->abort_flag)) {
+        if (lane == 0 &&
+            poll_all(a.table->done, a.nq, a.epoch, a.status, a.timeout_ns, &tail->abort_flag)) {
             fence_proxy_async_global();           // the image is read by the async proxy
             const int ntiles = (a.tiles - band0 + bands - 1) / bands;   // tiles of this CTA
             const int nstg = a.resident ? a.nst : ntiles * a.nst;
@@ -623,18 +711,16 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         const int et = threadIdx.x - 128;                 // 0..127 over the epilogue warps
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
         const float inv = 1.0f / 16129.0f;
-        // warp 4 polls quantizer 0's table; the other epilogue warps wait on it in shared memory
+        // one thread polls the quantizers' done words (acquiring what they wrote) and arrives
+        // on tbar; lane 0 of each epilogue warp acquires that by its wait on tbar, and the
+        // __syncwarp orders it before the reads of its other lanes
+        if (et == 0 &&
+            poll_all(a.table->done, a.nq, a.epoch, a.status, a.timeout_ns, &tail->abort_flag))
+            mbar_arrive(smem_addr(&tail->tbar));
         int ok = 0;
-        if (warp == 4 && lane == 0) {
-            ok = poll_words(&a.table->ready, 1, a.epoch, a.status, a.timeout_ns, &tail->abort_flag)
-                     ? 1 : 0;
-            if (ok) mbar_arrive(smem_addr(&tail->tbar));
-        } else if (lane == 0) {
-            ok = wait(smem_addr(&tail->tbar), 0) ? 1 : 0;
-        }
+        if (lane == 0) ok = wait(smem_addr(&tail->tbar), 0) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        // every lane acquires the published table itself (it is there: one load each)
-        if (ok && acquire_word(&a.table->ready) != a.epoch) ok = 0;
+        __syncwarp();
         const int n_out = ok ? a.table->n_out : 0;
         float sca[DM];
 #pragma unroll
@@ -754,7 +840,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int64_t cap, int sms) {
     DecodePlan p;
     const int64_t kblocks = ceil_div(K, DBK);
-    p.nq = (int)std::max<int64_t>(1, std::min<int64_t>(kDecodeMaxQuantizers, kblocks / QKB));
+    p.nq = (int)std::min<int64_t>(kDecodeMaxQuantizers, ceil_div(kblocks, QKB));
     p.bpq = (int)ceil_div(kblocks, p.nq);
     p.nq = (int)ceil_div(kblocks, p.bpq);                 // every quantizer owns k-blocks
     const int64_t streamers = std::max(1, sms - p.nq);
@@ -778,7 +864,8 @@ DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int64_t cap, int sms) {
     const int64_t slack = (int64_t)(DMMA_M - p.Rt) * DBK;
     const int64_t room = SMEM_LIMIT - 1024 - (int64_t)p.ring_off - slack;
     p.stages = (int)std::max<int64_t>(0, std::min<int64_t>(DMAX_STAGES, room / stage));
-    // a quantizer: tables, M x (its columns) of X, their image
+    p.inflight = std::max(1, std::min(DINFLIGHT, p.stages));
+    // a quantizer: tables, its slice of X, the image of its k-blocks
     const int64_t qsmem = QX_OFF + M * p.bpq * DBK * 2 + (int64_t)p.bpq * p.rows * DBK + 1024;
     p.smem = (int)std::max<int64_t>(p.ring_off + p.stages * stage + slack + 1024, qsmem);
     return p;
@@ -806,7 +893,8 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
         sms = sms_cache[dev];
     }
     const DecodePlan p = decode_plan(d.M, d.N, d.K, d.cap, sms);
-    if (p.stages < 2 || p.smem > SMEM_LIMIT) return cudaErrorInvalidValue;
+    if (p.stages < 2 || p.smem > SMEM_LIMIT || p.bpq * DBK / 8 > QMAX_CHUNKS)
+        return cudaErrorInvalidValue;
 
     DArgs a;
     a.X = d.X;
@@ -841,6 +929,7 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     a.tiles = p.tiles;
     a.kblocks = p.kblocks;
     a.stages = p.stages;
+    a.inflight = p.inflight;
     a.nq = p.nq;
     a.bpq = p.bpq;
     a.nst = p.nst;

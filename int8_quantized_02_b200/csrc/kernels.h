@@ -70,29 +70,29 @@ namespace llmint8 {
 
 // Decode path (M <= kDecodeMaxM, K <= kDecodeMaxK, at most kDecodeMaxOutliers outlier
 // columns): one weight-streaming tcgen05 kernel per call.  Its first CTAs quantize X (each a
-// slice of the columns) and publish the outlier columns, row scales and the int8 operand image
-// through a DecodeTable and the image in the workspace; every other CTA streams a band of
-// weight rows.
+// slice of the columns; they exchange their partial row maxima and outlier counts) and publish
+// the outlier columns, row scales and the int8 operand image through a DecodeTable and the
+// image in the workspace; every other CTA streams a band of weight rows.
 constexpr int kDecodeMaxM = 16;
 constexpr int kDecodeMaxK = 16384;
 constexpr int kDecodeMaxOutliers = 256;
 
-// What the quantizer CTAs publish (workspace, 256-byte aligned).  Every word tagged with the
-// call number is stored with release semantics after the data it covers:
-//   pready[q]  quantizer q's outlier bits (flags of its chunks) and row maxima (part[q]);
-//   iready[q]  quantizer q's k-blocks of the operand image;
-//   ready      quantizer 0's row scales, outlier list and counts.
+// What the quantizer CTAs publish (workspace, 256-byte aligned).
+//   part[q][m]  (call << 32) | fp32 bits of quantizer q's row-m maximum of |x| over the regular
+//               columns of its slice (m < kDecodeMaxM), then (call << 32) | the number of
+//               outlier columns in its slice: one 64-bit store each, so a word that carries
+//               the call's number carries its value;
+//   done[q]     the call's number, stored with release semantics once quantizer q's k-blocks of
+//               the operand image and its entries of idx are written (quantizer 0: also sca,
+//               total and n_out).
 constexpr int kDecodeMaxQuantizers = 8;
 struct DecodeTable {
-    unsigned long long ready;
-    unsigned long long pready[kDecodeMaxQuantizers];
-    unsigned long long iready[kDecodeMaxQuantizers];
+    unsigned long long done[kDecodeMaxQuantizers];
+    unsigned long long part[kDecodeMaxQuantizers][kDecodeMaxM + 1];
     int32_t total;                            // outlier columns found
     int32_t n_out;                            // ... of them listed (<= capacity)
     float sca[kDecodeMaxM];                   // row absmax over the regular columns
-    float part[kDecodeMaxQuantizers][kDecodeMaxM];   // per-quantizer row maxima
     int32_t idx[kDecodeMaxOutliers];          // outlier columns, ascending
-    uint8_t flags[kDecodeMaxK / 8];           // outlier bits of each 8-column chunk
 };
 
 // Bytes of the int8 operand image the quantizer writes: one block of 16 rows (8 when M <= 8)
@@ -107,6 +107,7 @@ struct DecodePlan {
     int tiles = 0, grid = 0, kblocks = 0;
     int rows = 0;            // rows of an operand-image block (8 or 16)
     int stages = 0, smem = 0;
+    int inflight = 0;        // weight stages a streamer keeps on their way at most
     int nq = 0;              // quantizer CTAs (the first nq of the grid)
     int bpq = 0;             // k-blocks per quantizer
     int nst = 0;             // weight stages per tile (2 k-blocks each)
