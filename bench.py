@@ -8,6 +8,8 @@ with the same keys.  Workloads (seeded synthetic inputs, int8_quantized_02_b200.
   decode     X [b, 4096] for b in (1, 8, 16), six outlier columns |x| in [6, 60] on every row;
              CB [16384, 4096] quantized once beforehand.  One step = the three llmint8_linear
              calls.  Metric: weight-streaming GB/s = sum_b (N*K + 4N + 2bK + 2bN) / time.
+  decode175b the same three calls at the 175B-class projection shape: X [b, 12288] against
+             CB [49152, 12288] (604 MB).  GB/s as for decode.
   ffn6.7b    X [2048, 4096] . W1^T (16384 outputs), then X2 [2048, 16384] . W2^T (4096 outputs);
              six outlier columns of U(6, 20) on 75 % of rows.  Metric: TOPS = 2MNK / time.
   proj175b   X [4096, 12288] . W^T (49152 outputs), W ~ N(0, 0.01).  TOPS.
@@ -185,13 +187,14 @@ def _weights(L, torch, N, K, std, copies):
 
 def build_workload(name, L, torch):
     calls = []
-    if name == "decode":
-        N, K = 16384, 4096
+    if name in DECODE_WORKLOADS:
+        make = synth.decode if name == "decode" else synth.decode175b
+        N, K, std = make(1).N, make(1).K, make(1).w_std
         copies = max(2, -(-3 * L2_BYTES // (N * K)) + 1)   # > 3 x L2 of weights in rotation
-        CBs, SCBs = _weights(L, torch, N, K, 0.02, copies)
+        CBs, SCBs = _weights(L, torch, N, K, std, copies)
         rotation = [0]
         for b in DECODE_BATCHES:
-            wl = synth.decode(b)
+            wl = make(b)
             X = torch.from_numpy(wl.make_x()[0]).cuda()
             nbytes = N * K + 4 * N + 2 * b * K + 2 * b * N
             calls.append(Call(L, torch, X, CBs, SCBs, 6.0, wl.name, nbytes,
@@ -263,8 +266,9 @@ def spread(values):
 # ------------------------------------------------------------------------ our arm ----
 
 # Seconds of timed work the repeats of each workload's region add up to.
-TARGET_S = {"decode": 1.0, "ffn6.7b": 0.5, "proj175b": 0.5, "sweep": 0.5}
-ALL_WORKLOADS = ("decode", "ffn6.7b", "proj175b", "sweep")
+TARGET_S = {"decode": 1.0, "decode175b": 0.5, "ffn6.7b": 0.5, "proj175b": 0.5, "sweep": 0.5}
+ALL_WORKLOADS = ("decode", "decode175b", "ffn6.7b", "proj175b", "sweep")
+DECODE_WORKLOADS = ("decode", "decode175b")
 
 
 def run_workload(name, args, rank, world, local_rank):
@@ -478,7 +482,7 @@ def workload_config(name, calls):
            "calls": [{"name": c.name, "M": c.M, "K": c.K, "N": c.N, "threshold": c.t,
                       "max_outliers": c.cap} for c in calls],
            "parallelism": "replicas"}
-    if name == "decode":
+    if name in DECODE_WORKLOADS:
         cfg["l2"] = (f"{len(calls[0].CBs)} rotating int8 weight copies "
                      f"({len(calls[0].CBs) * calls[0].N * calls[0].K / 2**20:.0f} MiB > 126 MiB L2)")
     else:
@@ -494,14 +498,15 @@ def _oracle_sample(name):
     of the token rows)."""
     from oracle import oracle
     pieces, units = [], 0
-    if name == "decode":
-        N, K = 16384, 4096
-        rows = 2048                                   # 1/8 of the output channels
-        CB, SCB = oracle.quantize_weight_colwise(synth.weight(rows, K, 0.02, seed=0))
+    if name in DECODE_WORKLOADS:
+        make = synth.decode if name == "decode" else synth.decode175b
+        N, K, std = make(1).N, make(1).K, make(1).w_std
+        rows = 2048 if name == "decode" else 512       # a slice of the output channels
+        CB, SCB = oracle.quantize_weight_colwise(synth.weight(rows, K, std, seed=0))
         for b in DECODE_BATCHES:
-            pieces.append((synth.decode(b).make_x()[0], CB, SCB, 6.0))
+            pieces.append((make(b).make_x()[0], CB, SCB, 6.0))
             units += rows * K + 4 * rows + 2 * b * K + 2 * b * rows
-        desc = (f"decode b=1,8,16: X [b, {K}] against {rows} of the {N} output channels")
+        desc = (f"{name} b=1,8,16: X [b, {K}] against {rows} of the {N} output channels")
         return pieces, units, desc
     specs = {"ffn6.7b": [(synth.FFN_W1, 6.0), (synth.FFN_W2, 6.0)],
              "proj175b": [(synth.PROJ_175B, 6.0)],
@@ -537,7 +542,7 @@ def cpu_baseline(name, budget_s=15.0):
         t0 = time.perf_counter()
         _oracle_step(pieces)
         times.append(time.perf_counter() - t0)
-    unit = "GB/s" if name == "decode" else "TOPS"
+    unit = "GB/s" if name in DECODE_WORKLOADS else "TOPS"
     sec = statistics.median(times)
     return {"value": unit_value(units, sec, unit), "unit": unit, "cores": _cores(),
             "kind": "oracle", "sample": f"{desc}; median of {len(times)} runs of {sec:.3f} s"}
@@ -554,7 +559,7 @@ def run_reference(args, rank, world):
     for _ in range(args.steps):
         _oracle_step(pieces)
     sec = time.perf_counter() - t0
-    unit = "GB/s" if args.workload == "decode" else "TOPS"
+    unit = "GB/s" if args.workload in DECODE_WORKLOADS else "TOPS"
     value = unit_value(units * args.steps, sec, unit)
     return {
         "impl": "reference",

@@ -52,7 +52,8 @@ typedef enum {
     LLMINT8_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the matching *_workspace_size() */
     LLMINT8_ERR_OUTLIER_CAPACITY = 4,    /* (device) more outlier columns than the capacity */
     LLMINT8_ERR_TIMEOUT = 5,             /* (device) a bounded wait in a kernel gave up */
-    LLMINT8_ERR_CUDA = 6                 /* a CUDA runtime call or launch failed */
+    LLMINT8_ERR_CUDA = 6,                /* a CUDA runtime call or launch failed */
+    LLMINT8_ERR_DEVICE_CHECK = 7         /* (device, debug build only) a bounds check failed */
 } llmint8_status;
 
 /*
@@ -198,7 +199,8 @@ LLMINT8_API llmint8_status llmint8_dequant(const int8_t *CB, const float *SCB, i
 /*
  * Synchronizes `stream` and returns the device status word of a workspace used by the
  * last llmint8_linear / llmint8_quantize_rows_and_find_outliers call on it
- * (LLMINT8_OK, LLMINT8_ERR_OUTLIER_CAPACITY or LLMINT8_ERR_TIMEOUT), or LLMINT8_ERR_CUDA.
+ * (LLMINT8_OK, LLMINT8_ERR_OUTLIER_CAPACITY, LLMINT8_ERR_TIMEOUT or, in the debug build,
+ * LLMINT8_ERR_DEVICE_CHECK), or LLMINT8_ERR_CUDA.
  * The result is meaningful only for a workspace that at least one call has used; a
  * zero-filled one reads LLMINT8_OK.
  */
@@ -230,6 +232,17 @@ LLMINT8_API llmint8_status llmint8_workspace_outlier_weights(const void *ws, int
 
 /* Static English text for a status code. */
 LLMINT8_API const char *llmint8_status_string(llmint8_status status);
+
+/*
+ * Build flags of the loaded library: bit 0 is set in the debug build (libllmint8_debug.so,
+ * compiled with LLMINT8_DEBUG).  There the kernels also check, on the device, that every
+ * outlier column index they list or read is below K, that no more than the capacity are
+ * listed, and that every tile they store lies inside its output; a failed check records
+ * LLMINT8_ERR_DEVICE_CHECK in the workspace's device status (read with
+ * llmint8_device_status) and the kernel carries on without trapping.  Results are otherwise
+ * the release build's, bit for bit.
+ */
+LLMINT8_API int llmint8_build_flags(void);
 
 /*
  * Upper bound, in nanoseconds, of every wait inside the GEMM and decode kernels of later calls

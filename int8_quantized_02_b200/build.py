@@ -1,6 +1,11 @@
 """Builds the sm_100a shared library ``libllmint8.so`` in-tree with nvcc.
 
-    python -m int8_quantized_02_b200.build [--force] [--verbose-ptxas]
+    python -m int8_quantized_02_b200.build [--force] [--verbose-ptxas] [--debug]
+
+``--debug`` builds ``libllmint8_debug.so`` instead: the same sources compiled with
+``LLMINT8_DEBUG``, whose kernels add device-side bounds checks that record
+LLMINT8_ERR_DEVICE_CHECK in the workspace status (the binding loads it when the environment
+variable LLMINT8_DEBUG is 1).
 """
 from __future__ import annotations
 
@@ -14,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libllmint8.so")
+LIB_DEBUG = os.path.join(PKG, "libllmint8_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -32,27 +38,31 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + \
         glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *NVCC_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}"]
+    if debug:
+        cmd += ["-DLLMINT8_DEBUG"]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     cmd += ["-o", tmp, *sources()]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose_ptxas="--verbose-ptxas" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose_ptxas="--verbose-ptxas" in sys.argv,
+                debug="--debug" in sys.argv))

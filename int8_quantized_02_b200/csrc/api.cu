@@ -6,12 +6,39 @@
 #include <atomic>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
 using namespace llmint8;
 
 namespace {
+
+// An NVTX range (domain "llmint8", named after the entry point) around every call that
+// launches work, so that a profiler's timeline shows the layer's calls.  Without a tool
+// attached it costs a pointer test.
+class CallRange {
+  public:
+    explicit CallRange(const char *name) {
+        nvtxEventAttributes_t e = {};
+        e.version = NVTX_VERSION;
+        e.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+        e.messageType = NVTX_MESSAGE_TYPE_ASCII;
+        e.message.ascii = name;
+        nvtxDomainRangePushEx(domain(), &e);
+    }
+    ~CallRange() { nvtxDomainRangePop(domain()); }
+    CallRange(const CallRange &) = delete;
+    CallRange &operator=(const CallRange &) = delete;
+
+  private:
+    static nvtxDomainHandle_t domain() {
+        static const nvtxDomainHandle_t d = nvtxDomainCreateA("llmint8");
+        return d;
+    }
+};
+#define LLMINT8_CALL_RANGE() CallRange llmint8_call_range_(__func__)
 
 constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
@@ -177,8 +204,17 @@ const char *llmint8_status_string(llmint8_status s) {
         case LLMINT8_ERR_OUTLIER_CAPACITY: return "more outlier columns than the capacity";
         case LLMINT8_ERR_TIMEOUT: return "a bounded wait in a kernel timed out";
         case LLMINT8_ERR_CUDA: return "CUDA error";
+        case LLMINT8_ERR_DEVICE_CHECK: return "a device-side bounds check failed (debug build)";
     }
     return "unknown status";
+}
+
+int llmint8_build_flags(void) {
+#ifdef LLMINT8_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 llmint8_status llmint8_set_wait_timeout_ns(uint64_t ns) {
@@ -198,6 +234,7 @@ size_t llmint8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t ma
 
 llmint8_status llmint8_quantize_weight_colwise(const uint16_t *W, int64_t N, int64_t K,
                                                int8_t *CB, float *SCB, void *stream) {
+    LLMINT8_CALL_RANGE();
     if (!W || !CB || !SCB) return LLMINT8_ERR_INVALID_ARG;
     if (!aligned16(W) || !aligned16(CB) || !aligned4(SCB)) return LLMINT8_ERR_INVALID_ARG;
     if (!shape_ok_mk(N, K)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
@@ -207,6 +244,7 @@ llmint8_status llmint8_quantize_weight_colwise(const uint16_t *W, int64_t N, int
 
 llmint8_status llmint8_dequant(const int8_t *CB, const float *SCB, int64_t N, int64_t K,
                                uint16_t *W_out, void *stream) {
+    LLMINT8_CALL_RANGE();
     if (!CB || !SCB || !W_out) return LLMINT8_ERR_INVALID_ARG;
     if (!aligned16(CB) || !aligned16(W_out) || !aligned4(SCB)) return LLMINT8_ERR_INVALID_ARG;
     if (!shape_ok_mk(N, K)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
@@ -219,6 +257,7 @@ llmint8_status llmint8_quantize_rows_and_find_outliers(const uint16_t *X, int64_
                                                        int32_t *outlier_idx, int32_t *n_outliers,
                                                        int64_t cap, void *ws, size_t ws_bytes,
                                                        void *stream) {
+    LLMINT8_CALL_RANGE();
     if (!X || !Xq || !SCA || !n_outliers || !ws || (cap > 0 && !outlier_idx))
         return LLMINT8_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(Xq) || !aligned4(SCA) || !aligned4(n_outliers) ||
@@ -300,6 +339,7 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
                               const uint16_t *W_fp16, float threshold, int64_t max_outliers,
                               uint16_t *Y, void *ws, size_t ws_bytes, void *stream,
                               int32_t *C_debug) {
+    LLMINT8_CALL_RANGE();
     const llmint8_status chk = check_linear(X, M, K, CB, SCB, N, bias, W_fp16, threshold,
                                             max_outliers, Y, ws, ws_bytes, C_debug);
     if (chk != LLMINT8_OK) return chk;
@@ -350,6 +390,7 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
 
 llmint8_status llmint8_outlier_bitmap(const uint16_t *X, int64_t M, int64_t K, float threshold,
                                      uint32_t *bitmap, void *ws, size_t ws_bytes, void *stream) {
+    LLMINT8_CALL_RANGE();
     if (!X || !bitmap || !ws) return LLMINT8_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned4(bitmap) || !aligned16(ws)) return LLMINT8_ERR_INVALID_ARG;
     if (isnan(threshold)) return LLMINT8_ERR_INVALID_ARG;
@@ -369,6 +410,7 @@ llmint8_status llmint8_linear_with_bitmaps(const uint16_t *X, int64_t M, int64_t
                                            const uint32_t *bitmaps, int64_t n_bitmaps,
                                            int64_t max_outliers, uint16_t *Y, void *ws,
                                            size_t ws_bytes, void *stream, int32_t *C_debug) {
+    LLMINT8_CALL_RANGE();
     if (!bitmaps || !aligned4(bitmaps)) return LLMINT8_ERR_INVALID_ARG;
     if (n_bitmaps < 1 || n_bitmaps > kMaxBitmaps) return LLMINT8_ERR_INVALID_ARG;
     // the threshold plays no part: 6 only satisfies the shared checks
@@ -416,6 +458,7 @@ llmint8_status llmint8_linear_host(const uint16_t *X_host, int64_t M, int64_t K,
                                    const uint16_t *bias, const uint16_t *W_fp16, float threshold,
                                    int64_t max_outliers, uint16_t *Y_host, uint16_t *X_dev,
                                    uint16_t *Y_dev, void *ws, size_t ws_bytes, void *stream) {
+    LLMINT8_CALL_RANGE();
     if (!X_host || !Y_host) return LLMINT8_ERR_INVALID_ARG;
     const llmint8_status chk = check_linear(X_dev, M, K, CB, SCB, N, bias, W_fp16, threshold,
                                             max_outliers, Y_dev, ws, ws_bytes, nullptr);
@@ -439,7 +482,8 @@ llmint8_status llmint8_device_status(const void *ws, void *stream) {
     if (cudaMemcpy(words, ws, sizeof(words), cudaMemcpyDeviceToHost) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     // epochs start at 1: a zero-filled header has recorded no call and no timeout
-    if ((words[0] >> 4) != 0 && (words[1] >> 4) == (words[0] >> 4)) return LLMINT8_ERR_TIMEOUT;
+    if ((words[0] >> 4) != 0 && (words[1] >> 4) == (words[0] >> 4))
+        return static_cast<llmint8_status>(words[1] & 0xFull);
     return static_cast<llmint8_status>(words[0] & 0xFull);
 }
 
@@ -456,6 +500,7 @@ llmint8_status llmint8_workspace_outlier_count(const void *ws, void *stream, int
 llmint8_status llmint8_workspace_outlier_weights(const void *ws, int64_t M, int64_t N, int64_t K,
                                                  int64_t max_outliers, uint16_t *Wo,
                                                  int64_t n_cols, void *stream) {
+    LLMINT8_CALL_RANGE();
     if (!ws || !Wo || !aligned16(ws) || !aligned16(Wo)) return LLMINT8_ERR_INVALID_ARG;
     if (!shape_ok_mk(M, K) || !shape_ok_n(N)) return LLMINT8_ERR_UNSUPPORTED_SHAPE;
     if (max_outliers < 0 || max_outliers > K || n_cols < 0 || n_cols > max_outliers)
@@ -533,6 +578,7 @@ llmint8_status llmint8_linear_noalloc(const uint16_t *X, int64_t M, int64_t K, c
                                       const uint16_t *W_fp16, float threshold,
                                       int64_t max_outliers, uint16_t *Y, void *stream,
                                       void **scratch_out) {
+    LLMINT8_CALL_RANGE();
     if (!X || !CB || !SCB || !Y) return LLMINT8_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(CB) || !aligned16(SCB) || !aligned16(Y) ||
         (bias && !aligned16(bias)) || (W_fp16 && !aligned16(W_fp16)))

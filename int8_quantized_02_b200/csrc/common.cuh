@@ -15,7 +15,8 @@ namespace llmint8 {
 // Layout of the first 256 bytes of every workspace.
 struct WsHeader {
     unsigned long long status;   // (call epoch << 4) | llmint8_status, one writer per call
-    unsigned long long timeout;  // (call epoch << 4) | LLMINT8_ERR_TIMEOUT after a timeout
+    unsigned long long timeout;  // (call epoch << 4) | LLMINT8_ERR_TIMEOUT after a timeout (or,
+                                 // debug build, | LLMINT8_ERR_DEVICE_CHECK after a failed check)
     int32_t n_outliers;          // true number of outlier columns found by the last call
     uint32_t pad[59];
 };
@@ -63,10 +64,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Device-side conditions of a call.  Every call gets a new epoch.  Exactly one thread of
 // the call stores (epoch << 4) | code into the status word (the outlier-count result,
 // written before anything can time out in that kernel); any thread whose bounded wait
-// gives up stores (epoch << 4) | TIMEOUT into the timeout word.  The host reports TIMEOUT
-// when both words carry the same epoch, else the status word's code.  Plain stores of one
-// value per word: no ordering between CTAs or kernels matters and the workspace needs no
-// initialization.
+// gives up stores (epoch << 4) | TIMEOUT into the timeout word, and in the debug build any
+// thread whose device check fails stores (epoch << 4) | DEVICE_CHECK there.  The host
+// reports the timeout word's code when both words carry the same epoch, else the status
+// word's code.  Plain stores of one value per word: no ordering between CTAs or kernels
+// matters and the workspace needs no initialization.
 struct StatusRef {
     unsigned long long *word;
     unsigned long long *timeout_word;
@@ -78,7 +80,25 @@ struct StatusRef {
         *reinterpret_cast<volatile unsigned long long *>(timeout_word) =
             tag | (unsigned long long)LLMINT8_ERR_TIMEOUT;
     }
+    __device__ __forceinline__ void check_failed() const {
+        *reinterpret_cast<volatile unsigned long long *>(timeout_word) =
+            tag | (unsigned long long)LLMINT8_ERR_DEVICE_CHECK;
+    }
 };
+
+// Device-side bounds check of the debug build (compiled with LLMINT8_DEBUG): a false
+// condition records LLMINT8_ERR_DEVICE_CHECK through `status` and execution goes on.  The
+// release build compiles it to nothing.
+#ifdef LLMINT8_DEBUG
+#define LLMINT8_DCHECK(cond, status)          \
+    do {                                      \
+        if (!(cond)) (status).check_failed(); \
+    } while (0)
+#else
+#define LLMINT8_DCHECK(cond, status) \
+    do {                             \
+    } while (0)
+#endif
 
 // Every wait of a pipeline goes through this: it gives up after `timeout_ns`, or as soon
 // as another thread of the CTA gave up, records LLMINT8_ERR_TIMEOUT in the workspace

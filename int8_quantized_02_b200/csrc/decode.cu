@@ -480,6 +480,7 @@ __device__ void quantize_x(const DArgs &a, uint8_t *smem) {
         while (b) {
             const int e = __ffs(b) - 1;
             b &= b - 1;
+            LLMINT8_DCHECK(c0 + c * 8 + e < a.K, a.status);
             if (pos < a.cap) a.table->idx[pos] = c0 + c * 8 + e;
             ++pos;
         }
@@ -726,7 +727,11 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
 #pragma unroll
         for (int mm = 0; mm < DM; ++mm) sca[mm] = ok ? a.table->sca[mm] : 0.0f;
         // the outlier columns and X at them (a 16-row [j][m] table; rows >= M hold 0)
-        for (int i = et; i < n_out; i += 128) tail->idx[i] = a.table->idx[i];
+        LLMINT8_DCHECK(n_out >= 0 && n_out <= a.cap, a.status);
+        for (int i = et; i < n_out; i += 128) {
+            tail->idx[i] = a.table->idx[i];
+            LLMINT8_DCHECK(tail->idx[i] >= 0 && tail->idx[i] < a.K, a.status);
+        }
         for (int i = et; i < n_out * DM; i += 128) {
             const int j = i / DM, mm = i % DM;
             xo[i] = mm < a.M ? a.X[(int64_t)mm * a.K + a.table->idx[j]] : __float2half_rn(0.0f);
@@ -806,6 +811,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 for (int mm = 0; mm < DM; ++mm) {
                     if (mm < a.M) {
                         const float y = fmaf((float)(int32_t)d[mm], sca[mm] * scale, o[mm]);
+                        LLMINT8_DCHECK(mm < a.M && n < a.N, a.status);
                         a.Y[(int64_t)mm * a.N + n] = __float2half_rn(y);
                         if (a.C_debug) a.C_debug[(int64_t)mm * a.N + n] = (int32_t)d[mm];
                     }

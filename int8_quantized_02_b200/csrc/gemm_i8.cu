@@ -227,6 +227,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
 
     // Outlier configuration of this call (uniform over the grid).
     const int n_out = (int)min((int64_t)*a.count, a.cap);
+    LLMINT8_DCHECK(n_out >= 0 && n_out <= a.cap && n_out <= a.K, a.status);
     const bool all_outliers = n_out >= a.K;            // then C == 0: skip the int8 blocks
     const bool reg_out = n_out > 0 && n_out <= kRegOutliers && !all_outliers;
     const int nob = reg_out ? 0 : (n_out + 63) / 64;   // fp16 k-blocks of 64 columns
@@ -497,6 +498,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                                 packed[j4 * 2] = pack_half2(y[0], y[1]);
                                 packed[j4 * 2 + 1] = pack_half2(y[2], y[3]);
                             }
+                            LLMINT8_DCHECK(row < a.M && nb + g * 16 + 16 <= a.N, a.status);
                             uint4 *dst = reinterpret_cast<uint4 *>(yrow + g * 16);
                             dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
                             dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);

@@ -208,6 +208,7 @@ outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t
         while (v) {
             const int b = __ffs(v) - 1;
             v &= v - 1;
+            LLMINT8_DCHECK((w0 + i) * 32 + b < K, status);
             if (pos < cap) idx[pos] = (int32_t)((w0 + i) * 32 + b);
             ++pos;
         }

@@ -13,7 +13,10 @@ import threading
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libllmint8.so")
+# LLMINT8_DEBUG=1 selects the debug build (device-side bounds checks; see llmint8_build_flags)
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "libllmint8_debug.so" if os.environ.get("LLMINT8_DEBUG") == "1"
+                         else "libllmint8.so")
 _lock = threading.Lock()
 _lib = None
 
@@ -24,6 +27,7 @@ ERR_WORKSPACE_TOO_SMALL = 3
 ERR_OUTLIER_CAPACITY = 4
 ERR_TIMEOUT = 5
 ERR_CUDA = 6
+ERR_DEVICE_CHECK = 7
 
 # Names and prototypes exactly as declared in include/llmint8.h.
 _P, _I64, _F32, _SZ, _U64 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t,
@@ -40,6 +44,7 @@ PROTOTYPES = {
     "llmint8_device_status": (ctypes.c_int, [_P, _P]),
     "llmint8_workspace_outlier_count": (ctypes.c_int, [_P, _P, _P]),
     "llmint8_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "llmint8_build_flags": (ctypes.c_int, []),
     "llmint8_set_wait_timeout_ns": (ctypes.c_int, [_U64]),
     "llmint8_set_profile_events": (ctypes.c_int, [_P, _P]),
     "llmint8_kernel_launch_count": (_U64, []),
@@ -91,6 +96,11 @@ def load():
 
 def status_string(code: int) -> str:
     return load().llmint8_status_string(int(code)).decode()
+
+
+def build_flags() -> int:
+    """llmint8_build_flags(): bit 0 set when the loaded library is the debug build."""
+    return int(load().llmint8_build_flags())
 
 
 llmint8_status_string = status_string

@@ -100,6 +100,13 @@ def decode(batch: int) -> Workload:
     return Workload(f"decode_b{batch}", batch, 4096, 16384, 6, 6.0, 60.0, 1.0, 0.02)
 
 
+def decode175b(batch: int) -> Workload:
+    """Decode at the 175B-class projection shape: X [batch, 12288] with the projection's
+    activation recipe (six outlier columns of U(6, 20) on 75 % of rows); W [49152 out,
+    12288 in] ~ N(0, 0.01), quantized once beforehand."""
+    return Workload(f"decode175b_b{batch}", batch, 12288, 49152, 6, 6.0, 20.0, 0.75, 0.01)
+
+
 FFN_W1 = Workload("ffn6.7b_w1", 2048, 4096, 16384, 6, 6.0, 20.0, 0.75, 0.02)
 FFN_W2 = Workload("ffn6.7b_w2", 2048, 16384, 4096, 6, 6.0, 20.0, 0.75, 0.02)
 PROJ_175B = Workload("proj175b", 4096, 12288, 49152, 6, 6.0, 20.0, 0.75, 0.01)

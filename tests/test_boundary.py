@@ -55,10 +55,25 @@ def test_only_the_c_abi_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(7):
+    for code in range(8):
         s = llmint8.status_string(code)
         assert s and s != "unknown status"
     assert llmint8.status_string(99) == "unknown status"
+
+
+def test_release_and_debug_builds_export_the_same_abi(lib):
+    # the release library reports no debug checks; the debug build (LLMINT8_DEBUG) reports
+    # them and exports exactly the same symbols
+    assert llmint8.build_flags() & 1 == 0
+    path = build_mod.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    dbg.llmint8_build_flags.restype = ctypes.c_int
+    assert dbg.llmint8_build_flags() & 1 == 1
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True,
+                         check=True).stdout
+    assert set(re.findall(r"\bT (\w+)", out)) == set(declared_functions())
+    dbg.llmint8_status_string.restype = ctypes.c_char_p
+    assert b"debug" in dbg.llmint8_status_string(llmint8.ERR_DEVICE_CHECK)
 
 
 def test_workspace_sizes(lib):

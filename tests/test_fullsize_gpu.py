@@ -1,7 +1,8 @@
 """Parity at the full sizes of the benchmark workloads, through the calls the benchmark times.
 
 Every workload of the benchmark - decode (X [b, 4096], b = 1, 8, 16, against CB [16384, 4096]),
-the 6.7B-class FFN pair, the 175B-class projection and the outlier-density sweep - is run on
+decode at the 175B-class projection shape (X [b, 12288] against CB [49152, 12288]), the
+6.7B-class FFN pair, the 175B-class projection and the outlier-density sweep - is run on
 the GPU at its full size with the benchmark's threshold and outlier capacity.  The int8 weight
 (CB, SCB), the quantized rows (Xq, SCA) and the outlier column list are compared bit for bit
 in full; the layer output is compared in full for the decode shapes (the oracle finishes
@@ -130,6 +131,13 @@ def test_ffn_full_size(wl):
 
 def test_proj175b_full_size():
     _check(synth.PROJ_175B, 6.0, 512)
+
+
+@pytest.mark.parametrize("batch", [1, 16])
+def test_decode175b_full_size(batch):
+    # decode at the 175B-class projection shape (K = 12288 past the 8192 of the decode
+    # workload, N = 49152): the single-kernel decode path, output compared in full
+    _check(synth.decode175b(batch), 6.0, 64)
 
 
 @pytest.mark.parametrize("n_out,threshold", [(0, 6.0), (6, 6.0), (64, 6.0), (512, 6.0),
