@@ -12,6 +12,11 @@ with the same keys.  Workloads (seeded synthetic inputs, int8_quantized_02_b200.
              CB [49152, 12288] (604 MB).  GB/s as for decode.
   ffn6.7b    X [2048, 4096] . W1^T (16384 outputs), then X2 [2048, 16384] . W2^T (4096 outputs);
              six outlier columns of U(6, 20) on 75 % of rows.  Metric: TOPS = 2MNK / time.
+  ffn6.7b_chain  the FFN pair chained: W2 takes W1's output Y1 as its X.  The W1 call
+             (llmint8_linear_next_bitmaps) also writes the outlier bitmaps of Y1, and the W2
+             call (llmint8_linear_with_bitmaps) uses them, so it makes no outlier scan of its
+             own.  Y1 of these random weights has about 700 columns reaching 6.0 (capacity
+             1024).  TOPS.
   proj175b   X [4096, 12288] . W^T (49152 outputs), W ~ N(0, 0.01).  TOPS.
   sweep      X [4096, 8192] . W^T (8192 outputs); one step = K' in {0, 6, 64, 512} at
              threshold 6, plus threshold=inf and threshold=0.  TOPS.
@@ -174,6 +179,78 @@ class Call:
         plans[i]()
 
 
+class ChainHead(Call):
+    """The first layer of a chained pair: llmint8_linear_next_bitmaps, which also writes the
+    outlier bitmaps of its Y (`bits`) for the second layer."""
+
+    def __init__(self, *args, next_threshold=6.0, **kw):
+        self.next_t = next_threshold
+        super().__init__(*args, **kw)
+
+    def _call(self, X):
+        L, torch = self.L, self.torch
+        if not hasattr(self, "bits"):
+            self.bits = torch.empty(((self.M + 31) // 32, (self.N + 31) // 32),
+                                    dtype=torch.int32, device="cuda")
+        fn = L.load().llmint8_linear_next_bitmaps
+        args = (L._ptr(X), self.M, self.K, L._ptr(self.CBs[0]), L._ptr(self.SCBs[0]), self.N,
+                None, None, L.ctypes.c_float(self.t), self.cap, L._ptr(self.Y), L._ptr(self.ws),
+                self.ws.numel(), L._stream(None), None, L.ctypes.c_float(self.next_t),
+                L._ptr(self.bits))
+
+        def call():
+            code = fn(*args)
+            if code != L.OK:
+                raise L.LLMInt8Error(code, "llmint8_linear_next_bitmaps")
+        return call
+
+    def plan(self, X=None):
+        return [self._call(self.X if X is None else X)]
+
+    def host_plan(self, X_host, Y_host, X_dev, stream):
+        run = self._call(X_dev)
+
+        def call():
+            X_dev.copy_(X_host, non_blocking=True)
+            run()
+        return [call]
+
+
+class ChainTail(Call):
+    """The second layer of a chained pair: llmint8_linear_with_bitmaps on the head's Y with
+    the head's bitmaps (no outlier scan of its own)."""
+
+    def __init__(self, L, torch, head, CBs, SCBs, name, units, kernel_bytes, d2h_bytes, cap):
+        self.head = head
+        super().__init__(L, torch, head.Y, CBs, SCBs, head.next_t, name, units, kernel_bytes,
+                         0, d2h_bytes, cap, [0])
+
+    def _call(self):
+        L = self.L
+        fn = L.load().llmint8_linear_with_bitmaps
+        bits = self.head.bits
+        args = (L._ptr(self.head.Y), self.M, self.K, L._ptr(self.CBs[0]), L._ptr(self.SCBs[0]),
+                self.N, None, None, L._ptr(bits), bits.shape[0], self.cap, L._ptr(self.Y),
+                L._ptr(self.ws), self.ws.numel(), L._stream(None), None)
+
+        def call():
+            code = fn(*args)
+            if code != L.OK:
+                raise L.LLMInt8Error(code, "llmint8_linear_with_bitmaps")
+        return call
+
+    def plan(self, X=None):
+        return [self._call()]
+
+    def host_plan(self, X_host, Y_host, X_dev, stream):
+        run = self._call()
+
+        def call():
+            run()
+            Y_host.copy_(self.Y, non_blocking=True)
+        return [call]
+
+
 def _weights(L, torch, N, K, std, copies):
     W = torch.from_numpy(synth.weight(N, K, std, seed=0)).cuda()
     CB, SCB = L.llmint8_quantize_weight_colwise(W)
@@ -201,6 +278,18 @@ def build_workload(name, L, torch):
                               N * K + 4 * N + b * K + 4 * b + 2 * b * N, 2 * b * K, 2 * b * N, 64,
                               rotation))
         unit, metric_bound = "GB/s", "hbm"
+    elif name == "ffn6.7b_chain":
+        w1, w2 = synth.FFN_W1, synth.FFN_W2
+        CB1, SCB1 = _weights(L, torch, w1.N, w1.K, w1.w_std, 1)
+        CB2, SCB2 = _weights(L, torch, w2.N, w2.K, w2.w_std, 1)
+        X = torch.from_numpy(w1.make_x()[0]).cuda()
+        head = ChainHead(L, torch, X, CB1, SCB1, 6.0, "ffn6.7b_w1_next_bitmaps", w1.int8_ops,
+                         w1.M * w1.K * 2 + w1.N * w1.K + 2 * w1.M * w1.N,
+                         2 * w1.M * w1.K, 0, 512, [0], next_threshold=6.0)
+        tail = ChainTail(L, torch, head, CB2, SCB2, "ffn6.7b_w2_with_bitmaps", w2.int8_ops,
+                         w2.M * w2.K * 2 + w2.N * w2.K + 2 * w2.M * w2.N, 2 * w2.M * w2.N, 1024)
+        calls = [head, tail]
+        unit, metric_bound = "TOPS", "tensor"
     elif name in ("ffn6.7b", "proj175b", "sweep"):
         if name == "ffn6.7b":
             specs = [(synth.FFN_W1, 6.0), (synth.FFN_W2, 6.0)]
@@ -266,8 +355,9 @@ def spread(values):
 # ------------------------------------------------------------------------ our arm ----
 
 # Seconds of timed work the repeats of each workload's region add up to.
-TARGET_S = {"decode": 1.0, "decode175b": 0.5, "ffn6.7b": 0.5, "proj175b": 0.5, "sweep": 0.5}
-ALL_WORKLOADS = ("decode", "decode175b", "ffn6.7b", "proj175b", "sweep")
+TARGET_S = {"decode": 1.0, "decode175b": 0.5, "ffn6.7b": 0.5, "ffn6.7b_chain": 0.5,
+            "proj175b": 0.5, "sweep": 0.5}
+ALL_WORKLOADS = ("decode", "decode175b", "ffn6.7b", "ffn6.7b_chain", "proj175b", "sweep")
 DECODE_WORKLOADS = ("decode", "decode175b")
 
 
@@ -405,7 +495,7 @@ def run_workload(name, args, rank, world, local_rank):
     e2e_vals = [whole_job_value(step_units, args.steps, world, t, unit) for t in e2e_times]
     check_status(" (end to end)")
     for j, c in enumerate(calls):
-        if not torch.equal(hosts[j][1], c.Y.cpu()):
+        if c.d2h_bytes and not torch.equal(hosts[j][1], c.Y.cpu()):
             raise SystemExit(f"{c.name} (end to end): host Y differs from the device Y")
 
     out = {
@@ -509,6 +599,9 @@ def _oracle_sample(name):
         desc = (f"{name} b=1,8,16: X [b, {K}] against {rows} of the {N} output channels")
         return pieces, units, desc
     specs = {"ffn6.7b": [(synth.FFN_W1, 6.0), (synth.FFN_W2, 6.0)],
+             # the chain's arithmetic is the layer's (its bitmaps are the outlier detection the
+             # oracle's layer makes): the same sample as the FFN pair
+             "ffn6.7b_chain": [(synth.FFN_W1, 6.0), (synth.FFN_W2, 6.0)],
              "proj175b": [(synth.PROJ_175B, 6.0)],
              "sweep": [(synth.sweep(k), 6.0) for k in (0, 6, 64, 512)]
              + [(synth.sweep(6, float("inf")), float("inf")), (synth.sweep(0, 0.0), 0.0)]}[name]

@@ -127,6 +127,34 @@ LLMINT8_API llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t 
 LLMINT8_API size_t llmint8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t max_outliers);
 
 /*
+ * llmint8_linear_next_bitmaps: llmint8_linear that also finds, while it writes Y, the outlier
+ * columns of a next layer that takes Y as its input X.  Outliers are found per feature column
+ * of a layer's input (blog section LLM.int8() 温和总结, step 1), so for that layer they are
+ * the columns of Y where some row reaches its threshold; forming them here saves the next
+ * call the pass over its input that llmint8_linear makes to find them.  X, M, K, CB, SCB, N,
+ * bias, W_fp16, threshold, max_outliers, Y, ws, ws_bytes, stream and C_debug, and every
+ * result, are as for llmint8_linear.  Then:
+ *   next_threshold  the next layer's threshold (rules as in
+ *                   llmint8_quantize_rows_and_find_outliers: <= 0 marks every column; NaN ->
+ *                   LLMINT8_ERR_INVALID_ARG).
+ *   next_bitmaps    uint32 [ceil(M/32)][ceil(N/32)], device, 4-byte aligned, owned by the
+ *                   caller, fully overwritten: bit (n % 32) of word [b][n / 32] is set iff some
+ *                   row m of the 32-row block b (32 b <= m < min(M, 32 b + 32)) has
+ *                   |Y[m, n]| >= next_threshold, Y as stored (fp16).  Give them to the next
+ *                   layer's llmint8_linear_with_bitmaps with n_bitmaps = ceil(M/32).
+ * The GEMM path forms each word in the epilogue that writes those values of Y (an OR over a
+ * warp's 32 rows; no atomics); the decode path ORs each warp's 32 output columns into the
+ * words, which its kernel zeroes first.
+ */
+LLMINT8_API llmint8_status llmint8_linear_next_bitmaps(const uint16_t *X, int64_t M, int64_t K,
+                                           const int8_t *CB, const float *SCB, int64_t N,
+                                           const uint16_t *bias, const uint16_t *W_fp16,
+                                           float threshold, int64_t max_outliers, uint16_t *Y,
+                                           void *ws, size_t ws_bytes, void *stream,
+                                           int32_t *C_debug, float next_threshold,
+                                           uint32_t *next_bitmaps);
+
+/*
  * Token-parallel (M-split) layers.  When the rows of X are split over ranks, the outlier set
  * must still be that of the whole X: an outlier column is one where ANY row reaches the
  * threshold (blog section LLM.int8() 温和总结: outliers are found per feature column of the
@@ -256,8 +284,9 @@ LLMINT8_API llmint8_status llmint8_set_wait_timeout_ns(uint64_t ns);
  * Measurement hooks (no counterpart on the pages; they let a benchmark time the product
  * kernel of a call with CUDA events and count launches):
  *   llmint8_set_profile_events(start, stop): two cudaEvent_t.  While both are non-NULL,
- *     every llmint8_linear call records `start` on its stream immediately before its
- *     product kernel (the GEMM; on the decode path, the pair of decode kernels) and `stop`
+ *     every llmint8_linear, llmint8_linear_next_bitmaps, llmint8_linear_with_bitmaps and
+ *     llmint8_linear_noalloc call records `start` on its stream immediately before its
+ *     product kernel (the GEMM; on the decode path, the decode kernel) and `stop`
  *     immediately after it.  NULL, NULL disables.
  *     Process-wide; the caller owns the events and must keep them alive while set.
  *   llmint8_kernel_launch_count(): number of kernels this library has launched in the

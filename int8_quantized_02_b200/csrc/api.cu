@@ -157,6 +157,8 @@ DecodeLaunch decode_launch(const uint16_t *X, int64_t M, int64_t K, const int8_t
     d.wo_pitch = 0;
     d.bitmaps = nullptr;
     d.n_bitmaps = 0;
+    d.ybits = nullptr;
+    d.ythreshold = 0.0f;
     d.count = &h->n_outliers;
     d.table = table;
     d.image = image;
@@ -175,6 +177,15 @@ llmint8_status run_decode(const DecodeLaunch &d, cudaStream_t s) {
     cudaEvent_t ev0 = g_prof_start.load(), ev1 = g_prof_stop.load();
     if (ev0 && record_profile_event(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
     if (launch_decode(d, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (ev1 && record_profile_event(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    return LLMINT8_OK;
+}
+
+// launch_gemm between the process-wide profile events (when set).
+llmint8_status run_gemm(const GemmLaunch &g, cudaStream_t s) {
+    cudaEvent_t ev0 = g_prof_start.load(), ev1 = g_prof_stop.load();
+    if (ev0 && record_profile_event(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (launch_gemm(g, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
     if (ev1 && record_profile_event(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
     return LLMINT8_OK;
 }
@@ -319,6 +330,8 @@ GemmLaunch gemm_launch(const LinearLayout &L, void *ws, const int8_t *CB, const 
     g.bias = reinterpret_cast<const __half *>(bias);
     g.Y = reinterpret_cast<__half *>(Y);
     g.C_debug = C_debug;
+    g.ybits = nullptr;
+    g.ythreshold = 0.0f;
     g.status = status;
     g.M = M;
     g.N = N;
@@ -330,16 +343,13 @@ GemmLaunch gemm_launch(const LinearLayout &L, void *ws, const int8_t *CB, const 
 // Upper bound of the bitmaps one llmint8_linear_with_bitmaps call merges (ranks).
 constexpr int64_t kMaxBitmaps = 65536;
 
-}  // namespace
-
-extern "C" {
-
-llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
-                              const float *SCB, int64_t N, const uint16_t *bias,
-                              const uint16_t *W_fp16, float threshold, int64_t max_outliers,
-                              uint16_t *Y, void *ws, size_t ws_bytes, void *stream,
-                              int32_t *C_debug) {
-    LLMINT8_CALL_RANGE();
+// llmint8_linear, and with ybits non-null also the outlier bitmaps of Y for the next layer
+// (llmint8_linear_next_bitmaps).
+llmint8_status linear_call(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
+                           const float *SCB, int64_t N, const uint16_t *bias,
+                           const uint16_t *W_fp16, float threshold, int64_t max_outliers,
+                           uint16_t *Y, void *ws, size_t ws_bytes, void *stream,
+                           int32_t *C_debug, uint32_t *ybits, float ythreshold) {
     const llmint8_status chk = check_linear(X, M, K, CB, SCB, N, bias, W_fp16, threshold,
                                             max_outliers, Y, ws, ws_bytes, C_debug);
     if (chk != LLMINT8_OK) return chk;
@@ -348,7 +358,6 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     WsHeader *h = at<WsHeader>(ws, 0);
     const StatusRef status = next_status(h);
     const __half *Xh = reinterpret_cast<const __half *>(X);
-    cudaEvent_t ev0 = g_prof_start.load(), ev1 = g_prof_stop.load();
     cudaError_t e;
 
     if (use_decode_path(M, K, threshold, max_outliers)) {
@@ -361,6 +370,8 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
             d.Wo = at<__half>(ws, L.wo);
             d.wo_pitch = L.pitch;
         }
+        d.ybits = ybits;
+        d.ythreshold = ythreshold;
         return run_decode(d, s);
     }
 
@@ -371,7 +382,8 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
     __half *Xo = at<__half>(ws, L.xo);
     __half *Wo = at<__half>(ws, L.wo);
 
-    e = launch_outlier_detect(Xh, M, K, threshold, L.plan, at<uint32_t>(ws, L.partial), bitmap,
+    e = launch_outlier_detect(Xh, M, K, threshold, L.plan, at<uint32_t>(ws, L.partial),
+                              bitmap,
                               idx, max_outliers, &h->n_outliers, status, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     e = launch_quantize_rows(Xh, M, K, bitmap, idx, &h->n_outliers, max_outliers, L.pitch, Xq, SCA,
@@ -379,13 +391,38 @@ llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int
                              reinterpret_cast<const __half *>(W_fp16), N,
                              max_outliers > 0 ? Wo : nullptr, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-    const GemmLaunch g = gemm_launch(L, ws, CB, SCB, bias, Y, C_debug, status, M, N, K,
-                                     max_outliers);
-    if (ev0 && record_profile_event(ev0, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
-    e = launch_gemm(g, s);
-    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-    if (ev1 && record_profile_event(ev1, s) != cudaSuccess) return LLMINT8_ERR_CUDA;
-    return LLMINT8_OK;
+    GemmLaunch g = gemm_launch(L, ws, CB, SCB, bias, Y, C_debug, status, M, N, K, max_outliers);
+    g.ybits = ybits;
+    g.ythreshold = ythreshold;
+    return run_gemm(g, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+llmint8_status llmint8_linear(const uint16_t *X, int64_t M, int64_t K, const int8_t *CB,
+                              const float *SCB, int64_t N, const uint16_t *bias,
+                              const uint16_t *W_fp16, float threshold, int64_t max_outliers,
+                              uint16_t *Y, void *ws, size_t ws_bytes, void *stream,
+                              int32_t *C_debug) {
+    LLMINT8_CALL_RANGE();
+    return linear_call(X, M, K, CB, SCB, N, bias, W_fp16, threshold, max_outliers, Y, ws,
+                       ws_bytes, stream, C_debug, nullptr, 0.0f);
+}
+
+llmint8_status llmint8_linear_next_bitmaps(const uint16_t *X, int64_t M, int64_t K,
+                                           const int8_t *CB, const float *SCB, int64_t N,
+                                           const uint16_t *bias, const uint16_t *W_fp16,
+                                           float threshold, int64_t max_outliers, uint16_t *Y,
+                                           void *ws, size_t ws_bytes, void *stream,
+                                           int32_t *C_debug, float next_threshold,
+                                           uint32_t *next_bitmaps) {
+    LLMINT8_CALL_RANGE();
+    if (!next_bitmaps || !aligned4(next_bitmaps) || isnan(next_threshold))
+        return LLMINT8_ERR_INVALID_ARG;
+    return linear_call(X, M, K, CB, SCB, N, bias, W_fp16, threshold, max_outliers, Y, ws,
+                       ws_bytes, stream, C_debug, next_bitmaps, next_threshold);
 }
 
 llmint8_status llmint8_outlier_bitmap(const uint16_t *X, int64_t M, int64_t K, float threshold,
@@ -399,7 +436,8 @@ llmint8_status llmint8_outlier_bitmap(const uint16_t *X, int64_t M, int64_t K, f
     if (ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE_TOO_SMALL;
     WsHeader *h = at<WsHeader>(ws, 0);
     return from_cuda(launch_outlier_detect(reinterpret_cast<const __half *>(X), M, K, threshold,
-                                           L.plan, at<uint32_t>(ws, L.partial), bitmap,
+                                           L.plan, at<uint32_t>(ws, L.partial),
+                                           bitmap,
                                            at<int32_t>(ws, L.idx), K, &h->n_outliers,
                                            next_status(h), static_cast<cudaStream_t>(stream)));
 }
@@ -448,9 +486,8 @@ llmint8_status llmint8_linear_with_bitmaps(const uint16_t *X, int64_t M, int64_t
                              reinterpret_cast<const __half *>(W_fp16), N,
                              max_outliers > 0 ? Wo : nullptr, s);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-    return from_cuda(launch_gemm(gemm_launch(L, ws, CB, SCB, bias, Y, C_debug, status, M, N, K,
-                                             max_outliers),
-                                 s));
+    return run_gemm(gemm_launch(L, ws, CB, SCB, bias, Y, C_debug, status, M, N, K, max_outliers),
+                    s);
 }
 
 llmint8_status llmint8_linear_host(const uint16_t *X_host, int64_t M, int64_t K,

@@ -7,6 +7,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "llmint8.h"
 
@@ -85,6 +86,44 @@ struct StatusRef {
             tag | (unsigned long long)LLMINT8_ERR_DEVICE_CHECK;
     }
 };
+
+// Packed-half helpers on raw bits: |x| (clear the sign bits), |x| >= t per half (0xffff
+// where true), max per half.  fp16 comparisons and maxima are exact.
+__device__ __forceinline__ uint32_t habs2_bits(uint32_t v) { return v & 0x7fff7fffu; }
+__device__ __forceinline__ uint32_t hge2_bits(uint32_t a, uint32_t t) {
+    return __hge2_mask(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&t));
+}
+__device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
+    const __half2 r = __hmax2(*reinterpret_cast<const __half2 *>(&a),
+                              *reinterpret_cast<const __half2 *>(&b));
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+// A threshold t > 0 as the smallest fp16 >= t, in both halves of a word: for an fp16 x,
+// |x| >= t exactly when |x| >= that value (fp16 compares, packed two at a time).
+inline uint32_t fp16_threshold_pair(float t) {
+    const __half t16 = __float2half_ru(t);
+    const uint32_t tb = (uint32_t)*reinterpret_cast<const uint16_t *>(&t16);
+    return tb | (tb << 16);
+}
+
+// For a threshold t > 0: the smallest fp32 f >= 0 with |fp16_rn(f)| >= (the smallest fp16
+// >= t), so that for every fp32 y, |fp16_rn(y)| >= t exactly when |y| >= f (fp16 rounding to
+// nearest is monotone).  Found by bisection over the non-negative fp32 bit patterns.
+inline float fp16_rounded_threshold_f32(float t) {
+    const float t16 = __half2float(__float2half_ru(t));   // may be +inf
+    uint32_t lo = 0u, hi = 0x7f800000u;                     // f(hi) = +inf qualifies
+    while (lo < hi) {
+        const uint32_t mid = lo + (hi - lo) / 2;
+        float f;
+        memcpy(&f, &mid, 4);
+        if (__half2float(__float2half_rn(f)) >= t16) hi = mid;
+        else lo = mid + 1;
+    }
+    float f;
+    memcpy(&f, &lo, 4);
+    return f;
+}
 
 // Device-side bounds check of the debug build (compiled with LLMINT8_DEBUG): a false
 // condition records LLMINT8_ERR_DEVICE_CHECK through `status` and execution goes on.  The

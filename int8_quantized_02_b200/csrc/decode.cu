@@ -129,18 +129,6 @@ __device__ __forceinline__ void tma_load_2d_policy(uint32_t dst, const CUtensorM
         : "memory");
 }
 
-// Packed-half helpers on raw bits: |x| (clear the sign bits), |x| >= t per half (0xffff
-// where true), max per half.  fp16 comparisons and maxima are exact.
-__device__ __forceinline__ uint32_t habs2_bits(uint32_t v) { return v & 0x7fff7fffu; }
-__device__ __forceinline__ uint32_t hge2_bits(uint32_t a, uint32_t t) {
-    return __hge2_mask(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&t));
-}
-__device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
-    const __half2 r = __hmax2(*reinterpret_cast<const __half2 *>(&a),
-                              *reinterpret_cast<const __half2 *>(&b));
-    return *reinterpret_cast<const uint32_t *>(&r);
-}
-
 // Shared memory of the quantizer CTA.
 constexpr int QMAX_CHUNKS = 256;         // 8-column chunks of a slice (16 k-blocks)
 constexpr int QWORDS = kDecodeMaxQuantizers * (DM + 1);
@@ -188,6 +176,10 @@ struct DArgs {
     int64_t wo_pitch;
     const uint32_t *bitmaps;             // [n_bitmaps][ceil(K/32)] given outlier set, or null
     int n_bitmaps;
+    uint32_t *ybits;                     // [ceil(N/32)] outlier bitmap of Y for the next
+                                         // layer, or null (zeroed by quantizer 0)
+    float ytf;                           // its threshold on the fp32 value
+    int ybits_all;                       // threshold <= 0: every column
     int32_t *count;
     DecodeTable *table;                  // workspace: what the quantizer publishes
     uint8_t *image;                      // workspace: the int8 operand image, block by block
@@ -486,6 +478,9 @@ __device__ void quantize_x(const DArgs &a, uint8_t *smem) {
         }
     }
     if (qi == 0) {
+        // the streamers OR their columns into Y's bitmap only after they acquire done[0]
+        if (a.ybits)
+            for (int i = threadIdx.x; i < (a.N + 31) / 32; i += DTHREADS) a.ybits[i] = 0u;
         if (threadIdx.x < DM) a.table->sca[threadIdx.x] = q->sca[threadIdx.x];
         if (threadIdx.x == DM) {
             const int total = q->total;
@@ -806,6 +801,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
             if (lane == 0) mbar_arrive(smem_addr(&tail->acc_empty[acc]));
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
+            bool yflag = false;   // some |fp16 Y[m, n]| >= the next layer's threshold
             if (live) {
 #pragma unroll
                 for (int mm = 0; mm < DM; ++mm) {
@@ -814,7 +810,19 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                         LLMINT8_DCHECK(mm < a.M && n < a.N, a.status);
                         a.Y[(int64_t)mm * a.N + n] = __float2half_rn(y);
                         if (a.C_debug) a.C_debug[(int64_t)mm * a.N + n] = (int32_t)d[mm];
+                        // |fp16(y)| >= the next threshold <=> |y| >= ytf
+                        yflag = yflag || a.ybits_all || fabsf(y) >= a.ytf;
                     }
+                }
+            }
+            if (a.ybits) {
+                // this warp's 32 consecutive columns, ORed into the one or two words they
+                // straddle (bands need not start on a multiple of 32)
+                const uint32_t bal = __ballot_sync(0xffffffffu, yflag);
+                const int c0 = tile * a.Rt + qd * 32, sh = c0 & 31;
+                if (lane == 0 && bal) {
+                    atomicOr(a.ybits + (c0 >> 5), bal << sh);
+                    if (sh && (bal >> (32 - sh))) atomicOr(a.ybits + (c0 >> 5) + 1, bal >> (32 - sh));
                 }
             }
         }
@@ -914,6 +922,9 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     a.wo_pitch = d.wo_pitch;
     a.bitmaps = d.bitmaps;
     a.n_bitmaps = (int)d.n_bitmaps;
+    a.ybits = d.ybits;
+    a.ytf = d.ybits && d.ythreshold > 0.0f ? fp16_rounded_threshold_f32(d.ythreshold) : 0.0f;
+    a.ybits_all = d.ybits && d.ythreshold <= 0.0f ? 1 : 0;
     a.count = d.count;
     a.table = d.table;
     a.image = d.image;
@@ -924,12 +935,7 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     a.K = (int)d.K;
     a.cap = (int)d.cap;
     a.threshold = d.threshold;
-    {
-        // smallest fp16 >= threshold (threshold > 0 here), in both halves
-        const __half t16 = __float2half_ru(d.threshold);
-        const uint32_t tb = (uint32_t)*reinterpret_cast<const uint16_t *>(&t16);
-        a.thr2 = tb | (tb << 16);
-    }
+    a.thr2 = fp16_threshold_pair(d.threshold);   // threshold > 0 on this path
     a.rows = p.rows;
     a.Rt = p.Rt;
     a.tiles = p.tiles;

@@ -102,6 +102,10 @@ struct Args {
     const __half *bias;
     __half *Y;
     int32_t *C_debug;
+    uint32_t *ybits;         // outlier bitmaps of Y for the next layer, or null
+    int ybits_words;         // ceil(N / 32)
+    float ytf;               // its threshold on the fp32 value (fp16_rounded_threshold_f32)
+    int ybits_all;           // threshold <= 0: every column
     StatusRef status;
     int M, N, K;
     int num_kb;
@@ -474,6 +478,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                     for (int j = 0; j < 32; ++j) pf[j] = __float_as_uint(p[j]);
                 }
                 const int groups = min(32, a.N - nb) / 16;   // 1 or 2 groups of 16 columns
+                uint32_t ymask = 0;   // bit j: |fp16 Y[row, nb + j]| >= the next threshold
                 if (row_ok) {
                     __half *yrow = a.Y + (int64_t)row * a.N + nb;
                     int32_t *crow = a.C_debug ? a.C_debug + (int64_t)row * a.N + nb : nullptr;
@@ -495,6 +500,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                                     y[e] = fmaf((float)(int32_t)ci[j], rs * sbv[e],
                                                 __uint_as_float(pf[j]) + b[e]);
                                 }
+                                if (a.ybits) {
+                                    // |fp16(y)| >= the next threshold <=> |y| >= ytf
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e)
+                                        ymask |= (fabsf(y[e]) >= a.ytf ? 1u : 0u)
+                                                 << (g * 16 + j4 * 4 + e);
+                                }
                                 packed[j4 * 2] = pack_half2(y[0], y[1]);
                                 packed[j4 * 2 + 1] = pack_half2(y[2], y[3]);
                             }
@@ -511,6 +523,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                                                        ci[g * 16 + v * 4 + 3]);
                             }
                         }
+                    }
+                }
+                if (a.ybits) {
+                    // OR over the warp's 32 rows: one word of this 32-row block's bitmap
+                    if (a.ybits_all && row_ok) ymask = groups == 2 ? 0xffffffffu : 0xffffu;
+                    const uint32_t word = __reduce_or_sync(0xffffffffu, ymask);
+                    if (lane == 0 && m0 + q * 32 < a.M) {
+                        LLMINT8_DCHECK(nb < a.N, a.status);
+                        a.ybits[(int64_t)((m0 + q * 32) >> 5) * a.ybits_words + (nb >> 5)] = word;
                     }
                 }
             }
@@ -656,6 +677,10 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s) {
     a.bias = g.bias;
     a.Y = g.Y;
     a.C_debug = g.C_debug;
+    a.ybits = g.ybits;
+    a.ybits_words = (int)ceil_div(g.N, 32);
+    a.ytf = g.ybits && g.ythreshold > 0.0f ? fp16_rounded_threshold_f32(g.ythreshold) : 0.0f;
+    a.ybits_all = g.ybits && g.ythreshold <= 0.0f ? 1 : 0;
     a.status = g.status;
     a.M = (int)g.M;
     a.N = (int)g.N;

@@ -58,6 +58,9 @@ struct GemmLaunch {
     const __half *bias;      // [N] or null
     __half *Y;               // [M, N]
     int32_t *C_debug;        // [M, N] or null
+    uint32_t *ybits;         // [ceil(M/32)][ceil(N/32)] outlier bitmaps of Y for the next
+                             // layer (|Y| >= ythreshold per column and 32-row block), or null
+    float ythreshold;
     StatusRef status;
     int64_t M, N, K;
     uint64_t timeout_ns;
@@ -129,6 +132,8 @@ struct DecodeLaunch {
     int64_t wo_pitch;
     const uint32_t *bitmaps; // [n_bitmaps][ceil(K/32)]: the outlier set given, or null
     int64_t n_bitmaps;
+    uint32_t *ybits;         // [ceil(N/32)]: outlier bitmap of Y for the next layer, or null
+    float ythreshold;
     int32_t *count;          // device outlier count (workspace header)
     DecodeTable *table;      // workspace
     uint8_t *image;          // workspace: decode_image_bytes(M, K), 1024-byte aligned

@@ -39,6 +39,8 @@ PROTOTYPES = {
     "llmint8_quantize_workspace_size": (_SZ, [_I64, _I64]),
     "llmint8_linear": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _F32, _I64, _P, _P,
                                       _SZ, _P, _P]),
+    "llmint8_linear_next_bitmaps": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _F32,
+                                                   _I64, _P, _P, _SZ, _P, _P, _F32, _P]),
     "llmint8_linear_workspace_size": (_SZ, [_I64, _I64, _I64, _I64]),
     "llmint8_dequant": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "llmint8_device_status": (ctypes.c_int, [_P, _P]),
@@ -216,6 +218,43 @@ def llmint8_linear(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor, bias=No
                                  workspace.numel(), _stream(stream), _ptr(C_debug)),
            "llmint8_linear")
     return Y
+
+
+def llmint8_linear_next_bitmaps(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
+                                next_threshold: float = 6.0, bias=None, W_fp16=None,
+                                threshold: float = 6.0, max_outliers: int | None = None, Y=None,
+                                next_bitmaps=None, workspace=None, C_debug=None, stream=None):
+    """llmint8_linear that also returns the outlier bitmaps of Y for a next layer taking Y as
+    its input: (Y, bitmaps uint32 [ceil(M/32), ceil(N/32)]), ready for that layer's
+    llmint8_linear_with_bitmaps."""
+    M, K = X.shape
+    N = CB.shape[0]
+    _want(X, torch.float16, (M, K), "X")
+    _want(CB, torch.int8, (N, K), "CB")
+    _want(SCB, torch.float32, (N,), "SCB")
+    if bias is not None:
+        _want(bias, torch.float16, (N,), "bias")
+    if W_fp16 is not None:
+        _want(W_fp16, torch.float16, (N, K), "W_fp16")
+    if C_debug is not None:
+        _want(C_debug, torch.int32, (M, N), "C_debug")
+    cap = default_max_outliers(K, threshold) if max_outliers is None else int(max_outliers)
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    _want(Y, torch.float16, (M, N), "Y")
+    shape = ((M + 31) // 32, (N + 31) // 32)
+    if next_bitmaps is None:
+        next_bitmaps = torch.empty(shape, dtype=torch.int32, device=X.device)
+    if next_bitmaps.dtype not in (torch.int32, torch.uint32) or \
+            tuple(next_bitmaps.shape) != shape or not next_bitmaps.is_contiguous():
+        raise ValueError(f"next_bitmaps: want a contiguous 32-bit tensor of shape {shape}")
+    if workspace is None:
+        workspace = torch.empty((llmint8_linear_workspace_size(M, N, K, cap),), dtype=torch.uint8,
+                                device=X.device)
+    _check(load().llmint8_linear_next_bitmaps(
+        _ptr(X), M, K, _ptr(CB), _ptr(SCB), N, _ptr(bias), _ptr(W_fp16), ctypes.c_float(threshold),
+        cap, _ptr(Y), _ptr(workspace), workspace.numel(), _stream(stream), _ptr(C_debug),
+        ctypes.c_float(next_threshold), _ptr(next_bitmaps)), "llmint8_linear_next_bitmaps")
+    return Y, next_bitmaps
 
 
 def llmint8_linear_fp16_weight(X: torch.Tensor, W: torch.Tensor, bias=None,

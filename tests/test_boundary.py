@@ -105,6 +105,19 @@ def test_wait_timeout_setter(lib):
     assert lib.llmint8_set_wait_timeout_ns(ctypes.c_uint64(0)) == 0   # restores the default
 
 
+def test_next_bitmaps_arguments_are_checked_before_any_launch(lib):
+    # a missing or misaligned bitmap output, or a NaN next threshold, is rejected on the host
+    fake = ctypes.c_void_p(1 << 20)     # aligned, never dereferenced: the checks come first
+    args = lambda nt, bits: (fake, 64, 1024, fake, fake, 1024, None, None,  # noqa: E731
+                             ctypes.c_float(6.0), 64, fake, fake, 1 << 30, None, None,
+                             ctypes.c_float(nt), bits)
+    assert lib.llmint8_linear_next_bitmaps(*args(6.0, None)) == llmint8.ERR_INVALID_ARG
+    assert lib.llmint8_linear_next_bitmaps(*args(6.0, ctypes.c_void_p((1 << 20) + 2))) == \
+        llmint8.ERR_INVALID_ARG
+    assert lib.llmint8_linear_next_bitmaps(*args(float("nan"), fake)) == \
+        llmint8.ERR_INVALID_ARG
+
+
 def test_argument_errors_before_any_launch(lib):
     # null pointers and bad shapes are rejected on the host, before any CUDA call
     assert lib.llmint8_linear(None, 16, 1024, None, None, 1024, None, None,
