@@ -248,80 +248,117 @@ struct GatherW {
     int64_t N;
 };
 
-// One CTA per row of X; CTAs past the last row gather Wo, one warp per weight row.
-// Row values stay in registers for K <= 8 * 256 * kCache.
+// Row quantization.  A CTA takes rows_per_cta rows, tpr = 256 / rows_per_cta threads each
+// (tpr a power of two, 32 ... 256, chosen so that a thread holds up to kCache 8-column chunks
+// of its row in registers); CTAs past the last row block gather Wo, one warp per weight row.
+// In packed fp16: the outlier halves of each chunk are cleared with a mask expanded from the
+// bitmap byte, the row absmax is a maximum of |x| pairs (exact), and the codes are
+// fl32(x * fl32(127 / absmax)) rounded half to even by adding 1.5 * 2^23 (exact for these
+// magnitudes), whose low byte is the int8 code.
 constexpr int kCache = 8;
 
-__global__ void __launch_bounds__(kThreads)
+// 0xffff in each half of the four words of a chunk whose outlier bit is set in b
+__device__ __forceinline__ void chunk_mask(uint32_t b, uint32_t (&m)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        m[e] = (((b >> (2 * e)) & 1u) ? 0x0000ffffu : 0u) |
+               (((b >> (2 * e + 1)) & 1u) ? 0xffff0000u : 0u);
+}
+__device__ __forceinline__ uint32_t hmax2_u32(uint32_t a, uint32_t b) {
+    const __half2 r = __hmax2(*reinterpret_cast<const __half2 *>(&a),
+                              *reinterpret_cast<const __half2 *>(&b));
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+// |x| pairs of a chunk with the outlier halves cleared, folded into the running maximum
+__device__ __forceinline__ uint32_t chunk_absmax(const uint4 &v, uint32_t skip, uint32_t acc) {
+    uint32_t m[4];
+    chunk_mask(skip, m);
+    acc = hmax2_u32(acc, v.x & 0x7fff7fffu & ~m[0]);
+    acc = hmax2_u32(acc, v.y & 0x7fff7fffu & ~m[1]);
+    acc = hmax2_u32(acc, v.z & 0x7fff7fffu & ~m[2]);
+    acc = hmax2_u32(acc, v.w & 0x7fff7fffu & ~m[3]);
+    return acc;
+}
+// the eight int8 codes of a chunk (0 at the outlier columns, and everywhere when s == 0)
+__device__ __forceinline__ uint2 chunk_codes(const uint4 &v, uint32_t skip, float s) {
+    uint32_t m[4];
+    chunk_mask(skip, m);
+    const uint32_t w[4] = {v.x & ~m[0], v.y & ~m[1], v.z & ~m[2], v.w & ~m[3]};
+    uint32_t c[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[e]));
+        c[2 * e] = __float_as_uint(__fadd_rn(__fmul_rn(f.x, s), 12582912.0f));
+        c[2 * e + 1] = __float_as_uint(__fadd_rn(__fmul_rn(f.y, s), 12582912.0f));
+    }
+    return make_uint2(__byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040),
+                                  0x5410),
+                      __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040),
+                                  0x5410));
+}
+
+__global__ void __launch_bounds__(kThreads, 4)
 quantize_rows_kernel(const __half *__restrict__ X, int64_t M, int64_t K,
                      const uint32_t *__restrict__ bitmap, const int32_t *__restrict__ idx,
                      const int32_t *__restrict__ count, int64_t cap, int64_t xo_pitch,
                      int8_t *__restrict__ Xq, float *__restrict__ SCA, __half *__restrict__ Xo,
-                     const GatherW gw) {
+                     int tpr_log2, int64_t row_ctas, const GatherW gw) {
     pdl_wait_then_release();
-    __shared__ float red[32];
-    const int64_t row = blockIdx.x;
-    if (row >= M) {
-        const int64_t n = (row - M) * (kThreads / 32) + (threadIdx.x >> 5);
+    __shared__ uint32_t red[kThreads / 32];
+    if ((int64_t)blockIdx.x >= row_ctas) {
+        const int64_t n = ((int64_t)blockIdx.x - row_ctas) * (kThreads / 32) + (threadIdx.x >> 5);
         if (n < gw.N)
             gather_w_row(gw.CB, gw.SCB, gw.W16, n, K, idx, min((int64_t)*count, cap), xo_pitch,
                          gw.Wo, threadIdx.x & 31);
         return;
     }
+    const int tpr = 1 << tpr_log2;
+    const int t = threadIdx.x & (tpr - 1);
+    const int64_t row = (int64_t)blockIdx.x * (kThreads >> tpr_log2) + (threadIdx.x >> tpr_log2);
+    const bool live = row < M;
     const int64_t nchunks = K / 8;
-    const uint4 *xr = reinterpret_cast<const uint4 *>(X + row * K);
+    const uint4 *xr = reinterpret_cast<const uint4 *>(X + (live ? row : 0) * K);
     uint4 cache[kCache];
-    float amax = 0.0f;
+    uint32_t skipc[kCache / 4] = {};         // the chunks' outlier bytes, four to a word
 #pragma unroll
     for (int i = 0; i < kCache; ++i) {       // issue every load before using any
-        const int64_t c = threadIdx.x + (int64_t)i * kThreads;
-        cache[i] = c < nchunks ? xr[c] : make_uint4(0, 0, 0, 0);
+        const int64_t c = t + (int64_t)i * tpr;
+        const bool in = live && c < nchunks;
+        cache[i] = in ? xr[c] : make_uint4(0, 0, 0, 0);
+        if (in) skipc[i / 4] |= ((bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu) << (8 * (i % 4));
     }
+    uint32_t am = 0u;                        // |x| maxima, fp16 pairs
 #pragma unroll
-    for (int i = 0; i < kCache; ++i) {
-        const int64_t c = threadIdx.x + (int64_t)i * kThreads;
-        if (c < nchunks) {
-            const uint32_t skip = (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu;
-            float f[8];
-            unpack8(cache[i], f);
+    for (int i = 0; i < kCache; ++i)
+        am = chunk_absmax(cache[i], (skipc[i / 4] >> (8 * (i % 4))) & 0xffu, am);
+    for (int64_t c = t + (int64_t)kCache * tpr; live && c < nchunks; c += tpr)
+        am = chunk_absmax(xr[c], (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu, am);
+    // the row's maximum: over the warp, then over the row's warps
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if (!((skip >> e) & 1u)) amax = fmaxf(amax, fabsf(f[e]));
-        }
-    }
-    for (int64_t c = threadIdx.x + (int64_t)kCache * kThreads; c < nchunks; c += kThreads) {
-        const uint32_t skip = (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu;
-        float f[8];
-        unpack8(xr[c], f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            if (!((skip >> e) & 1u)) amax = fmaxf(amax, fabsf(f[e]));
-    }
-    amax = block_max(amax, red);
-    if (threadIdx.x == 0) SCA[row] = amax;
+    for (int o = 16; o > 0; o >>= 1) am = hmax2_u32(am, __shfl_xor_sync(0xffffffffu, am, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
+    __syncthreads();
+    const int wpr = tpr >> 5;                // warps per row
+    const int w0 = (threadIdx.x >> 5) & ~(wpr - 1);
+    for (int w = 0; w < wpr; ++w) am = hmax2_u32(am, red[w0 + w]);
+    const __half2 h = *reinterpret_cast<const __half2 *>(&am);
+    const float amax = fmaxf(__low2float(h), __high2float(h));
+    if (!live) return;
+    if (t == 0) SCA[row] = amax;
     const float s = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
     uint2 *qr = reinterpret_cast<uint2 *>(Xq + row * K);
 #pragma unroll
     for (int i = 0; i < kCache; ++i) {
-        const int64_t c = threadIdx.x + (int64_t)i * kThreads;
-        if (c < nchunks) {
-            const uint32_t skip = (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu;
-            float f[8];
-            unpack8(cache[i], f);
-            qr[c] = quant8(f, s, amax > 0.0f ? skip : 0xffu);
-        }
+        const int64_t c = t + (int64_t)i * tpr;
+        if (c < nchunks) qr[c] = chunk_codes(cache[i], (skipc[i / 4] >> (8 * (i % 4))) & 0xffu, s);
     }
-    for (int64_t c = threadIdx.x + (int64_t)kCache * kThreads; c < nchunks; c += kThreads) {
-        const uint32_t skip = (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu;
-        float f[8];
-        unpack8(xr[c], f);
-        qr[c] = quant8(f, s, amax > 0.0f ? skip : 0xffu);
-    }
+    for (int64_t c = t + (int64_t)kCache * tpr; c < nchunks; c += tpr)
+        qr[c] = chunk_codes(xr[c], (bitmap[c >> 2] >> ((c & 3) * 8)) & 0xffu, s);
     if (Xo != nullptr) {
         const int64_t n_o = min((int64_t)*count, cap);
         const int64_t n_o64 = align_up(n_o, 64);
         const __half *x = X + row * K;
-        for (int64_t j = threadIdx.x; j < n_o64; j += kThreads)
+        for (int64_t j = t; j < n_o64; j += tpr)
             Xo[row * xo_pitch + j] = j < n_o ? x[idx[j]] : __float2half_rn(0.0f);
     }
 }
@@ -475,9 +512,14 @@ cudaError_t launch_quantize_rows(const __half *X, int64_t M, int64_t K, const ui
     gw.Wo = Wo;
     gw.N = Wo != nullptr ? N : 0;
     const int64_t gather_ctas = ceil_div(gw.N, kThreads / 32);
-    const cudaError_t e = launch_pdl(quantize_rows_kernel, dim3((unsigned)(M + gather_ctas)),
-                                     dim3(kThreads), s, X, M, K, bitmap, idx, count, cap,
-                                     xo_pitch, Xq, SCA, Xo, gw);
+    // threads per row: enough for kCache chunks each, 32 ... 256
+    int tpr_log2 = 5;
+    while (tpr_log2 < 8 && ((int64_t)kCache << tpr_log2) < K / 8) ++tpr_log2;
+    const int64_t row_ctas = ceil_div(M, kThreads >> tpr_log2);
+    const cudaError_t e = launch_pdl(quantize_rows_kernel,
+                                     dim3((unsigned)(row_ctas + gather_ctas)), dim3(kThreads), s,
+                                     X, M, K, bitmap, idx, count, cap, xo_pitch, Xq, SCA, Xo,
+                                     tpr_log2, row_ctas, gw);
     note_launches(1);
     return e;
 }
