@@ -123,6 +123,32 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
         "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar_cluster)
         : "memory");
 }
+// The same loads with an L2 eviction policy.  The quantized rows Xq are re-read by every wave
+// of output tiles (the tiles walk M fastest), so their loads ask L2 to evict them last; the
+// weight loads keep the default policy (the 16 M tiles of a weight tile do not all run at the
+// same moment, and evict-first weights were re-read from HBM: 2.78 against 1.72 GB per
+// launch on the 175B projection, while evict-last Xq alone gives 1.55 GB).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap *tm, int x, int y,
+                                                 uint32_t bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar), "l"(pol)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap *tm, int x,
+                                                      int y, uint32_t bar_cluster, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar_cluster), "l"(pol)
+        : "memory");
+}
 __device__ __forceinline__ void mma_i8_pair(uint32_t d, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -248,6 +274,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer ----
         if (lane == 0) {
+            const uint64_t keep = l2_policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t used = 0, last_parity = 0;   // per stage: issued at least once / parity
@@ -265,10 +292,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                     if (kb < nkb) {
                         const int kr = rotated_kblock(kb, tile / a.tiles_m, nkb);
                         if (PAIR) {
-                            tma_load_2d_pair(sa, &tmA, kr * BKB, m0, fbar);
+                            tma_load_2d_pair_hint(sa, &tmA, kr * BKB, m0, fbar, keep);
                             tma_load_2d_pair(sa + A_BYTES, &tmB, kr * BKB, n0, fbar);
                         } else {
-                            tma_load_2d(sa, &tmA, kr * BKB, m0, full);
+                            tma_load_2d_hint(sa, &tmA, kr * BKB, m0, full, keep);
                             tma_load_2d(sa + A_BYTES, &tmB, kr * BKB, n0, full);
                         }
                     } else {

@@ -162,6 +162,10 @@ LINEAR_CASES = {
     "outliers_16_epilogue": (200, 1024, 528, 16, 6.0, True, False),
     "outliers_17_tensor_cores": (200, 1024, 528, 17, 6.0, True, False),
     "outliers_9_fp16_w": (150, 512, 272, 9, 6.0, True, True),
+    # the tensor-core outlier product on CTA pairs and single CTAs, one and two fp16 k-blocks
+    "outliers_40_tensor_cores_pair": (300, 4096, 528, 40, 6.0, True, False),
+    "outliers_64_tensor_cores_single": (100, 4096, 272, 64, 6.0, False, False),
+    "outliers_65_tensor_cores": (200, 8192, 272, 65, 6.0, True, False),
     "K32_half_outliers": (40, 32, 64, 16, 6.0, False, False),
 }
 
