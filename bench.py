@@ -463,8 +463,9 @@ def run_workload(name, args, rank, world, local_rank):
                                  world, device="cuda") for j in range(len(calls))]
         achieved = step_units / sum(call_s) / 1e12
         peak, roof_unit = 2.0 * peaks["bf16_tflops"], "TOPS"   # int8 = 2 x bf16 (nominal)
-        kernel_name = ("llmint8_gemm_pair_kernel" if all(c.M > 128 for c in calls)
-                       else "llmint8_gemm_kernel")
+        kernel_name = ", ".join(dict.fromkeys(
+            ("llmint8_gemm_pair" if c.M > 128 else "llmint8_gemm")
+            + ("_bits" if isinstance(c, ChainHead) else "") + "_kernel" for c in calls))
         timing = "CUDA events around each GEMM launch, one region of K steps"
         for j, c in enumerate(calls):
             per_call[c.name] = {"kernel_us": call_s[j] * 1e6,

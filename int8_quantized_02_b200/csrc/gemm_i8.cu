@@ -194,7 +194,7 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-template <bool PAIR>
+template <bool PAIR, bool YBITS>
 __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensorMap &tmB,
                                           const CUtensorMap &tmXo, const CUtensorMap &tmWo,
                                           const Args &a) {
@@ -527,7 +527,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                                     y[e] = fmaf((float)(int32_t)ci[j], rs * sbv[e],
                                                 __uint_as_float(pf[j]) + b[e]);
                                 }
-                                if (a.ybits) {
+                                if (YBITS) {
                                     // |fp16(y)| >= the next threshold <=> |y| >= ytf
 #pragma unroll
                                     for (int e = 0; e < 4; ++e)
@@ -552,7 +552,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                         }
                     }
                 }
-                if (a.ybits) {
+                if (YBITS) {
                     // OR over the warp's 32 rows: one word of this 32-row block's bitmap
                     if (a.ybits_all && row_ok) ymask = groups == 2 ? 0xffffffffu : 0xffffu;
                     const uint32_t word = __reduce_or_sync(0xffffffffu, ymask);
@@ -599,21 +599,21 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
     }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-llmint8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmXo,
-                    const __grid_constant__ CUtensorMap tmWo, const Args a) {
-    gemm_body<false>(tmA, tmB, tmXo, tmWo, a);
-}
-
-// M > 128: clusters of two CTAs, 256 x 256 tiles.
-__global__ void __launch_bounds__(THREADS, 1)
-llmint8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                         const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmXo,
-                         const __grid_constant__ CUtensorMap tmWo, const Args a) {
-    gemm_body<true>(tmA, tmB, tmXo, tmWo, a);
-}
+// The kernels: single CTAs (M <= 128) or clusters of two CTAs with 256 x 256 tiles (M > 128),
+// each also in a form that writes the next layer's outlier bitmaps of Y (llmint8_linear_next_
+// bitmaps), so that the plain form carries none of that work.
+#define LLMINT8_GEMM_KERNEL(NAME, PAIR, YBITS)                                                   \
+    __global__ void __launch_bounds__(THREADS, 1)                                               \
+        NAME(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,  \
+             const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo, \
+             const Args a) {                                                                    \
+        gemm_body<PAIR, YBITS>(tmA, tmB, tmXo, tmWo, a);                                        \
+    }
+LLMINT8_GEMM_KERNEL(llmint8_gemm_kernel, false, false)
+LLMINT8_GEMM_KERNEL(llmint8_gemm_pair_kernel, true, false)
+LLMINT8_GEMM_KERNEL(llmint8_gemm_bits_kernel, false, true)
+LLMINT8_GEMM_KERNEL(llmint8_gemm_pair_bits_kernel, true, true)
+#undef LLMINT8_GEMM_KERNEL
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
@@ -668,14 +668,16 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s) {
         if (!d.attr_set) {
             err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
             if (err != cudaSuccess) return err;
-            err = cudaFuncSetAttribute(llmint8_gemm_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       smem_bytes<false>());
-            if (err != cudaSuccess) return err;
-            err = cudaFuncSetAttribute(llmint8_gemm_pair_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       smem_bytes<true>());
-            if (err != cudaSuccess) return err;
+            for (auto k : {llmint8_gemm_kernel, llmint8_gemm_bits_kernel}) {
+                err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           smem_bytes<false>());
+                if (err != cudaSuccess) return err;
+            }
+            for (auto k : {llmint8_gemm_pair_kernel, llmint8_gemm_pair_bits_kernel}) {
+                err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           smem_bytes<true>());
+                if (err != cudaSuccess) return err;
+            }
             d.attr_set = true;
         }
         sms = d.sms;
@@ -733,8 +735,9 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t s) {
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = pair ? 2 : 1;
-    err = pair ? cudaLaunchKernelEx(&cfg, llmint8_gemm_pair_kernel, tmA, tmB, tmXo, tmWo, a)
-               : cudaLaunchKernelEx(&cfg, llmint8_gemm_kernel, tmA, tmB, tmXo, tmWo, a);
+    auto kernel = pair ? (g.ybits ? llmint8_gemm_pair_bits_kernel : llmint8_gemm_pair_kernel)
+                       : (g.ybits ? llmint8_gemm_bits_kernel : llmint8_gemm_kernel);
+    err = cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmXo, tmWo, a);
     note_launches(1);
     return err != cudaSuccess ? err : cudaGetLastError();
 }
