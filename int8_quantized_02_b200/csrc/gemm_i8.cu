@@ -14,12 +14,14 @@
 // absmax vectors, the outlier part through a 16-bit product, and the two are summed in the
 // epilogue before the single rounding to fp16.
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer: k-blocks of Xq / CB (128 B of K each), then of Xo / Wo
 //               (64 fp16 of K each) - both fill the same shared-memory stages (48 KB, or
 //               32 KB per CTA of a pair, whose loads complete on the pair leader's barrier);
 //   warp 1      TMEM allocator and MMA issuer (one thread; of a pair, the leader's only);
-//   warps 2..5  epilogue: TMEM -> registers -> dequantize, add P and bias -> fp16 -> global.
+//   warps 2..9  epilogue: TMEM -> registers -> dequantize, add P and bias -> fp16 -> global;
+//               warp w reads TMEM lanes 32 * (w % 4) (the hardware's lane quadrant), and the
+//               two warps of a quadrant take the two halves of the tile's columns.
 // TMEM (512 columns): the int32 accumulator is double-buffered (2 x 256 columns) so the
 // epilogue of a tile overlaps the main loop of the next.  The outlier product P takes one of
 // two routes:
@@ -47,7 +49,10 @@ namespace {
 constexpr int BM = 128;                 // tile rows (M) held by one CTA
 constexpr int BN = 256;                 // tile columns (N)
 constexpr int BKB = 128;                // bytes of K per stage row (128 int8 or 64 fp16)
-constexpr int THREADS = 192;
+// Epilogue warps: two per TMEM lane quadrant, each taking half of the tile's columns, so
+// that two warps per scheduler share the epilogue work of a tile.
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 
 // Single CTA (PAIR = false): 128 x 256 tiles, 4 stages of 16 + 32 KB.  CTA pair: 256 x 256
 // tiles, each CTA 6 stages of 16 KB (its Xq rows) + 16 KB (its half of the weight rows).
@@ -67,7 +72,7 @@ constexpr int kRegOutliers = 16;        // outlier columns formed in the epilogu
 // [o][lane] fp32
 constexpr int SL_W_BYTES = kRegOutliers * BN * 2;
 constexpr int SL_XO_WARP = kRegOutliers * 32 * 4;
-constexpr int SL_BYTES = SL_W_BYTES + BN * 4 + BN * 4 + 4 * SL_XO_WARP;
+constexpr int SL_BYTES = SL_W_BYTES + BN * 4 + BN * 4 + EPI_WARPS * SL_XO_WARP;
 
 template <int NSTAGES>
 struct Tail {
@@ -76,7 +81,7 @@ struct Tail {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t mma_done;
-    uint64_t slice_full;                // the four epilogue warps staged the column slice
+    uint64_t slice_full;                // the epilogue warps staged the column slice
     uint64_t slice_empty;               // ... and are done reading it
     uint64_t loads_drained;             // pair, second CTA: the leader drained every load
     uint64_t peer_exit;                 // pair, leader: the second CTA made its last arrive
@@ -227,11 +232,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&tail->acc_full[s]), 1);
             // the epilogue warps of this CTA (and of the second CTA of a pair) release it
-            mbar_init(smem_addr(&tail->acc_empty[s]), PAIR ? 8 : 4);
+            mbar_init(smem_addr(&tail->acc_empty[s]), PAIR ? 2 * EPI_WARPS : EPI_WARPS);
         }
         mbar_init(smem_addr(&tail->mma_done), 1);
-        mbar_init(smem_addr(&tail->slice_full), 4);
-        mbar_init(smem_addr(&tail->slice_empty), 4);
+        mbar_init(smem_addr(&tail->slice_full), EPI_WARPS);
+        mbar_init(smem_addr(&tail->slice_empty), EPI_WARPS);
         mbar_init(smem_addr(&tail->loads_drained), 1);
         mbar_init(smem_addr(&tail->peer_exit), 1);
         tail->abort_flag = 0;
@@ -253,7 +258,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
     if (PAIR) cluster_barrier_all();
     // the quantized operands, scales and outlier list of this call are complete after this
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // No early launch_dependents: the kernel after this one (the next call's outlier scan)
+    // then starts when this grid ends instead of parking its CTAs beside the GEMM's; with
+    // eight epilogue warps that was 6 % faster on the 6.7B FFN step.
 
     // Outlier configuration of this call (uniform over the grid).
     const int n_out = (int)min((int64_t)*a.count, a.cap);
@@ -401,7 +408,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
         // ----------------------------------------------------------------- epilogue ----
         const int q = warp & 3;                        // TMEM lane quadrant of this warp
         const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-        const int wq = warp - 2;                       // this warp's quarter of the slice
+        const int wq = warp - 2;                       // this warp's share of the slice
+        constexpr int kSliceCols = BN / EPI_WARPS;      // columns it stages
+        constexpr int kChunks = BN / 32 / (EPI_WARPS / 4);   // 32-column chunks it finishes
+        const int c0 = (wq / 4) * kChunks;              // its first chunk
         int acc = 0;
         uint32_t acc_phase = 0, sl_phase = 0;
         bool first = true;
@@ -409,7 +419,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
             const int m0 = (tile % a.tiles_m) * C::TILE_M + (int)rank * BM;   // this CTA's rows
             const int n0 = (tile / a.tiles_m) * BN;
             // The tile's column slice (SCB, bias and, with few outlier columns, Wo), staged
-            // while the tensor cores still work on the tile: each warp one quarter of it,
+            // while the tensor cores still work on the tile: each warp an equal share of it,
             // after every warp is done with the previous tile's slice.
             {
                 int okq = 1;
@@ -417,7 +427,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                     okq = wait(smem_addr(&tail->slice_empty), sl_phase ^ 1) ? 1 : 0;
                 okq = __shfl_sync(0xffffffffu, okq, 0);
                 if (!okq) break;
-                for (int cc = wq * 64 + lane; cc < wq * 64 + 64; cc += 32) {
+                for (int cc = wq * kSliceCols + lane; cc < (wq + 1) * kSliceCols; cc += 32) {
                     const int n = n0 + cc;
                     const bool in = n < a.N;
                     sl_scb[cc] = in ? __ldg(a.SCB + n) : 0.0f;
@@ -467,7 +477,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = c0; c < c0 + kChunks; ++c) {
                 const int nb = n0 + c * 32;
                 if (nb >= a.N) break;
                 uint32_t ci[32], pf[32];
