@@ -86,13 +86,14 @@ outlier_scan_kernel(const __half *__restrict__ X, int64_t M, int64_t K, float th
     if (chunk < nchunks) {
         const uint4 *p = reinterpret_cast<const uint4 *>(X) + r0 * nchunks + chunk;
         int64_t r = r0;
-        for (; r + 4 <= r1; r += 4) {
-            uint4 v[4];
+        // eight rows' loads in flight before any use: the scan is bound by bytes in flight
+        for (; r + 8 <= r1; r += 8) {
+            uint4 v[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = __ldg(p + u * nchunks);
-            p += 4 * nchunks;
+            for (int u = 0; u < 8; ++u) v[u] = __ldg(p + u * nchunks);
+            p += 8 * nchunks;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 float f[8];
                 unpack8(v[u], f);
 #pragma unroll
@@ -219,24 +220,39 @@ outlier_compact_kernel(const uint32_t *__restrict__ partial, int splits, int64_t
     }
 }
 
-// The fp16 weights of the outlier columns for weight row n (one warp).
-__device__ __forceinline__ void gather_w_row(const int8_t *__restrict__ CB,
-                                             const float *__restrict__ SCB,
-                                             const __half *__restrict__ W16, int64_t n, int64_t K,
-                                             const int32_t *__restrict__ idx, int64_t n_o,
-                                             int64_t pitch, __half *__restrict__ Wo, int lane) {
+// Weight rows a gather warp takes when the outlier columns are few (at most 64): the loads of
+// all of them are issued before any use, and the gather CTAs past the first eighth have no
+// rows and exit at once.  With more columns a warp takes one row, so that there are enough
+// warps for the longer chains of loads.
+constexpr int kGatherRows = 8;
+
+// The fp16 weights of the outlier columns for weight rows n0 .. n0 + rows - 1 (one warp; lane
+// j of a pass takes outlier column j).
+__device__ __forceinline__ void gather_w_rows(const int8_t *__restrict__ CB,
+                                              const float *__restrict__ SCB,
+                                              const __half *__restrict__ W16, int64_t n0,
+                                              int rows, int64_t N, int64_t K,
+                                              const int32_t *__restrict__ idx, int64_t n_o,
+                                              int64_t pitch, __half *__restrict__ Wo, int lane) {
     const int64_t n_o64 = align_up(n_o, 64);
-    const float scb = SCB[n];
     for (int64_t j = lane; j < n_o64; j += 32) {
-        __half v = __float2half_rn(0.0f);
-        if (j < n_o) {
-            const int64_t col = idx[j];
-            if (W16 != nullptr)
-                v = W16[n * K + col];
-            else
-                v = __float2half_rn(__fdiv_rn(__fmul_rn((float)CB[n * K + col], scb), 127.0f));
+        const int64_t col = j < n_o ? idx[j] : 0;
+        __half v[kGatherRows];
+#pragma unroll
+        for (int r = 0; r < kGatherRows; ++r) {
+            const int64_t n = n0 + r;
+            v[r] = __float2half_rn(0.0f);
+            if (r < rows && j < n_o && n < N) {
+                if (W16 != nullptr)
+                    v[r] = W16[n * K + col];
+                else
+                    v[r] = __float2half_rn(
+                        __fdiv_rn(__fmul_rn((float)CB[n * K + col], SCB[n]), 127.0f));
+            }
         }
-        Wo[n * pitch + j] = v;
+#pragma unroll
+        for (int r = 0; r < kGatherRows; ++r)
+            if (r < rows && n0 + r < N) Wo[(n0 + r) * pitch + j] = v[r];
     }
 }
 
@@ -306,10 +322,13 @@ quantize_rows_kernel(const __half *__restrict__ X, int64_t M, int64_t K,
     pdl_wait_then_release();
     __shared__ uint32_t red[kThreads / 32];
     if ((int64_t)blockIdx.x >= row_ctas) {
-        const int64_t n = ((int64_t)blockIdx.x - row_ctas) * (kThreads / 32) + (threadIdx.x >> 5);
-        if (n < gw.N)
-            gather_w_row(gw.CB, gw.SCB, gw.W16, n, K, idx, min((int64_t)*count, cap), xo_pitch,
-                         gw.Wo, threadIdx.x & 31);
+        const int64_t n_o = min((int64_t)*count, cap);
+        const int rows = n_o <= 64 ? kGatherRows : 1;
+        const int64_t n0 =
+            (((int64_t)blockIdx.x - row_ctas) * (kThreads / 32) + (threadIdx.x >> 5)) * rows;
+        if (n0 < gw.N)
+            gather_w_rows(gw.CB, gw.SCB, gw.W16, n0, rows, gw.N, K, idx, n_o, xo_pitch, gw.Wo,
+                          threadIdx.x & 31);
         return;
     }
     const int tpr = 1 << tpr_log2;
@@ -511,7 +530,7 @@ cudaError_t launch_quantize_rows(const __half *X, int64_t M, int64_t K, const ui
     gw.W16 = W16;
     gw.Wo = Wo;
     gw.N = Wo != nullptr ? N : 0;
-    const int64_t gather_ctas = ceil_div(gw.N, kThreads / 32);
+    const int64_t gather_ctas = ceil_div(gw.N, kThreads / 32);   // one row per warp at most
     // threads per row: enough for kCache chunks each, 32 ... 256
     int tpr_log2 = 5;
     while (tpr_log2 < 8 && ((int64_t)kCache << tpr_log2) < K / 8) ++tpr_log2;
