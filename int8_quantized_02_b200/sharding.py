@@ -11,7 +11,10 @@ section LLM.int8() 温和总结, step 1: outliers are extracted by column from t
 state), so a rank's own rows do not decide it.  Each rank computes its rows' bitmap
 (`llmint8_outlier_bitmap`), the ranks all-gather the bitmaps (ceil(K/32) words each), and each
 rank runs the layer on its rows with the OR of all of them (`llmint8_linear_with_bitmaps`).
-Its rows of Y are then the same bytes as those rows of the unsplit layer.
+Its rows of the int8 codes and of the int32 product are then those of the unsplit layer, and
+its rows of Y are within the layer's tolerance of them: the same bytes when the same kernel
+serves both (the decode kernel at M <= 16, the GEMM otherwise), since the two kernels may
+round the last fp32 step differently.
 
 Every rank must make the same collective calls in the same order, a rank without rows too.
 The arithmetic of the layer runs in the library's kernels; this module only slices tensors
