@@ -83,3 +83,33 @@ def test_chain_bitmaps_and_second_layer(name):
     Y2_o, C2_o = oracle.linear(Y1_h, CB2_o, SCB2_o, threshold=t2, want_C=True)
     assert np.array_equal(host(C2), C2_o), f"{name}: C of the second layer"
     assert_y_close(host(Y2), Y2_o, f"{name}: Y of the second layer")
+
+
+@pytest.mark.parametrize("path", ["gemm_pair", "decode"])
+def test_next_bitmaps_at_fp16_rounding_boundaries(path):
+    """Thresholds placed on the stored values of Y1 and between them: exactly a value of |Y1|,
+    just above it, and the midpoints to the neighbouring fp16 values on either side, where a
+    threshold that compared the unrounded fp32 result (or rounded the threshold the wrong
+    way) would flag a different set.  The bitmaps must still be the oracle's set of the
+    stored fp16 Y1."""
+    M, K, N = (160, 512, 272) if path == "gemm_pair" else (8, 512, 272)
+    X = synth.activations(M, K, 2, 6.0, 20.0, 0.75, seed=77)[0]
+    W1 = synth.weight(N, K, 0.02, seed=78)
+    CB1, SCB1 = L.llmint8_quantize_weight_colwise(dev(W1))
+    Y1 = L.llmint8_linear(dev(X), CB1, SCB1, threshold=6.0, max_outliers=64)
+    a = np.sort(np.abs(host(Y1).astype(np.float32)).ravel())
+    picks = [a[int(len(a) * f)] for f in (0.9, 0.99, 0.999)] + [a[-1]]
+    for v in picks:
+        v16 = np.float16(v)
+        up = np.nextafter(v16, np.float16(np.inf))
+        down = np.nextafter(v16, np.float16(0))
+        for t in (float(v16), float(np.nextafter(np.float32(v16), np.float32(np.inf))),
+                  (float(v16) + float(up)) / 2, (float(v16) + float(down)) / 2,
+                  float(np.nextafter(np.float32((float(v16) + float(down)) / 2), np.float32(0)))):
+            if not t > 0:
+                continue
+            Y, bits = L.llmint8_linear_next_bitmaps(dev(X), CB1, SCB1, next_threshold=t,
+                                                    threshold=6.0, max_outliers=64)
+            assert np.array_equal(host(Y).view(np.uint16), host(Y1).view(np.uint16))
+            want = _expected_bitmaps(host(Y), t)
+            assert np.array_equal(host(bits).view(np.uint32), want), f"{path}: t = {t!r}"
