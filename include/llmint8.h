@@ -112,7 +112,8 @@ LLMINT8_API size_t llmint8_quantize_workspace_size(int64_t M, int64_t K);
  *   C_debug int32 [M, N] or NULL: when given, also receives the exact int8 accumulators C.
  * Kernels (int8 codes, outlier columns and C do not depend on the choice; Y may differ in
  * the last fp32 rounding): M <= 16, K <= 16384, threshold > 0 and max_outliers <= 256 run one
- * weight-streaming tcgen05 kernel whose CTAs each quantize X themselves.  Other shapes run
+ * kernel whose first CTAs quantize X (each a slice of the columns) while the others stream
+ * the weight through tcgen05 MMAs.  Other shapes run
  * outlier detection, row quantization (with the gather of the outlier weight rows) and a
  * persistent tcgen05 GEMM, on CTA pairs when M > 128.  Kernels of a call are launched as
  * programmatic dependents: each may start while the work before it on the stream finishes,

@@ -135,7 +135,7 @@ def test_proj175b_full_size():
 
 @pytest.mark.parametrize("batch", [1, 16])
 def test_decode175b_full_size(batch):
-    # decode at the 175B-class projection shape (K = 12288 past the 8192 of the decode
+    # decode at the 175B-class projection shape (K = 12288, three times the K of the decode
     # workload, N = 49152): the single-kernel decode path, output compared in full
     _check(synth.decode175b(batch), 6.0, 64)
 
