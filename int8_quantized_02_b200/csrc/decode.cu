@@ -3,30 +3,33 @@
 // At decode sizes the layer is bound by streaming the int8 weight CB from HBM once; the rest
 // must hide under that stream.  One kernel per call, one CTA per SM:
 //
-//   CTA 0, the quantizer: waits for the previous grid on the stream (X may be its output),
-//       reads X once and finds the outlier columns (|x| >= threshold in any row, an OR over
-//       the lanes holding a column's rows) and the row maxima over the regular columns,
-//       lists the outlier columns in ascending order and publishes that table (row absmax,
-//       per-chunk outlier bits, the list) in the workspace with a release store of the call
-//       number; then it exits, so the next call's quantizer can take its SM early.
-//   CTAs 1.., the streamers, each own a band of Rt consecutive weight rows (output channels);
-//       Rt = ceil(N / streamers) rounded up to 8 rows (at most 128), so the bands spread
-//       evenly over every SM and no streamer waits on another:
-//     warp 0      TMA producer: 128-byte k-blocks of the band through a shared-memory ring;
-//     warps 2, 3  wait for the table, then write the int8 codes of X (absmax quantization with
-//                 the published row scales, outlier columns 0) one k-block at a time into a
-//                 small ring of operand images (K-major, 128-byte swizzle), in the order the
-//                 MMAs consume them, re-reading that block of X from L2;
-//     warp 1      one thread issues tcgen05.mma kind::i8 with the weight rows as the 128-row
-//                 operand and the image block as the 16-column operand, D[n, m] = sum_k
-//                 CB[n, k] Xq[m, k], into int32 TMEM sub-accumulators;
-//     warps 4..7  epilogue: while the weights stream, each thread (one output channel n)
-//                 forms the fp16 outlier part sum_{j in O} X[m, O_j] * W_o[n, O_j] + bias_n and
-//                 its scale; after the last MMA: y = D * SCA_m * SCB_n / 127^2 + that part.
-// Every loop is rolled (the SM fetches little code while the weight stream keeps the memory
-// system busy), and the operand image is never held whole, so K is not bound by shared
-// memory.  Same method and rounding as the GEMM path (LLM.int8() summary, sections
-// الابتكار الثاني and الصورة الكاملة; blog sections MatMul 内部 and 用法).  Every wait is bounded.
+//   CTAs 0 .. nq-1, the quantizers (nq <= 8): each waits for the previous grid on the stream
+//       (X may be its output) and owns a slice of k-blocks.  It copies its columns of X to
+//       shared memory, finds their outlier bits (|x| >= threshold in any row) and, per row, the
+//       maximum of |x| over its regular columns, and publishes those maxima and its outlier
+//       count as call-tagged words.  Reading every quantizer's words gives it the row scales of
+//       the whole layer and its place in the ascending outlier list; it writes the int8 codes
+//       of its slice as a block of the operand image (K-major, 128-byte swizzle, the layout of
+//       the MMA's B operand in shared memory), stores it to the workspace with one bulk copy,
+//       lists its outlier columns and releases done[q] with the call number.
+//   CTAs nq.., the streamers, each own bands of Rt consecutive weight rows (output channels);
+//       Rt = ceil(N / streamers) rounded up to 8 rows (at most 128), so the bands spread evenly
+//       over every SM and no streamer waits on another:
+//     warp 0      TMA producer: 2-k-block stages of the band through a shared-memory ring, at
+//                 most `inflight` on their way, issued before the quantizers finish;
+//     warp 2      once every done[q] holds the call number, copies the image blocks into
+//                 shared memory with bulk copies (once when they all fit, else through a ring);
+//     warps 1, 3  one thread each issues tcgen05.mma kind::i8 with the weight rows as the
+//                 128-row operand and an image block as the 16-column operand, D[n, m] = sum_k
+//                 CB[n, k] Xq[m, k], into its own int32 TMEM accumulator (alternate stages);
+//     warps 4..7  epilogue: while the weights stream, each thread (one output channel n) forms
+//                 the fp16 outlier part sum_{j in O} X[m, O_j] * W_o[n, O_j] + bias_n and its
+//                 scale; after the last MMA: y = D * SCA_m * SCB_n / 127^2 + that part, and
+//                 with a next threshold the outlier bitmap of Y for the next layer.
+// Loops are rolled (little code to fetch while the weight stream keeps the memory system
+// busy), and K is bound by the quantizers' slices, not by shared memory.  Same method and
+// rounding as the GEMM path (LLM.int8() summary, sections الابتكار الثاني and الصورة الكاملة;
+// blog sections MatMul 内部 and 用法).  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include <cstddef>
@@ -177,9 +180,10 @@ struct DArgs {
     const uint32_t *bitmaps;             // [n_bitmaps][ceil(K/32)] given outlier set, or null
     int n_bitmaps;
     uint32_t *ybits;                     // [ceil(N/32)] outlier bitmap of Y for the next
-                                         // layer, or null (zeroed by quantizer 0)
+                                         // layer, or null
     float ytf;                           // its threshold on the fp32 value
     int ybits_all;                       // threshold <= 0: every column
+    int ncols32;                         // 32 * ceil(N / 32): the columns the bitmap covers
     int32_t *count;
     DecodeTable *table;                  // workspace: what the quantizer publishes
     uint8_t *image;                      // workspace: the int8 operand image, block by block
@@ -478,9 +482,6 @@ __device__ void quantize_x(const DArgs &a, uint8_t *smem) {
         }
     }
     if (qi == 0) {
-        // the streamers OR their columns into Y's bitmap only after they acquire done[0]
-        if (a.ybits)
-            for (int i = threadIdx.x; i < (a.N + 31) / 32; i += DTHREADS) a.ybits[i] = 0u;
         if (threadIdx.x < DM) a.table->sca[threadIdx.x] = q->sca[threadIdx.x];
         if (threadIdx.x == DM) {
             const int total = q->total;
@@ -816,13 +817,23 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 }
             }
             if (a.ybits) {
-                // this warp's 32 consecutive columns, ORed into the one or two words they
-                // straddle (bands need not start on a multiple of 32)
+                // this warp's columns of the band (and any past N, which read as 0) are its own
+                // bits of the one or two words they straddle (bands need not start on a
+                // multiple of 32): clear those to be 0, then set those to be 1, so the bitmap
+                // needs no clearing first and the other bits of a shared word are untouched
                 const uint32_t bal = __ballot_sync(0xffffffffu, yflag);
+                const uint32_t own = __ballot_sync(0xffffffffu, (live || n >= a.N) && n < a.ncols32);
                 const int c0 = tile * a.Rt + qd * 32, sh = c0 & 31;
-                if (lane == 0 && bal) {
-                    atomicOr(a.ybits + (c0 >> 5), bal << sh);
-                    if (sh && (bal >> (32 - sh))) atomicOr(a.ybits + (c0 >> 5) + 1, bal >> (32 - sh));
+                if (lane == 0 && own) {
+                    uint32_t *w0 = a.ybits + (c0 >> 5);
+                    if (own << sh) {
+                        atomicAnd(w0, ~((own & ~bal) << sh));
+                        if (bal << sh) atomicOr(w0, bal << sh);
+                    }
+                    if (sh && (own >> (32 - sh))) {
+                        atomicAnd(w0 + 1, ~((own & ~bal) >> (32 - sh)));
+                        if (bal >> (32 - sh)) atomicOr(w0 + 1, bal >> (32 - sh));
+                    }
                 }
             }
         }
@@ -925,6 +936,7 @@ cudaError_t launch_decode(const DecodeLaunch &d, cudaStream_t s) {
     a.ybits = d.ybits;
     a.ytf = d.ybits && d.ythreshold > 0.0f ? fp16_rounded_threshold_f32(d.ythreshold) : 0.0f;
     a.ybits_all = d.ybits && d.ythreshold <= 0.0f ? 1 : 0;
+    a.ncols32 = (int)(ceil_div(d.N, 32) * 32);
     a.count = d.count;
     a.table = d.table;
     a.image = d.image;

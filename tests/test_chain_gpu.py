@@ -113,3 +113,24 @@ def test_next_bitmaps_at_fp16_rounding_boundaries(path):
             assert np.array_equal(host(Y).view(np.uint16), host(Y1).view(np.uint16))
             want = _expected_bitmaps(host(Y), t)
             assert np.array_equal(host(bits).view(np.uint32), want), f"{path}: t = {t!r}"
+
+
+@pytest.mark.parametrize("path", ["gemm_pair", "gemm_single", "decode_k1024", "decode_k8192"])
+def test_next_bitmaps_overwrite_a_dirty_buffer(path):
+    """The bitmaps of Y are written whole, padding bits past N included: a buffer that holds
+    all ones, or another call's bitmaps, ends up equal to the oracle's set either way."""
+    M, K = {"gemm_pair": (160, 512), "gemm_single": (96, 512), "decode_k1024": (5, 1024),
+            "decode_k8192": (5, 8192)}[path]
+    N = 1040                                      # not a multiple of 32: a padded last word
+    X = synth.activations(M, K, 2, 6.0, 20.0, 0.75, seed=91)[0]
+    W1 = synth.weight(N, K, 0.02, seed=92)
+    CB1, SCB1 = L.llmint8_quantize_weight_colwise(dev(W1))
+    shape = ((M + 31) // 32, (N + 31) // 32)
+    for t, fill in ((2.0, -1), (1.0, -1), (3.0, None)):
+        bits = torch.full(shape, -1, dtype=torch.int32, device="cuda") if fill is not None \
+            else bits                               # the previous call's bitmaps
+        Y, bits = L.llmint8_linear_next_bitmaps(dev(X), CB1, SCB1, next_threshold=t,
+                                                threshold=6.0, max_outliers=64,
+                                                next_bitmaps=bits)
+        want = _expected_bitmaps(host(Y), t)
+        assert np.array_equal(host(bits).view(np.uint32), want), f"{path}: t = {t}"
