@@ -99,8 +99,9 @@ __device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
     return *reinterpret_cast<const uint32_t *>(&r);
 }
 
-// A threshold t > 0 as the smallest fp16 >= t, in both halves of a word: for an fp16 x,
-// |x| >= t exactly when |x| >= that value (fp16 compares, packed two at a time).
+// A threshold t as the smallest fp16 >= t, in both halves of a word: for an fp16 x,
+// |x| >= t exactly when |x| >= that value (fp16 compares, packed two at a time), for every t
+// (zero, negative and past the fp16 range included; a NaN x compares false either way).
 inline uint32_t fp16_threshold_pair(float t) {
     const __half t16 = __float2half_ru(t);
     const uint32_t tb = (uint32_t)*reinterpret_cast<const uint16_t *>(&t16);

@@ -530,7 +530,9 @@ cudaError_t launch_quantize_rows(const __half *X, int64_t M, int64_t K, const ui
     gw.W16 = W16;
     gw.Wo = Wo;
     gw.N = Wo != nullptr ? N : 0;
-    const int64_t gather_ctas = ceil_div(gw.N, kThreads / 32);   // one row per warp at most
+    // one weight row per warp, or kGatherRows when the outlier count cannot pass 64 (the
+    // kernel takes kGatherRows whenever the count it reads is at most 64)
+    const int64_t gather_ctas = ceil_div(gw.N, (int64_t)(kThreads / 32) * (cap <= 64 ? kGatherRows : 1));
     // threads per row: enough for kCache chunks each, 32 ... 256
     int tpr_log2 = 5;
     while (tpr_log2 < 8 && ((int64_t)kCache << tpr_log2) < K / 8) ++tpr_log2;

@@ -81,6 +81,19 @@ def _quantize_cases():
     X[5] = 7.0                       # a row that is outlier-only
     yield "planted", X, 6.0
     yield "wide_K", _x(4, 20000 // 16 * 16, 5, seed=8), 6.0
+    # thresholds that are not fp16 values: the kernels compare fp16 |x| with the smallest fp16
+    # at or above t, which must flag exactly the entries with |x| >= t
+    X = _x(8, 64, 0, seed=10)
+    X[0, 3] = 6.0                              # below t
+    X[1, 7] = np.float16(6.00390625)           # the next fp16 above 6: at least t
+    X[2, 11] = -np.float16(6.00390625)
+    X[3, 20] = np.float16(6.0) * -1
+    yield "t_between_fp16_values", X, 6.001
+    yield "negative_t_every_column", _x(9, 128, 0, seed=11), -1.0
+    X = _x(6, 96, 0, seed=12)
+    X[2, 40] = np.inf                          # only an infinity reaches t past the fp16 range
+    X[4, 41] = np.float16(65504.0)
+    yield "t_past_fp16_max", X, 70000.0
 
 
 @pytest.mark.parametrize("name,X,t", list(_quantize_cases()), ids=lambda v: v if isinstance(v, str) else "")
