@@ -3,7 +3,10 @@
 #include <math.h>
 #include <string.h>
 
+#include <unistd.h>
+
 #include <atomic>
+#include <chrono>
 #include <mutex>
 
 #include <nvtx3/nvToolsExt.h>
@@ -43,7 +46,18 @@ class CallRange {
 constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<uint64_t> g_launches{0};
-std::atomic<unsigned long long> g_epoch{1};   // one per call that writes a status word
+// The first call number of this process: in [1, 2^31), mixed from the clock and the process
+// id, so that call-tagged words another process left in the same device memory (workspaces are
+// not cleared) are unlikely to carry a number this process uses.
+unsigned long long first_epoch() {
+    unsigned long long x = (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+    x ^= (unsigned long long)getpid() * 0x9e3779b97f4a7c15ull;
+    x ^= x >> 29;
+    x *= 0xbf58476d1ce4e5b9ull;
+    x ^= x >> 32;
+    return 1ull + (x & 0x7ffffffeull);
+}
+std::atomic<unsigned long long> g_epoch{first_epoch()};   // one per call that writes a status word
 
 StatusRef next_status(WsHeader *h) {
     return StatusRef{&h->status, &h->timeout, g_epoch.fetch_add(1) << 4};
@@ -518,7 +532,7 @@ llmint8_status llmint8_device_status(const void *ws, void *stream) {
     unsigned long long words[2] = {0, 0};   // status, timeout
     if (cudaMemcpy(words, ws, sizeof(words), cudaMemcpyDeviceToHost) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    // epochs start at 1: a zero-filled header has recorded no call and no timeout
+    // epochs are never 0: a zero-filled header has recorded no call and no timeout
     if ((words[0] >> 4) != 0 && (words[1] >> 4) == (words[0] >> 4))
         return static_cast<llmint8_status>(words[1] & 0xFull);
     return static_cast<llmint8_status>(words[0] & 0xFull);

@@ -180,6 +180,11 @@ LINEAR_CASES = {
     "outliers_64_tensor_cores_single": (100, 4096, 272, 64, 6.0, False, False),
     "outliers_65_tensor_cores": (200, 8192, 272, 65, 6.0, True, False),
     "K32_half_outliers": (40, 32, 64, 16, 6.0, False, False),
+    # more CTA-pair tiles (80) than pairs on a B200 (74): a second, partly idle wave (ragged M,
+    # N, K; two k-blocks a tile; the tensor-core outlier product)
+    "pair_tiles_80": (300, 1040, 10000, 3, 6.0, True, False),
+    "pair_tiles_80_two_kblocks": (512, 256, 10240, 0, 6.0, False, False),
+    "pair_tiles_80_outliers_20": (300, 1040, 10000, 20, 6.0, True, False),
 }
 
 
