@@ -51,7 +51,10 @@ constexpr int DKS = 2;                  // k-blocks per weight stage (one wait, 
 constexpr int DMAX_STAGES = 32;
 constexpr int DIMG_MAX = 32;            // operand-image stages at most ...
 constexpr int DIMG_BYTES = 65536;       // ... and the shared memory they take at most
-constexpr int QKB = 4;                  // k-blocks per quantizer CTA (aim)
+// k-blocks per quantizer CTA (aim).  Each quantizer phase is bound by latency, not by its
+// slice's size, so fewer quantizers mean fewer partials to exchange and more streamers: at
+// K = 4096, 4 quantizers (8 k-blocks each) beat 2, 3, 5 and 8 at every batch size measured.
+constexpr int QKB = 8;
 constexpr int DINFLIGHT = 3;            // weight stages a streamer keeps on their way
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
 // Two MMA issuers per CTA (warps 1 and 3): issuer i takes the weight stages j with
