@@ -55,7 +55,9 @@ constexpr int DIMG_BYTES = 65536;       // ... and the shared memory they take a
 // slice's size, so fewer quantizers mean fewer partials to exchange and more streamers: at
 // K = 4096, 4 quantizers (8 k-blocks each) beat 2, 3, 5 and 8 at every batch size measured.
 constexpr int QKB = 8;
-constexpr int DINFLIGHT = 3;            // weight stages a streamer keeps on their way
+// Weight stages a streamer keeps on their way: a short queue keeps the quantizers' latency-bound
+// chain fast (1 stage starves the stream, 3 or 5 slow the chain; 2 measured best).
+constexpr int DINFLIGHT = 2;
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
 // Two MMA issuers per CTA (warps 1 and 3): issuer i takes the weight stages j with
 // j % 2 == i of every tile, into its own int32 accumulator of 16 columns; the epilogue adds the
