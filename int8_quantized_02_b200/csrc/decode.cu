@@ -168,6 +168,7 @@ struct DTail {
     uint64_t tbar;                       // the quantizer's table is published (one poller)
     uint32_t tmem_base;
     int abort_flag;
+    int streaming;                       // the MMAs run: the producer may keep more in flight
     int32_t idx[kDecodeMaxOutliers];     // outlier columns, ascending (epilogue copy)
 };
 static_assert(offsetof(DTail, acc_full) % 8 == 0, "mbarriers are 8-byte aligned");
@@ -549,6 +550,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
         }
         mbar_init(smem_addr(&tail->tbar), 1);
         tail->abort_flag = 0;
+        tail->streaming = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmCB);
     }
@@ -580,10 +582,14 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                     int sj = j + rot;
                     if (sj >= a.nst) sj -= a.nst;
                     const int kb0 = sj * DKS, nkb = min(DKS, a.kblocks - kb0);
-                    // at most `inflight` stages on their way: a short memory queue keeps the
-                    // latency of everything else on the GPU (X, the tables, the image) low
-                    if (issued >= a.inflight) {
-                        const int prev = issued - a.inflight;
+                    // at most `inflight` stages on their way while X is quantized: a short
+                    // memory queue keeps the latency of everything else on the GPU (X, the
+                    // tables, the image) low; once the MMAs run, up to four (fewer than the
+                    // ring's stages, so the stage waited on is still that use's)
+                    const int depth = *reinterpret_cast<volatile int *>(&tail->streaming)
+                                          ? min(4, S - 1) : a.inflight;
+                    if (issued >= depth) {
+                        const int prev = issued - depth;
                         if (!wait(smem_addr(&tail->full[prev % S]), (uint32_t)(prev / S) & 1u))
                             goto drain;
                     }
@@ -639,6 +645,7 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                         good = false;
                         break;
                     }
+                    if (issuer == 0) *reinterpret_cast<volatile int *>(&tail->streaming) = 1;
                     tc_fence_after();
                     for (int h = 0; h < nkb; ++h) {
                         const uint32_t sa = ring_base + (uint32_t)stage * stage_bytes + h * kbox;
