@@ -315,6 +315,17 @@ def build_workload(name, L, torch):
     return calls, unit, metric_bound
 
 
+def int8_peak_kind(clocks):
+    """Which measured bf16 figure a prefill line is judged against: its repeated regions keep
+    the tensor cores busy for about half a second, and when their clock record shows the
+    power cap (or SM clocks below 95 % of the maximum) the kernels ran in the sustained
+    regime; otherwise the burst figure.  Returns (peaks key, capped)."""
+    capped = "sw_power_cap" in clocks.get("reasons", []) or bool(
+        clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
+        and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
+    return ("bf16_tflops_sustained" if capped else "bf16_tflops"), capped
+
+
 def unit_value(units, seconds, unit):
     return units / seconds / 1e9 if unit == "GB/s" else units / seconds / 1e12
 
@@ -462,15 +473,8 @@ def run_workload(name, args, rank, world, local_rank):
                                      for s_ in range(args.steps)) / 1e3 / args.steps,
                                  world, device="cuda") for j in range(len(calls))]
         achieved = step_units / sum(call_s) / 1e12
-        # int8 = 2 x bf16 (the nominal dense ratio).  The repeated regions keep the tensor
-        # cores busy for about half a second: when the clock record shows the power cap (or
-        # SM clocks well below their maximum) the kernels ran in the sustained regime, whose
-        # measured bf16 figure is then the denominator; otherwise the burst figure.
-        ck = clk.summary()
-        capped = "sw_power_cap" in ck.get("reasons", []) or (
-            ck.get("sm_mhz") and ck.get("sm_max_mhz") and ck["sm_mhz"] < 0.95 * ck["sm_max_mhz"])
-        peak_kind = "bf16_tflops_sustained" if capped else "bf16_tflops"
-        peak, roof_unit = 2.0 * peaks[peak_kind], "TOPS"
+        peak_kind, capped = int8_peak_kind(clk.summary())
+        peak, roof_unit = 2.0 * peaks[peak_kind], "TOPS"   # int8 = 2 x bf16 (nominal ratio)
         burst_peak = 2.0 * peaks["bf16_tflops"]
         kernel_name = ", ".join(dict.fromkeys(
             ("llmint8_gemm_pair" if c.M > 128 else "llmint8_gemm")

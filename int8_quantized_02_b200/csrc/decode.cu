@@ -16,7 +16,8 @@
 //       Rt = ceil(N / streamers) rounded up to 8 rows (at most 128), so the bands spread evenly
 //       over every SM and no streamer waits on another:
 //     warp 0      TMA producer: 2-k-block stages of the band through a shared-memory ring, at
-//                 most `inflight` on their way, issued before the quantizers finish;
+//                 most two on their way while X is quantized (a short queue keeps the
+//                 quantizers' latency-bound chain fast) and up to four once the MMAs run;
 //     warp 2      once every done[q] holds the call number, copies the image blocks into
 //                 shared memory with bulk copies (once when they all fit, else through a ring);
 //     warps 1, 3  one thread each issues tcgen05.mma kind::i8 with the weight rows as the

@@ -1,5 +1,6 @@
 """bench.py's host-side rules, on the CPU: the peaks fall back to the stated figures without a
-measured-peaks file, and the repeat count and spread of the repeated timed region."""
+measured-peaks file, the prefill peak follows the clock record, and the repeat count and
+spread of the repeated timed region."""
 from __future__ import annotations
 
 import os
@@ -43,3 +44,16 @@ def test_spread():
     assert s["p10"] == 1.0 and s["p90"] == 5.0
     s = bench.spread([float(i) for i in range(101)])
     assert s["p10"] == 10.0 and s["p90"] == 90.0 and s["median"] == 50.0
+
+
+def test_int8_peak_follows_the_clock_record():
+    assert bench.int8_peak_kind({"sm_mhz": 1780, "sm_max_mhz": 1965,
+                                 "reasons": ["sw_power_cap"]}) == ("bf16_tflops_sustained", True)
+    # clocks held well below the maximum with no reason recorded: not the burst regime either
+    assert bench.int8_peak_kind({"sm_mhz": 1500, "sm_max_mhz": 1965, "reasons": []})[0] == \
+        "bf16_tflops_sustained"
+    assert bench.int8_peak_kind({"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}) == \
+        ("bf16_tflops", False)
+    # no NVML: no evidence of a cap
+    assert bench.int8_peak_kind({"sm_mhz": None, "sm_max_mhz": None, "reasons": []}) == \
+        ("bf16_tflops", False)
