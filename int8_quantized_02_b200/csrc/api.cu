@@ -50,7 +50,8 @@ std::atomic<uint64_t> g_launches{0};
 // id, so that call-tagged words another process left in the same device memory (workspaces are
 // not cleared) are unlikely to carry a number this process uses.
 unsigned long long first_epoch() {
-    unsigned long long x = (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+    unsigned long long x =
+        (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
     x ^= (unsigned long long)getpid() * 0x9e3779b97f4a7c15ull;
     x ^= x >> 29;
     x *= 0xbf58476d1ce4e5b9ull;

@@ -835,7 +835,8 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                 // multiple of 32): clear those to be 0, then set those to be 1, so the bitmap
                 // needs no clearing first and the other bits of a shared word are untouched
                 const uint32_t bal = __ballot_sync(0xffffffffu, yflag);
-                const uint32_t own = __ballot_sync(0xffffffffu, (live || n >= a.N) && n < a.ncols32);
+                const uint32_t own =
+                    __ballot_sync(0xffffffffu, (live || n >= a.N) && n < a.ncols32);
                 const int c0 = tile * a.Rt + qd * 32, sh = c0 & 31;
                 if (lane == 0 && own) {
                     uint32_t *w0 = a.ybits + (c0 >> 5);

@@ -532,7 +532,8 @@ cudaError_t launch_quantize_rows(const __half *X, int64_t M, int64_t K, const ui
     gw.N = Wo != nullptr ? N : 0;
     // one weight row per warp, or kGatherRows when the outlier count cannot pass 64 (the
     // kernel takes kGatherRows whenever the count it reads is at most 64)
-    const int64_t gather_ctas = ceil_div(gw.N, (int64_t)(kThreads / 32) * (cap <= 64 ? kGatherRows : 1));
+    const int64_t rows_per_warp = cap <= 64 ? kGatherRows : 1;
+    const int64_t gather_ctas = ceil_div(gw.N, (int64_t)(kThreads / 32) * rows_per_warp);
     // threads per row: enough for kCache chunks each, 32 ... 256
     int tpr_log2 = 5;
     while (tpr_log2 < 8 && ((int64_t)kCache << tpr_log2) < K / 8) ++tpr_log2;
