@@ -144,8 +144,9 @@ LLMINT8_API size_t llmint8_linear_workspace_size(int64_t M, int64_t N, int64_t K
  *                   |Y[m, n]| >= next_threshold, Y as stored (fp16).  Give them to the next
  *                   layer's llmint8_linear_with_bitmaps with n_bitmaps = ceil(M/32).
  * The GEMM path forms each word in the epilogue that writes those values of Y (an OR over a
- * warp's 32 rows; no atomics); the decode path ORs each warp's 32 output columns into the
- * words, which its kernel zeroes first.
+ * warp's 32 rows; no atomics); on the decode path each warp owns its output columns' bits of
+ * the words they straddle (and the bits past N) and writes them with an atomic AND, then an
+ * atomic OR, so nothing needs clearing first.
  */
 LLMINT8_API llmint8_status llmint8_linear_next_bitmaps(const uint16_t *X, int64_t M, int64_t K,
                                            const int8_t *CB, const float *SCB, int64_t N,
