@@ -849,6 +849,10 @@ llmint8_decode_kernel(const __grid_constant__ CUtensorMap tmCB, const DArgs a) {
                         if (bal >> (32 - sh)) atomicOr(w0 + 1, bal >> (32 - sh));
                     }
                 }
+                // the last word's bits past N, which no band's lanes may reach when the bands
+                // are wide: no one sets them, so one AND clears them
+                if (tile == a.tiles - 1 && qd == 0 && lane == 0 && (a.N & 31))
+                    atomicAnd(a.ybits + (a.N >> 5), (1u << (a.N & 31)) - 1u);
             }
         }
     }

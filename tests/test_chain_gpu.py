@@ -115,13 +115,16 @@ def test_next_bitmaps_at_fp16_rounding_boundaries(path):
             assert np.array_equal(host(bits).view(np.uint32), want), f"{path}: t = {t!r}"
 
 
-@pytest.mark.parametrize("path", ["gemm_pair", "gemm_single", "decode_k1024", "decode_k8192"])
+@pytest.mark.parametrize("path", ["gemm_pair", "gemm_single", "decode_k1024", "decode_k8192",
+                                  "decode_wide_bands"])
 def test_next_bitmaps_overwrite_a_dirty_buffer(path):
     """The bitmaps of Y are written whole, padding bits past N included: a buffer that holds
-    all ones, or another call's bitmaps, ends up equal to the oracle's set either way."""
-    M, K = {"gemm_pair": (160, 512), "gemm_single": (96, 512), "decode_k1024": (5, 1024),
-            "decode_k8192": (5, 8192)}[path]
-    N = 1040                                      # not a multiple of 32: a padded last word
+    all ones, or another call's bitmaps, ends up equal to the oracle's set either way.  N is
+    not a multiple of 32 (a padded last word); with N = 16560 the decode bands are 120 rows
+    wide and no band's lanes reach the last word's padding bits."""
+    M, K, N = {"gemm_pair": (160, 512, 1040), "gemm_single": (96, 512, 1040),
+               "decode_k1024": (5, 1024, 1040), "decode_k8192": (5, 8192, 1040),
+               "decode_wide_bands": (1, 1024, 16560)}[path]
     X = synth.activations(M, K, 2, 6.0, 20.0, 0.75, seed=91)[0]
     W1 = synth.weight(N, K, 0.02, seed=92)
     CB1, SCB1 = L.llmint8_quantize_weight_colwise(dev(W1))
